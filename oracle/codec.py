@@ -1,0 +1,217 @@
+"""ctypes front end of the C oracle codec (``nf4_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
+Pages followed:
+  "LoRA 与 QLoRA" (whoami-wesleyyou.top), QLoRA sections "1. NF4" and
+  "2. Double Quantization (DQ)";
+  "QLoRA: Efficient Finetuning of Quantized LLMs" deck "3 QLoRA Finetuning"
+  (learn.ifs.name), cards 1-4;
+  jjjymmm.cn 2024/03 QLoRA post, sections "4-bit NormalFloat(NF4)",
+  "Double Quantization" and "QLoRA".
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+#: Offset of the outermost quantile.  The pages do not print it; the printed
+#: NF4 table (jjjymmm.cn, "4-bit NormalFloat(NF4)") pins it to [0.96768,
+#: 0.96773].  This closed form, halfway between the half-bin offsets of 16 and
+#: 15 equal-mass bins, lies in that window.
+DELTA = 1.0 - 0.5 * (1.0 / 32.0 + 1.0 / 30.0)
+
+BLOCK = 64        # weights per absmax block ("LoRA 与 QLoRA", DQ: 64 weights)
+DQ_GROUP = 256    # block constants per DQ scale (deck card 4; jjjymmm.cn DQ)
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(_build.build())
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        L.oracle_normal_cdf.restype = ctypes.c_double
+        L.oracle_normal_cdf.argtypes = [ctypes.c_double]
+        L.oracle_normal_quantile.restype = ctypes.c_double
+        L.oracle_normal_quantile.argtypes = [ctypes.c_double]
+        L.oracle_nf4_codebook.restype = None
+        L.oracle_nf4_codebook.argtypes = [ctypes.c_double, P, P]
+        L.oracle_nf4_nearest.restype = ctypes.c_int
+        L.oracle_nf4_nearest.argtypes = [ctypes.c_float, P]
+        L.oracle_nf4_quantize.restype = None
+        L.oracle_nf4_quantize.argtypes = [P, I64, P, P, P]
+        L.oracle_pairwise_sum.restype = ctypes.c_double
+        L.oracle_pairwise_sum.argtypes = [P, I64]
+        L.oracle_dq_mean.restype = ctypes.c_float
+        L.oracle_dq_mean.argtypes = [P, I64]
+        L.oracle_nf4_double_quant.restype = None
+        L.oracle_nf4_double_quant.argtypes = [P, I64, P, P, P]
+        L.oracle_dq_restore.restype = ctypes.c_float
+        L.oracle_dq_restore.argtypes = [ctypes.c_int8, ctypes.c_float, ctypes.c_float]
+        L.oracle_bf16_rn.restype = ctypes.c_uint16
+        L.oracle_bf16_rn.argtypes = [ctypes.c_float]
+        L.oracle_nf4_dequant.restype = None
+        L.oracle_nf4_dequant.argtypes = [P, I64, P, P, P, P, P, P]
+        L.oracle_nf4_dequant_f32.restype = None
+        L.oracle_nf4_dequant_f32.argtypes = [P, I64, P, P, P, P, P, P]
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def normal_quantile(p: float) -> float:
+    """Q_Z(p) of N(0,1) by bisection ("LoRA 与 QLoRA", Gaussian 假设与分位数)."""
+    return lib().oracle_normal_quantile(float(p))
+
+
+def normal_cdf(x: float) -> float:
+    return lib().oracle_normal_cdf(float(x))
+
+
+def codebook(delta: float = DELTA):
+    """The 16 NF4 values, ascending: (float64 array, float32 array).
+
+    Asymmetric halves sharing one zero (deck card 3), normalized by the largest
+    quantile so the ends are exactly +-1 ("LoRA 与 QLoRA", 归一化与匹配)."""
+    c64 = np.zeros(16, np.float64)
+    c32 = np.zeros(16, np.float32)
+    lib().oracle_nf4_codebook(float(delta), _ptr(c64), _ptr(c32))
+    return c64, c32
+
+
+_CB32 = None
+
+
+def cb32():
+    global _CB32
+    if _CB32 is None:
+        _CB32 = codebook()[1]
+    return _CB32
+
+
+def nearest(x: float, cb=None) -> int:
+    cb = cb32() if cb is None else _c(cb, np.float32)
+    return lib().oracle_nf4_nearest(ctypes.c_float(x), _ptr(cb))
+
+
+def quantize(w):
+    """fp32 weights (any shape, numel % 64 == 0, flattened row-major) ->
+    (codes uint8 [numel/2], absmax fp32 [numel/64]).
+
+    jjjymmm.cn "4-bit NormalFloat(NF4)": divide by the block ABSMAX, take the
+    nearest quant-book value; "LoRA 与 QLoRA" DQ: one constant per 64 weights."""
+    w = _c(w, np.float32).reshape(-1)
+    n = w.size
+    if n % BLOCK:
+        raise ValueError("numel must be a multiple of 64")
+    codes = np.zeros(n // 2, np.uint8)
+    absmax = np.zeros(n // BLOCK, np.float32)
+    cb = cb32()
+    lib().oracle_nf4_quantize(_ptr(w), n, _ptr(cb), _ptr(codes), _ptr(absmax))
+    return codes, absmax
+
+
+def pairwise_sum(a) -> float:
+    a = _c(a, np.float32).reshape(-1)
+    return lib().oracle_pairwise_sum(_ptr(a), a.size)
+
+
+def dq_mean(absmax) -> np.float32:
+    a = _c(absmax, np.float32).reshape(-1)
+    return np.float32(lib().oracle_dq_mean(_ptr(a), a.size))
+
+
+def double_quant(absmax):
+    """fp32 block constants -> (qabs int8 [nb], scale fp32 [ceil(nb/256)], mu fp32).
+
+    "LoRA 与 QLoRA" DQ: r_j = (a_j - mu)/b, 8-bit rhat_j, mu and b in 32 bits;
+    deck card 4 / jjjymmm.cn DQ: blocks of 256 constants."""
+    a = _c(absmax, np.float32).reshape(-1)
+    nb = a.size
+    ng = (nb + DQ_GROUP - 1) // DQ_GROUP
+    qabs = np.zeros(nb, np.int8)
+    scale = np.zeros(ng, np.float32)
+    mu = np.zeros(1, np.float32)
+    lib().oracle_nf4_double_quant(_ptr(a), nb, _ptr(qabs), _ptr(scale), _ptr(mu))
+    return qabs, scale, mu[0]
+
+
+def dq_restore(qabs, scale, mu):
+    """ahat_j = fp32(mu + fp32(b_g * rhat_j)) for every j (vector form)."""
+    qabs = _c(qabs, np.int8).reshape(-1)
+    scale = _c(scale, np.float32).reshape(-1)
+    out = np.empty(qabs.size, np.float32)
+    L = lib()
+    for j in range(qabs.size):
+        out[j] = L.oracle_dq_restore(int(qabs[j]), float(scale[j // DQ_GROUP]), float(mu))
+    return out
+
+
+def bf16_rn(x: float) -> int:
+    return lib().oracle_bf16_rn(ctypes.c_float(x))
+
+
+def dequant(codes, numel, absmax=None, qabs=None, scale=None, mu=None):
+    """doubleDequant to BF16 bits (uint16 [numel]).
+
+    jjjymmm.cn "QLoRA": restore the constant first, then the weight with it;
+    deck card 1: weights are dequantized to BFloat16 for every matmul.
+    Pass ``absmax`` for plain NF4, or ``qabs, scale, mu`` for NF4 + DQ."""
+    codes = _c(codes, np.uint8).reshape(-1)
+    out = np.empty(numel, np.uint16)
+    mu_arr = None if mu is None else np.array([mu], np.float32)
+    lib().oracle_nf4_dequant(
+        _ptr(codes), numel,
+        _ptr(None if absmax is None else _c(absmax, np.float32)),
+        _ptr(None if qabs is None else _c(qabs, np.int8)),
+        _ptr(None if scale is None else _c(scale, np.float32)),
+        _ptr(mu_arr), _ptr(cb32()), _ptr(out))
+    return out
+
+
+def dequant_f32(codes, numel, absmax=None, qabs=None, scale=None, mu=None):
+    """As :func:`dequant`, returning the fp32 product before BF16 rounding."""
+    codes = _c(codes, np.uint8).reshape(-1)
+    out = np.empty(numel, np.float32)
+    mu_arr = None if mu is None else np.array([mu], np.float32)
+    lib().oracle_nf4_dequant_f32(
+        _ptr(codes), numel,
+        _ptr(None if absmax is None else _c(absmax, np.float32)),
+        _ptr(None if qabs is None else _c(qabs, np.int8)),
+        _ptr(None if scale is None else _c(scale, np.float32)),
+        _ptr(mu_arr), _ptr(cb32()), _ptr(out))
+    return out
+
+
+def bf16_bits_to_f64(bits):
+    """Widen BF16 bit patterns (uint16) exactly to float64."""
+    b = np.ascontiguousarray(bits, np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def unpack_codes(codes, numel):
+    """uint8 [numel/2] -> uint8 [numel] of 4-bit codes (element 2i = high nibble)."""
+    c = np.ascontiguousarray(codes, np.uint8).reshape(-1)
+    out = np.empty(numel, np.uint8)
+    out[0::2] = c >> 4
+    out[1::2] = c & 15
+    return out
+
+
+def constant_bytes(numel: int) -> int:
+    """Bytes of quantization constants with DQ: nb int8 codes, one fp32 scale per
+    256 constants, one fp32 mean."""
+    nb = numel // BLOCK
+    ng = (nb + DQ_GROUP - 1) // DQ_GROUP
+    return nb * 1 + ng * 4 + 4

@@ -1,0 +1,133 @@
+"""Pins of the oracle's double quantization and doubleDequant.
+
+Sources: "LoRA 与 QLoRA", QLoRA section 2 (r_j = (a_j - mu)/b, 8-bit rhat_j,
+ahat_j = mu + b rhat_j, about 4.127 bit/param); deck "3 QLoRA Finetuning",
+card 4 (8/64 + 32/(64*256) ~ 0.127 bits, blocks of 256); jjjymmm.cn 2024/03
+QLoRA post, "Double Quantization" (the same count, saving 0.373) and "QLoRA"
+(doubleDequant: constants first, then weights); deck card 1 (BF16 compute).
+"""
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from bit_nf4_quantized_07_b200 import synthetic
+from oracle import codec
+from tests.conftest import read_golden_values
+
+
+def _printed():
+    out = {}
+    for line in read_golden_values("dq_storage_printed.txt"):
+        k, v = line.split()[:2]
+        out[k] = float(v)
+    return out
+
+
+def test_bits_per_param_closed_forms_against_actual_byte_counts():
+    p = _printed()
+    numel = 4096 * 4096
+    w = synthetic.normal_f32((numel // 64, 64), 0.02, 21)
+    codes, absmax = codec.quantize(w)
+    qabs, scale, mu = codec.double_quant(absmax)
+    plain_bits = 8.0 * absmax.nbytes / numel
+    dq_bytes = qabs.nbytes + scale.nbytes + np.float32(mu).nbytes
+    dq_bits = 8.0 * dq_bytes / numel
+    assert dq_bytes == codec.constant_bytes(numel)
+    assert plain_bits == p["plain_constant_bits"]
+    assert 8.0 * codes.nbytes / numel + plain_bits == p["plain_total_bits"]
+    # per-tensor mean mu is the only term not in the printed count
+    assert dq_bits - 32.0 / numel == 8 / 64 + 32 / (64 * 256)
+    assert round(dq_bits, 3) == p["dq_constant_bits"]
+    assert round(plain_bits - dq_bits, 3) == p["dq_saving_bits"]
+    assert round(plain_bits - dq_bits, 2) == p["dq_saving_bits_card"]
+    assert round(8.0 * codes.nbytes / numel + dq_bits, 3) == p["dq_total_bits"]
+    saving_gb = 65e9 * (plain_bits - dq_bits) / 8 / 1e9
+    assert round(saving_gb) == p["saving_65b_gb"]
+
+
+def test_mean_within_one_ulp_of_exact_rational_mean():
+    for seed, nb in ((31, 4096), (32, 1000), (33, 1), (34, 70001)):
+        a = np.abs(synthetic.normal_f32(nb, 0.02, seed))
+        mu = codec.dq_mean(a)
+        exact = sum((Fraction(float(x)) for x in a), Fraction(0)) / nb
+        ulp = np.spacing(np.float32(abs(float(exact))))
+        assert abs(Fraction(float(mu)) - exact) <= Fraction(float(ulp))
+
+
+def test_pairwise_tree_sum():
+    # integers: every partial sum exact, so any tree gives the exact sum
+    a = np.arange(1, 1001, dtype=np.float32)
+    assert codec.pairwise_sum(a) == 500500.0
+    # a pair-order probe: 2^24 and the ones are not associative in fp32, but
+    # the binary64 tree adds them exactly
+    a = np.array([2.0 ** 24, 1.0, 1.0, 1.0, 1.0], np.float32)
+    assert codec.pairwise_sum(a) == 2.0 ** 24 + 4
+    # against an exact reference within binary64 pairwise-summation error
+    g = synthetic.normal_f32(12345, 1.0, 35)
+    s = codec.pairwise_sum(g)
+    exact = math.fsum(float(x) for x in g)
+    assert abs(s - exact) <= 14 * np.finfo(np.float64).eps * float(np.sum(np.abs(g.astype(np.float64))))
+
+
+def test_dq_error_bound_extremes_and_range():
+    w = synthetic.normal_f32((1000 * 64 // 64, 64 * 64), 0.02, 36)  # 64 000 blocks, last group partial
+    _, absmax = codec.quantize(w)
+    nb = absmax.size
+    qabs, scale, mu = codec.double_quant(absmax)
+    assert scale.size == (nb + 255) // 256
+    assert qabs.min() >= -127 and qabs.max() <= 127
+    ahat = codec.dq_restore(qabs, scale, mu)
+    b = np.repeat(scale, 256)[:nb].astype(np.float64)
+    err = np.abs(ahat.astype(np.float64) - absmax.astype(np.float64))
+    ulp = np.spacing(np.abs(absmax)).astype(np.float64)
+    assert np.all(err <= b / 2 + 2 * ulp + np.spacing(np.float32(mu)))
+    for g in range(scale.size):
+        blk = qabs[g * 256:(g + 1) * 256]
+        assert np.max(np.abs(blk.astype(np.int32))) == 127, "the group's extreme maps to +-127"
+
+
+def test_dq_degenerate_groups():
+    a = np.full(512, 0.25, np.float32)              # all equal: b == 0
+    qabs, scale, mu = codec.double_quant(a)
+    assert mu == np.float32(0.25) and np.all(scale == 0) and np.all(qabs == 0)
+    assert np.all(codec.dq_restore(qabs, scale, mu) == np.float32(0.25))
+    a = np.zeros(300, np.float32)                    # all-zero weights -> zero constants
+    qabs, scale, mu = codec.double_quant(a)
+    assert mu == 0 and np.all(qabs == 0)
+
+
+def test_bf16_rounding_against_torch():
+    g = np.random.Generator(np.random.PCG64(37))
+    x = (g.standard_normal(200000) * 10.0 ** g.integers(-30, 30, 200000)).astype(np.float32)
+    bits = x.view(np.uint32)
+    bits[:1000] = (bits[:1000] & 0xFFFF0000) | 0x8000          # exact ties
+    bits[1000:2000] = (bits[1000:2000] & 0xFFFF0000) | 0x7FFF
+    ours = np.array([codec.bf16_rn(float(v)) for v in x], np.uint16)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_dequant_definition_and_special_codes():
+    w = synthetic.normal_f32((64, 512), 0.02, 38)
+    n = w.size
+    codes, absmax = codec.quantize(w)
+    qabs, scale, mu = codec.double_quant(absmax)
+    q = codec.unpack_codes(codes, n).reshape(-1, 64)
+    ahat = codec.dq_restore(qabs, scale, mu)
+    f32 = codec.dequant_f32(codes, n, qabs=qabs, scale=scale, mu=mu).reshape(-1, 64)
+    _, cb = codec.codebook()
+    assert np.array_equal(f32, ahat[:, None] * cb[q])            # fp32 product, NumPy IEEE
+    bf = codec.dequant(codes, n, qabs=qabs, scale=scale, mu=mu).reshape(-1, 64)
+    ref = torch.from_numpy(np.ascontiguousarray(f32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bf, ref)
+    v = codec.bf16_bits_to_f64(bf)
+    assert np.all(v[q == 7] == 0.0)
+    top = codec.bf16_bits_to_f64(torch.from_numpy(ahat).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    tb = np.broadcast_to(top[:, None], q.shape)
+    assert np.all(v[q == 15] == tb[q == 15]) and np.all(v[q == 0] == -tb[q == 0])
+    # without DQ the plain absmax is the constant
+    plain = codec.dequant_f32(codes, n, absmax=absmax).reshape(-1, 64)
+    assert np.array_equal(plain, absmax[:, None] * cb[q])
