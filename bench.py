@@ -1,0 +1,412 @@
+"""Benchmark of the QLoRA-linear hot path on B200.
+
+One step = one pass of the whole path over one batch of the layer:
+  nf4_quantize (fp32 W0 -> NF4 codes + absmax) -> nf4_double_quant ->
+  nf4_dequant (materialised BF16 W', the standalone decode) ->
+  qlora_linear_fwd (U = X A^T, fused NF4 GEMM + adapter) ->
+  qlora_linear_bwd (G = dY B, fused dX GEMM, dA, dB).
+The default workload is the prefill-shaped MLP up-projection
+(W0 11008 x 4096, 2048 tokens, r = 16, s = 2), the fwd+bwd configuration of
+the headline metric.  value = algorithmic fwd+bwd FLOPs of all ranks / the
+slowest rank's device time for K steps (CUDA events), in TFLOP/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload prefill|large|pr1]
+
+Under torchrun (N > 1) every rank runs its own replica with its own tokens
+(weak scaling) and the data-parallel exchange, an all-reduce of dA and dB, is
+part of each step.  ``--impl reference`` times the CPU oracle on the host
+cores (rank 0 only) on a bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 (de)quant GB/s, % of B200 roofline"
+
+
+def _load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def _workload(name):
+    from bit_nf4_quantized_07_b200 import synthetic
+    return {"prefill": synthetic.PREFILL, "large": synthetic.LARGE, "pr1": synthetic.PR1}[name]
+
+
+def codec_bytes_per_param():
+    """Algorithmic bytes per parameter: quantize + DQ reads fp32 W0 and writes
+    codes, rhat and the group scales; dequant reads those and writes BF16."""
+    q = 4.0 + 0.5 + 1.0 / 64 + 4.0 / (64 * 256)
+    d = 0.5 + 1.0 / 64 + 4.0 / (64 * 256) + 2.0
+    return q, d
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.12)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle leg (reported baseline / reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(cfg, budget_s=15.0):
+    """Time the oracle, as it stands, on a bounded sample of one step and
+    extrapolate to the full step.  The sample (a row slice of W0 for the codec,
+    a token slice for the fp64 linear algebra) is sized so that it takes about
+    ``budget_s`` seconds.  Returns (step_seconds_estimate, info)."""
+    from bit_nf4_quantized_07_b200 import synthetic
+    from oracle import codec, linear
+    try:
+        from threadpoolctl import threadpool_info
+        blas_threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        blas_threads = os.cpu_count() or 1
+    # probe: 1/64 of the rows, 16 tokens; then size the real sample
+    row_frac = max(64, cfg.dout // 64)
+    w = synthetic.normal_f32((row_frac, cfg.din), cfg.w_sigma, 77)
+    t0 = time.perf_counter()
+    codec.quantize(w)
+    t_probe = max(1e-4, time.perf_counter() - t0)
+    row_frac = int(min(cfg.dout, max(64, row_frac * (0.3 * budget_s) / t_probe)))
+    w = synthetic.normal_f32((row_frac, cfg.din), cfg.w_sigma, 77)
+    t0 = time.perf_counter()
+    codes, absmax = codec.quantize(w)
+    qabs, scale, mu = codec.double_quant(absmax)
+    wp_bits = codec.dequant(codes, w.size, qabs=qabs, scale=scale, mu=mu)
+    t_codec = time.perf_counter() - t0
+    codec_full = t_codec * cfg.dout / row_frac
+    # fp64 forward + backward for a token slice against the full-size weight
+    ntok = max(1, min(cfg.n, 16))
+    g = np.random.Generator(np.random.PCG64(78))
+    Wp = np.repeat(codec.bf16_bits_to_f64(wp_bits).reshape(row_frac, cfg.din), cfg.dout // row_frac + 1,
+                   axis=0)[:cfg.dout]
+    X = g.standard_normal((ntok, cfg.din))
+    A = g.standard_normal((cfg.r, cfg.din)) * cfg.ab_sigma
+    B = g.standard_normal((cfg.dout, cfg.r)) * cfg.ab_sigma
+    dY = g.standard_normal((ntok, cfg.dout))
+    t0 = time.perf_counter()
+    linear.forward(Wp, X, A, B, cfg.s)
+    linear.backward(Wp, X, A, B, cfg.s, dY)
+    t_probe = max(1e-4, time.perf_counter() - t0)
+    ntok = int(min(cfg.n, max(ntok, ntok * (0.7 * budget_s) / t_probe)))
+    X = g.standard_normal((ntok, cfg.din))
+    dY = g.standard_normal((ntok, cfg.dout))
+    t0 = time.perf_counter()
+    linear.forward(Wp, X, A, B, cfg.s)
+    linear.backward(Wp, X, A, B, cfg.s, dY)
+    t_lin = time.perf_counter() - t0
+    lin_full = t_lin * cfg.n / ntok
+    info = {"kind": "oracle", "cores": int(blas_threads),
+            "sample": f"codec (C, 1 thread) on {row_frac}x{cfg.din} of W0 (x{cfg.dout / row_frac:.0f}); "
+                      f"fp64 fwd+bwd (NumPy BLAS) on {ntok} of {cfg.n} tokens (x{cfg.n / ntok:.0f}); "
+                      f"measured {t_codec + t_lin:.2f} s",
+            "codec_s_full": codec_full, "linear_s_full": lin_full}
+    return codec_full + lin_full, info
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = _workload(args.workload)
+    flops = cfg.fwd_flops() + cfg.bwd_flops()
+    # the whole run stays within about two minutes of host time
+    budget = max(0.5, min(15.0, 120.0 / (args.steps + 1)))
+    for _ in range(args.warmup):
+        oracle_sample(cfg, budget_s=0.05)
+    times, info = [], None
+    for _ in range(args.steps):
+        t, info = oracle_sample(cfg, budget_s=budget)
+        times.append(t)
+    step_s = sum(times) / len(times)
+    value = flops / step_s / 1e12
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": cfg.name, "dout": cfg.dout, "din": cfg.din, "n": cfg.n, "r": cfg.r,
+                      "parallelism": "host cores"},
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": info["cores"], "kind": "oracle",
+                            "sample": info["sample"]},
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
+# ---------------------------------------------------------------------------
+# GPU leg
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from bit_nf4_quantized_07_b200 import api, synthetic
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    cfg = _workload(args.workload)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # Inputs: NSETS rotating sets resident in HBM (each larger than a third of L2),
+    # so every step reads inputs last touched two steps earlier.
+    NSETS = 3
+    gen = torch.Generator(device=dev)
+    sets = []
+    for i in range(NSETS):
+        gen.manual_seed(1000 * cfg.index + 100 * rank + i)
+        W = torch.randn(cfg.dout, cfg.din, generator=gen, device=dev) * cfg.w_sigma
+        if cfg.outlier_rate > 0:
+            m = torch.rand(cfg.dout, cfg.din, generator=gen, device=dev) < cfg.outlier_rate
+            W = torch.where(m, W * 10.0, W)
+        X = torch.randn(cfg.n, cfg.din, generator=gen, device=dev).to(torch.bfloat16)
+        A = (torch.randn(cfg.r, cfg.din, generator=gen, device=dev) * cfg.ab_sigma).to(torch.bfloat16)
+        B = (torch.randn(cfg.dout, cfg.r, generator=gen, device=dev) * cfg.ab_sigma).to(torch.bfloat16)
+        dY = torch.randn(cfg.n, cfg.dout, generator=gen, device=dev).to(torch.bfloat16)
+        sets.append((W.contiguous(), X, A, B, dY))
+    numel = cfg.dout * cfg.din
+    nb = numel // 64
+    codes = torch.empty(numel // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(nb, dtype=torch.float32, device=dev)
+    qabs = torch.empty(nb, dtype=torch.int8, device=dev)
+    scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+    mu = torch.empty(1, dtype=torch.float32, device=dev)
+    wdq = torch.empty(cfg.dout, cfg.din, dtype=torch.bfloat16, device=dev)
+    Y = torch.empty(cfg.n, cfg.dout, dtype=torch.bfloat16, device=dev)
+    U = torch.empty(cfg.n, cfg.r, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(cfg.n, cfg.din, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(cfg.r, cfg.din, dtype=torch.float32, device=dev)
+    dB = torch.empty(cfg.dout, cfg.r, dtype=torch.float32, device=dev)
+    ws_dq = api.alloc_workspace(api.workspace_bytes(api.OP_DOUBLE_QUANT, nb), dev)
+    ws_f = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_FWD, cfg.dout, cfg.din, cfg.n, cfg.r), dev)
+    ws_b = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_BWD, cfg.dout, cfg.din, cfg.n, cfg.r), dev)
+    wq = api.NF4Weight(codes=codes, rows=cfg.dout, cols=cfg.din, absmax=absmax, qabs=qabs, dq_scale=scale,
+                       dq_mean=mu)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(i, marks=None):
+        W, X, A, B, dYs = sets[i % NSETS]
+        if marks is not None:
+            marks[0].record(stream)
+        api.nf4_quantize(W, codes, absmax)
+        api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)
+        if marks is not None:
+            marks[1].record(stream)
+        api.nf4_dequant(wq, wdq)
+        if marks is not None:
+            marks[2].record(stream)
+        api.qlora_linear_fwd(wq, X, A, B, cfg.s, Y=Y, U_out=U, ws=ws_f)
+        if marks is not None:
+            marks[3].record(stream)
+        api.qlora_linear_bwd(wq, X, A, B, cfg.s, dYs, U=U, dX=dX, dA=dA, dB=dB, ws=ws_b)
+        if marks is not None:
+            marks[4].record(stream)
+        if world > 1:
+            dist.all_reduce(dA)
+            dist.all_reduce(dB)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    marks = [[ev() for _ in range(5)] for _ in range(args.steps)]
+    start, stop = ev(), ev()
+    launches0 = api.launch_count()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(i, marks[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    launches = api.launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    elapsed_ms = start.elapsed_time(stop)
+    sec = {"quantize_dq": 0.0, "dequant": 0.0, "fwd": 0.0, "bwd": 0.0}
+    for m in marks:
+        sec["quantize_dq"] += m[0].elapsed_time(m[1])
+        sec["dequant"] += m[1].elapsed_time(m[2])
+        sec["fwd"] += m[2].elapsed_time(m[3])
+        sec["bwd"] += m[3].elapsed_time(m[4])
+    sec = {k: v / args.steps for k, v in sec.items()}
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # End to end through the C ABI with host buffers: copies inside the timed region.
+    W, X, A, B, dYs = sets[0]
+    hW, hX, hA, hB, hdY = (t.cpu().pin_memory() for t in (W, X, A, B, dYs))
+    dW, dXi, dAi, dBi, ddY = (torch.empty_like(t) for t in (W, X, A, B, dYs))
+    oY, odX, odA, odB = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (Y, dX, dA, dB))
+
+    def e2e_step():
+        for d, h in ((dW, hW), (dXi, hX), (dAi, hA), (dBi, hB), (ddY, hdY)):
+            d.copy_(h, non_blocking=True)
+        api.nf4_quantize(dW, codes, absmax)
+        api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)
+        api.nf4_dequant(wq, wdq)
+        api.qlora_linear_fwd(wq, dXi, dAi, dBi, cfg.s, Y=Y, U_out=U, ws=ws_f)
+        api.qlora_linear_bwd(wq, dXi, dAi, dBi, cfg.s, ddY, U=U, dX=dX, dA=dA, dB=dB, ws=ws_b)
+        if world > 1:
+            dist.all_reduce(dA)
+            dist.all_reduce(dB)
+        for h, d in ((oY, Y), (odX, dX), (odA, dA), (odB, dB)):
+            h.copy_(d, non_blocking=True)
+
+    h2d = sum(t.numel() * t.element_size() for t in (hW, hX, hA, hB, hdY))
+    d2h = sum(t.numel() * t.element_size() for t in (oY, odX, odA, odB))
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    flops = cfg.fwd_flops() + cfg.bwd_flops()
+    ms_per_step = elapsed_ms / args.steps
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    e2e_value = world * flops / (e2e_ms / e2e_steps * 1e-3) / 1e12
+    peaks = _load_peaks()
+    qb, db = codec_bytes_per_param()
+    fwd_tflops = cfg.fwd_flops() / (sec["fwd"] * 1e-3) / 1e12
+    roof = {"kernel": "qlora_linear_fwd (fused NF4 GEMM + U)", "bound": "tensor", "achieved": fwd_tflops,
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": fwd_tflops / peaks["bf16_tflops"],
+            "traffic": None, "peak_source": peaks["source"] + " bf16 burst"}
+    parts = {
+        "quantize_dq_GBs": numel * qb / (sec["quantize_dq"] * 1e-3) / 1e9,
+        "dequant_GBs": numel * db / (sec["dequant"] * 1e-3) / 1e9,
+        "fwd_TFLOPs": fwd_tflops,
+        "bwd_TFLOPs": cfg.bwd_flops() / (sec["bwd"] * 1e-3) / 1e12,
+        "ms": sec,
+        "hbm_peak_GBs": peaks["hbm_gbs"],
+    }
+    parts["quantize_dq_frac_hbm"] = parts["quantize_dq_GBs"] / peaks["hbm_gbs"]
+    parts["dequant_frac_hbm"] = parts["dequant_GBs"] / peaks["hbm_gbs"]
+    out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": cfg.name, "dout": cfg.dout, "din": cfg.din, "n": cfg.n, "r": cfg.r, "s": cfg.s,
+                      "global_batch": cfg.n * world, "parallelism": f"dp{world}",
+                      "step": "nf4_quantize+nf4_double_quant+nf4_dequant+qlora_linear_fwd+qlora_linear_bwd",
+                      "l2": "3 rotating input sets (W0 fp32 alone 180 MB > 126 MB L2)"},
+           "gpu_launches": launches, "roofline": roof, "parts": parts, "clocks": clk.summary(),
+           "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        step_s, info = oracle_sample(cfg)
+        out["cpu_baseline"] = {"value": flops / step_s / 1e12, "unit": "TFLOP/s", "cores": info["cores"],
+                               "kind": "oracle", "sample": info["sample"]}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["prefill", "large", "pr1"], default="prefill")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

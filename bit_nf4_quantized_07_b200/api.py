@@ -1,0 +1,234 @@
+"""Thin ctypes binding of libqlora_nf4.so (the C ABI in include/qlora_nf4.h).
+
+Argument marshalling only: tensors are torch CUDA tensors (torch provides the
+device memory and the current stream); every step of the computation runs in
+the library's CUDA kernels.  There is no fallback: if the library is missing
+or a call fails, an exception is raised.
+
+Function names follow the C entry points: ``nf4_quantize``,
+``nf4_double_quant``, ``nf4_dequant``, ``qlora_linear_fwd``,
+``qlora_linear_bwd``, plus ``workspace_bytes``, ``codebook``, ``version``.
+"""
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
+
+QLN_OK = 0
+STATUS_NAMES = {0: "QLN_OK", 1: "QLN_ERR_NULL", 2: "QLN_ERR_SHAPE", 3: "QLN_ERR_ALIGN", 4: "QLN_ERR_WORKSPACE",
+                5: "QLN_ERR_ARCH", 6: "QLN_ERR_CUDA", 7: "QLN_ERR_TIMEOUT", 8: "QLN_ERR_INTERNAL"}
+OP_DOUBLE_QUANT, OP_LINEAR_FWD, OP_LINEAR_BWD = 1, 2, 3
+
+#: Every symbol include/qlora_nf4.h declares.
+EXPORTS = ("nf4_quantize", "nf4_double_quant", "nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd",
+           "qln_workspace_bytes", "qln_codebook", "qln_status_str", "qln_version", "qln_launch_count")
+
+
+class QLNError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class CNF4Weight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p), ("qabs", ctypes.c_void_p),
+                ("dq_scale", ctypes.c_void_p), ("dq_mean", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libqlora_nf4.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with bit_nf4_quantized_07_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I32, SZ, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
+        WP = ctypes.POINTER(CNF4Weight)
+        sig = {
+            "nf4_quantize": ([P, I64, P, P, P], I32),
+            "nf4_double_quant": ([P, I64, P, P, P, P, SZ, P], I32),
+            "nf4_dequant": ([WP, P, P], I32),
+            "qlora_linear_fwd": ([WP, P, I64, P, P, I32, F, P, P, P, SZ, P], I32),
+            "qlora_linear_bwd": ([WP, P, I64, P, P, I32, F, P, P, P, P, P, P, SZ, P], I32),
+            "qln_workspace_bytes": ([I32, I64, I64, I64, I32], SZ),
+            "qln_codebook": ([P], None),
+            "qln_status_str": ([I32], ctypes.c_char_p),
+            "qln_version": ([], I32),
+            "qln_launch_count": ([], ctypes.c_uint64),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(fn, st):
+    if st != QLN_OK:
+        raise QLNError(fn, st)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def version() -> int:
+    return lib().qln_version()
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued since it was loaded."""
+    return int(lib().qln_launch_count())
+
+
+def codebook() -> torch.Tensor:
+    """The 16 fp32 NF4 values the kernels use (host copy)."""
+    out = (ctypes.c_float * 16)()
+    lib().qln_codebook(out)
+    return torch.tensor(list(out), dtype=torch.float32)
+
+
+def status_str(st: int) -> str:
+    return lib().qln_status_str(st).decode()
+
+
+def workspace_bytes(op: int, rows: int, cols: int = 0, n: int = 0, r: int = 0) -> int:
+    return int(lib().qln_workspace_bytes(op, rows, cols, n, r))
+
+
+def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """Device scratch (torch-allocated, 256-byte aligned by the caching allocator)."""
+    t = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+    assert t.data_ptr() % 256 == 0
+    return t
+
+
+@dataclass
+class NF4Weight:
+    """An NF4 weight [rows][cols] as stored on the device."""
+    codes: torch.Tensor                    # uint8 [rows*cols/2]
+    rows: int
+    cols: int
+    absmax: Optional[torch.Tensor] = None  # fp32 [nb]
+    qabs: Optional[torch.Tensor] = None    # int8 [nb]
+    dq_scale: Optional[torch.Tensor] = None
+    dq_mean: Optional[torch.Tensor] = None
+
+    def c_struct(self) -> CNF4Weight:
+        return CNF4Weight(self.codes.data_ptr(), self.absmax.data_ptr() if self.absmax is not None else None,
+                          self.qabs.data_ptr() if self.qabs is not None else None,
+                          self.dq_scale.data_ptr() if self.dq_scale is not None else None,
+                          self.dq_mean.data_ptr() if self.dq_mean is not None else None, self.rows, self.cols)
+
+
+def nf4_quantize(W: torch.Tensor, codes: Optional[torch.Tensor] = None, absmax: Optional[torch.Tensor] = None):
+    """fp32 W (any shape, numel % 64 == 0) -> (codes uint8 [numel/2], absmax fp32 [numel/64])."""
+    n = W.numel()
+    if codes is None:
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=W.device)
+    if absmax is None:
+        absmax = torch.empty(n // 64, dtype=torch.float32, device=W.device)
+    _need_cuda(W, codes, absmax)
+    _check("nf4_quantize", lib().nf4_quantize(_p(W), n, _p(codes), _p(absmax), _stream()))
+    return codes, absmax
+
+
+def nf4_double_quant(absmax: torch.Tensor, qabs=None, dq_scale=None, dq_mean=None, ws=None):
+    """fp32 absmax [nb] -> (qabs int8 [nb], dq_scale fp32 [ceil(nb/256)], dq_mean fp32 [1])."""
+    nb = absmax.numel()
+    dev = absmax.device
+    if qabs is None:
+        qabs = torch.empty(nb, dtype=torch.int8, device=dev)
+    if dq_scale is None:
+        dq_scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+    if dq_mean is None:
+        dq_mean = torch.empty(1, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = alloc_workspace(workspace_bytes(OP_DOUBLE_QUANT, nb), dev)
+    _need_cuda(absmax, qabs, dq_scale, dq_mean, ws)
+    _check("nf4_double_quant", lib().nf4_double_quant(_p(absmax), nb, _p(qabs), _p(dq_scale), _p(dq_mean), _p(ws),
+                                                      ws.numel(), _stream()))
+    return qabs, dq_scale, dq_mean
+
+
+def quantize_weight(W: torch.Tensor, double_quant: bool = True, ws=None) -> NF4Weight:
+    """nf4_quantize (+ nf4_double_quant) of a [rows][cols] fp32 weight."""
+    rows, cols = W.shape
+    codes, absmax = nf4_quantize(W)
+    w = NF4Weight(codes=codes, rows=rows, cols=cols, absmax=absmax)
+    if double_quant:
+        w.qabs, w.dq_scale, w.dq_mean = nf4_double_quant(absmax, ws=ws)
+    return w
+
+
+def nf4_dequant(w: NF4Weight, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """doubleDequant to BF16 [rows][cols]."""
+    if out is None:
+        out = torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=w.codes.device)
+    _need_cuda(w.codes, out)
+    cw = w.c_struct()
+    _check("nf4_dequant", lib().nf4_dequant(ctypes.byref(cw), _p(out), _stream()))
+    return out
+
+
+def qlora_linear_fwd(w: NF4Weight, X, A, B, s: float, Y=None, U_out=None, ws=None, want_u: bool = True):
+    """Y = X W'^T + s (X A^T) B^T.  Returns (Y [n][dout] bf16, U [n][r] bf16 or None)."""
+    n = X.shape[0]
+    r = A.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty(n, w.rows, dtype=torch.bfloat16, device=dev)
+    if U_out is None and want_u:
+        U_out = torch.empty(n, r, dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = alloc_workspace(workspace_bytes(OP_LINEAR_FWD, w.rows, w.cols, n, r), dev)
+    _need_cuda(X, A, B, Y, U_out, ws)
+    cw = w.c_struct()
+    _check("qlora_linear_fwd", lib().qlora_linear_fwd(ctypes.byref(cw), _p(X), n, _p(A), _p(B), r, float(s), _p(Y),
+                                                      _p(U_out), _p(ws), ws.numel(), _stream()))
+    return Y, U_out
+
+
+def qlora_linear_bwd(w: NF4Weight, X, A, B, s: float, dY, U=None, dX=None, dA=None, dB=None, ws=None):
+    """Returns (dX [n][din] bf16, dA [r][din] fp32, dB [dout][r] fp32)."""
+    n = X.shape[0]
+    r = A.shape[0]
+    dev = X.device
+    if dX is None:
+        dX = torch.empty(n, w.cols, dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty(r, w.cols, dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty(w.rows, r, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = alloc_workspace(workspace_bytes(OP_LINEAR_BWD, w.rows, w.cols, n, r), dev)
+    _need_cuda(X, A, B, dY, U, dX, dA, dB, ws)
+    cw = w.c_struct()
+    _check("qlora_linear_bwd", lib().qlora_linear_bwd(ctypes.byref(cw), _p(X), n, _p(A), _p(B), r, float(s), _p(dY),
+                                                      _p(U), _p(dX), _p(dA), _p(dB), _p(ws), ws.numel(), _stream()))
+    return dX, dA, dB
+
+
+def device_status(ws: torch.Tensor) -> int:
+    """The int32 status word at workspace offset 0 (synchronises the current stream)."""
+    return int(ws[:4].view(torch.int32).item())

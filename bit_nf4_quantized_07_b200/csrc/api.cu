@@ -1,0 +1,284 @@
+// C ABI of libqlora_nf4: argument checks, workspace layout, kernel dispatch.
+// Every entry point validates synchronously, then only enqueues work on the
+// caller's stream: no allocation, no synchronisation, no host-device copies.
+#include <string.h>
+
+#include <atomic>
+
+#include "qln_common.cuh"
+#include "qln_internal.h"
+
+namespace qln {
+static std::atomic<uint64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace qln
+
+namespace {
+using qln::note_launch;
+
+constexpr int kMaxDevices = 64;
+int g_arch_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
+int g_num_sms[kMaxDevices];
+
+qln_status check_device(int *num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QLN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return QLN_ERR_CUDA;
+    if (g_arch_ok[dev] == 0) {
+        int major = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return QLN_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return QLN_ERR_CUDA;
+        g_num_sms[dev] = sms;
+        g_arch_ok[dev] = (major == 10) ? 1 : -1;
+    }
+    if (g_arch_ok[dev] < 0) return QLN_ERR_ARCH;
+    *num_sms = g_num_sms[dev];
+    return QLN_OK;
+}
+
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Split-K choice for the token reductions: sized for a fixed target grid so
+// that the workspace size does not depend on the device queried.
+constexpr int kSplitTargetSms = 148;
+
+// Workspace layout of the linear calls (all offsets 256-byte aligned):
+//   [0, 256)        int32 device status word (0 = QLN_OK) + reserved
+//   fwd: sU [n][r] bf16, U [n][r] bf16 (used when U_out is NULL)
+//   bwd: Bt [r][dout] bf16, G [n][r] bf16, sG [n][r] bf16, U [n][r] bf16,
+//        dA partials, dB partials (fp32, split-K)
+struct FwdWs {
+    size_t sU, U, total;
+};
+struct BwdWs {
+    size_t Bt, G, sG, U, pA, pB, total;
+    int splitA, splitB;
+};
+
+FwdWs fwd_layout(int64_t n, int r) {
+    FwdWs L;
+    const size_t nr = round256((size_t)n * r * 2);
+    L.sU = 256;
+    L.U = L.sU + nr;
+    L.total = L.U + nr;
+    return L;
+}
+
+BwdWs bwd_layout(int64_t rows, int64_t cols, int64_t n, int r) {
+    BwdWs L;
+    const size_t nr = round256((size_t)n * r * 2);
+    L.Bt = 256;
+    L.G = L.Bt + round256((size_t)rows * r * 2);
+    L.sG = L.G + nr;
+    L.U = L.sG + nr;
+    L.splitA = qln::tn_reduce_splits(n, r, cols, kSplitTargetSms);
+    L.splitB = qln::tn_reduce_splits(n, rows, r, kSplitTargetSms);
+    L.pA = L.U + nr;
+    L.pB = L.pA + round256(qln::tn_reduce_partials_bytes(r, cols, L.splitA));
+    L.total = L.pB + round256(qln::tn_reduce_partials_bytes(rows, r, L.splitB));
+    return L;
+}
+
+qln_status check_weight(const qln_nf4_weight *w) {
+    if (!w || !w->codes) return QLN_ERR_NULL;
+    if (w->qabs) {
+        if (!w->dq_scale || !w->dq_mean) return QLN_ERR_NULL;
+    } else if (!w->absmax) {
+        return QLN_ERR_NULL;
+    }
+    if (w->rows <= 0 || w->cols <= 0 || (w->cols % 64) != 0) return QLN_ERR_SHAPE;
+    if (!aligned(w->codes, 16)) return QLN_ERR_ALIGN;
+    if (w->absmax && !aligned(w->absmax, 4)) return QLN_ERR_ALIGN;
+    if (w->dq_scale && !aligned(w->dq_scale, 4)) return QLN_ERR_ALIGN;
+    if (w->dq_mean && !aligned(w->dq_mean, 4)) return QLN_ERR_ALIGN;
+    return QLN_OK;
+}
+
+qln_status check_linear(const qln_nf4_weight *w, const uint16_t *X, int64_t n, const uint16_t *A,
+                        const uint16_t *B, int32_t r) {
+    qln_status s = check_weight(w);
+    if (s != QLN_OK) return s;
+    if (!X || !A || !B) return QLN_ERR_NULL;
+    if (n < 1 || r < 8 || r > 128 || (r % 8) != 0) return QLN_ERR_SHAPE;
+    if ((w->rows % 64) != 0) return QLN_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 16)) return QLN_ERR_ALIGN;
+    return QLN_OK;
+}
+
+qln_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QLN_OK : QLN_ERR_CUDA; }
+
+// B [rows][r] -> Bt [r][rows]
+__global__ void transpose_bf16_kernel(const uint16_t *__restrict__ B, int64_t rows, int r, uint16_t *__restrict__ Bt) {
+    const int64_t total = rows * r;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int64_t o = i / r;
+        const int j = (int)(i % r);
+        Bt[(int64_t)j * rows + o] = B[i];
+    }
+}
+
+// The fused weight GEMM: tcgen05 where the shape fills its tiles, otherwise
+// the register-level path.
+cudaError_t fused_gemm(const qln_nf4_weight *w, bool trans, const uint16_t *act, int64_t n, const uint16_t *lact,
+                       const uint16_t *lw, int r, uint16_t *out, int *status, cudaStream_t st, int num_sms) {
+    if (qln::nf4_tc_gemm_supported(w, trans, n, r))
+        return qln::launch_nf4_tc_gemm(w, trans, act, n, lact, lw, r, out, status, st, num_sms);
+    return qln::launch_nf4_mma_gemm(w, trans, act, n, lact, lw, r, out, status, st, num_sms);
+}
+
+}  // namespace
+
+extern "C" {
+
+qln_status nf4_quantize(const float *W, int64_t numel, uint8_t *codes, float *absmax, void *stream) {
+    if (!W || !codes || !absmax) return QLN_ERR_NULL;
+    if (numel <= 0 || (numel % 64) != 0) return QLN_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(absmax, 4)) return QLN_ERR_ALIGN;
+    int sms = 0;
+    qln_status s = check_device(&sms);
+    if (s != QLN_OK) return s;
+    return from_cuda(qln::launch_nf4_quantize(W, numel, codes, absmax, (cudaStream_t)stream, sms));
+}
+
+qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale, float *dq_mean,
+                            void *ws, size_t ws_bytes, void *stream) {
+    if (!absmax || !qabs || !dq_scale || !dq_mean || !ws) return QLN_ERR_NULL;
+    if (nb <= 0 || nb > qln::dq_max_blocks()) return QLN_ERR_SHAPE;
+    if (!aligned(absmax, 16) || !aligned(qabs, 4) || !aligned(dq_scale, 4) || !aligned(dq_mean, 4))
+        return QLN_ERR_ALIGN;
+    if (!aligned(ws, 256)) return QLN_ERR_ALIGN;
+    if (ws_bytes < qln::dq_workspace_bytes(nb)) return QLN_ERR_WORKSPACE;
+    int sms = 0;
+    qln_status s = check_device(&sms);
+    if (s != QLN_OK) return s;
+    return from_cuda(qln::launch_nf4_double_quant(absmax, nb, qabs, dq_scale, dq_mean, ws, (cudaStream_t)stream));
+}
+
+qln_status nf4_dequant(const qln_nf4_weight *w, uint16_t *out, void *stream) {
+    qln_status s = check_weight(w);
+    if (s != QLN_OK) return s;
+    if (!out) return QLN_ERR_NULL;
+    if (!aligned(out, 16)) return QLN_ERR_ALIGN;
+    int sms = 0;
+    s = check_device(&sms);
+    if (s != QLN_OK) return s;
+    return from_cuda(qln::launch_nf4_dequant(w, out, (cudaStream_t)stream, sms));
+}
+
+qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t n, const uint16_t *A,
+                            const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *U_out, void *ws,
+                            size_t ws_bytes, void *stream) {
+    qln_status st = check_linear(w, X, n, A, B, r);
+    if (st != QLN_OK) return st;
+    if (!Y || !ws) return QLN_ERR_NULL;
+    if (!aligned(Y, 16) || (U_out && !aligned(U_out, 16)) || !aligned(ws, 256)) return QLN_ERR_ALIGN;
+    const FwdWs L = fwd_layout(n, r);
+    if (ws_bytes < L.total) return QLN_ERR_WORKSPACE;
+    int sms = 0;
+    st = check_device(&sms);
+    if (st != QLN_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream;
+    char *wsb = reinterpret_cast<char *>(ws);
+    int *status = reinterpret_cast<int *>(wsb);
+    uint16_t *sU = reinterpret_cast<uint16_t *>(wsb + L.sU);
+    uint16_t *U = U_out ? U_out : reinterpret_cast<uint16_t *>(wsb + L.U);
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
+    if (e != cudaSuccess) return QLN_ERR_CUDA;
+    // U = X A^T (and s*U for the adapter MMA), then the fused weight GEMM.
+    e = qln::launch_lora_down(X, n, w->cols, A, w->cols, 1, r, s, U, sU, cs, sms);
+    if (e != cudaSuccess) return QLN_ERR_CUDA;
+    e = fused_gemm(w, false, X, n, sU, B, r, Y, status, cs, sms);
+    return from_cuda(e);
+}
+
+qln_status qlora_linear_bwd(const qln_nf4_weight *w, const uint16_t *X, int64_t n, const uint16_t *A,
+                            const uint16_t *B, int32_t r, float s, const uint16_t *dY, const uint16_t *U,
+                            uint16_t *dX, float *dA, float *dB, void *ws, size_t ws_bytes, void *stream) {
+    qln_status st = check_linear(w, X, n, A, B, r);
+    if (st != QLN_OK) return st;
+    if (!dY || !dX || !dA || !dB || !ws) return QLN_ERR_NULL;
+    if (!aligned(dY, 16) || !aligned(dX, 16) || !aligned(dA, 16) || !aligned(dB, 16) || !aligned(ws, 256) ||
+        (U && !aligned(U, 16)))
+        return QLN_ERR_ALIGN;
+    const BwdWs L = bwd_layout(w->rows, w->cols, n, r);
+    if (ws_bytes < L.total) return QLN_ERR_WORKSPACE;
+    int sms = 0;
+    st = check_device(&sms);
+    if (st != QLN_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream;
+    char *wsb = reinterpret_cast<char *>(ws);
+    int *status = reinterpret_cast<int *>(wsb);
+    uint16_t *Bt = reinterpret_cast<uint16_t *>(wsb + L.Bt);
+    uint16_t *G = reinterpret_cast<uint16_t *>(wsb + L.G);
+    uint16_t *sG = reinterpret_cast<uint16_t *>(wsb + L.sG);
+    float *pA = reinterpret_cast<float *>(wsb + L.pA);
+    float *pB = reinterpret_cast<float *>(wsb + L.pB);
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
+    if (e != cudaSuccess) return QLN_ERR_CUDA;
+    if (!U) {
+        uint16_t *Uw = reinterpret_cast<uint16_t *>(wsb + L.U);
+        e = qln::launch_lora_down(X, n, w->cols, A, w->cols, 1, r, s, Uw, nullptr, cs, sms);
+        if (e != cudaSuccess) return QLN_ERR_CUDA;
+        U = Uw;
+    }
+    {
+        const int64_t total = w->rows * r;
+        int64_t blocks = (total + 255) / 256;
+        if (blocks > 4096) blocks = 4096;
+        transpose_bf16_kernel<<<(unsigned)blocks, 256, 0, cs>>>(B, w->rows, r, Bt);
+        note_launch();
+        if (cudaGetLastError() != cudaSuccess) return QLN_ERR_CUDA;
+    }
+    // G = dY B (and s*G), dX = dY W' + (s G) A, dA = s G^T X, dB = s dY^T U.
+    e = qln::launch_lora_down(dY, n, w->rows, Bt, w->rows, 1, r, s, G, sG, cs, sms);
+    if (e != cudaSuccess) return QLN_ERR_CUDA;
+    e = fused_gemm(w, true, dY, n, sG, A, r, dX, status, cs, sms);
+    if (e != cudaSuccess) return QLN_ERR_CUDA;
+    e = qln::launch_tn_reduce(G, X, n, r, w->cols, s, dA, pA, L.splitA, cs);
+    if (e != cudaSuccess) return QLN_ERR_CUDA;
+    e = qln::launch_tn_reduce(dY, U, n, w->rows, r, s, dB, pB, L.splitB, cs);
+    return from_cuda(e);
+}
+
+size_t qln_workspace_bytes(int32_t op, int64_t rows, int64_t cols, int64_t n, int32_t r) {
+    switch (op) {
+        case QLN_OP_DOUBLE_QUANT:
+            return rows > 0 ? qln::dq_workspace_bytes(rows) : 0;
+        case QLN_OP_LINEAR_FWD:
+            return (n > 0 && r > 0) ? fwd_layout(n, r).total : 0;
+        case QLN_OP_LINEAR_BWD:
+            return (rows > 0 && cols > 0 && n > 0 && r > 0) ? bwd_layout(rows, cols, n, r).total : 0;
+        default:
+            return 0;
+    }
+}
+
+void qln_codebook(float out16[16]) {
+    for (int i = 0; i < 16; ++i) {
+        uint32_t b = qln::kNF4Bits[i];
+        memcpy(&out16[i], &b, 4);
+    }
+}
+
+const char *qln_status_str(qln_status st) {
+    switch (st) {
+        case QLN_OK: return "QLN_OK";
+        case QLN_ERR_NULL: return "QLN_ERR_NULL";
+        case QLN_ERR_SHAPE: return "QLN_ERR_SHAPE";
+        case QLN_ERR_ALIGN: return "QLN_ERR_ALIGN";
+        case QLN_ERR_WORKSPACE: return "QLN_ERR_WORKSPACE";
+        case QLN_ERR_ARCH: return "QLN_ERR_ARCH";
+        case QLN_ERR_CUDA: return "QLN_ERR_CUDA";
+        case QLN_ERR_TIMEOUT: return "QLN_ERR_TIMEOUT";
+        case QLN_ERR_INTERNAL: return "QLN_ERR_INTERNAL";
+        default: return "QLN_ERR_UNKNOWN";
+    }
+}
+
+int32_t qln_version(void) { return (1 << 16) | 0; }
+
+uint64_t qln_launch_count(void) { return qln::g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,115 @@
+// Shared device helpers of libqlora_nf4 (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qlora_nf4.h"
+
+namespace qln {
+
+// ---------------------------------------------------------------------------
+// The NF4 book: 16 fp32 values, ascending, exact zero at index 7, ends +-1.
+// Built (offline, in binary64, then rounded once to binary32) from normal
+// quantiles with separate negative and positive halves sharing one zero,
+// normalized by the largest quantile: deck "3 QLoRA Finetuning" cards 2-3,
+// "LoRA 与 QLoRA" section QLoRA 1 (归一化与匹配).  Positive half: Q_Z at 8 of 9
+// probabilities evenly spaced from delta to 1/2; negative half: -Q_Z at 7 of 8;
+// delta = 1 - (1/32 + 1/30)/2.  Matches the 4-decimal table printed in the
+// jjjymmm.cn post ("4-bit NormalFloat(NF4)").  Stored as bit patterns so the
+// values are exact; a CPU test compares them with an independent recomputation.
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr uint32_t kNF4Bits[16] = {
+    0xbf800000u, 0xbf3239b1u, 0xbf066b2eu, 0xbeca329eu, 0xbe91a24bu, 0xbe3d353du,
+    0xbdba7869u, 0x00000000u, 0x3da2fb01u, 0x3e24cadfu, 0x3e7c04dau, 0x3ead0336u,
+    0x3ee1a4b5u, 0x3f1007a9u, 0x3f3913b0u, 0x3f800000u};
+
+constexpr int kBlock = 64;     // weights per absmax block
+constexpr int kDqGroup = 256;  // block constants per DQ scale
+
+__device__ __forceinline__ float nf4_value(int q) { return __uint_as_float(kNF4Bits[q]); }
+
+// Snap thresholds: t_k = the largest fp32 value <= (c_k + c_{k+1}) / 2.
+// For an fp32 x, x > t_k  <=>  x is strictly closer to c_{k+1} than to c_k,
+// so  q = #{k : x > t_k}  is the nearest book entry with ties to the lower
+// code.  Halving is exact; __fadd_rd rounds the exact sum toward -inf.
+__device__ __forceinline__ float nf4_threshold(int k) {
+    return __fadd_rd(0.5f * nf4_value(k), 0.5f * nf4_value(k + 1));
+}
+
+// ---------------------------------------------------------------------------
+// Small conversions.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    // lo -> bits [0,16) (the lower address), hi -> bits [16,32); both RN.
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// doubleDequant of one block constant: ahat = fp32(mu + fp32(b * rhat)), the
+// product first, then the sum ("LoRA 与 QLoRA" section 2, reconstruction).
+__device__ __forceinline__ float dq_restore(int8_t rhat, float b, float mu) {
+    return __fadd_rn(mu, __fmul_rn(b, (float)rhat));
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers: cp.async, ldmatrix, legacy mma.sync (used by the skinny,
+// HBM-bound kernels and the small-n path).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem));
+}
+// Zero-filling form: copies src_bytes (0 or 16) and fills the rest with 0.
+__device__ __forceinline__ void cp_async16_zfill(void *smem, const void *gmem, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)), "l"(gmem),
+                 "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
+                                            const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
+                                                  const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldmatrix_x2(uint32_t &r0, uint32_t &r1, const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t &r0, uint32_t &r1, const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(smem_u32(p)));
+}
+
+// D[16x8] += A[16x16] (row) * B[16x8] (col), bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__host__ __device__ constexpr int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+}  // namespace qln

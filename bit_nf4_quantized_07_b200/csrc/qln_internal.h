@@ -1,0 +1,49 @@
+// Internal launchers of libqlora_nf4 (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/qlora_nf4.h"
+
+namespace qln {
+
+// Host-side count of kernels enqueued by this library (qln_launch_count).
+void note_launch();
+
+// codec.cu
+cudaError_t launch_nf4_quantize(const float *W, int64_t numel, uint8_t *codes, float *absmax,
+                                cudaStream_t st, int num_sms);
+cudaError_t launch_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,
+                                    void *ws, cudaStream_t st);
+cudaError_t launch_nf4_dequant(const qln_nf4_weight *w, uint16_t *out, cudaStream_t st, int num_sms);
+size_t dq_workspace_bytes(int64_t nb);
+int64_t dq_max_blocks();
+
+// lora_small.cu: skinny products around the adapters.
+//   out[t][j] = bf16(sum_k in[t][k] * wt(j, k)) and, if out_scaled != NULL,
+//   out_scaled[t][j] = bf16(scale * that sum); wt(j, k) = wt[j*wt_sj + k*wt_sk].
+cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int64_t wt_sj,
+                             int64_t wt_sk, int r, float scale, uint16_t *out, uint16_t *out_scaled,
+                             cudaStream_t st, int num_sms);
+//   C[m][c] = scale * sum_t P[t][m] * Q[t][c]  (P [n][M], Q [n][N] row-major), fp32 out.
+cudaError_t launch_tn_reduce(const uint16_t *P, const uint16_t *Q, int64_t n, int64_t M, int64_t N, float scale,
+                             float *C, float *partials, int splits, cudaStream_t st);
+size_t tn_reduce_partials_bytes(int64_t M, int64_t N, int splits);
+int tn_reduce_splits(int64_t n, int64_t M, int64_t N, int num_sms);
+
+// nf4_gemm_sm80.cu: fused NF4 decode + legacy mma.sync GEMM (small n).
+//   trans = false: out[t][m] = bf16(sum_k act[t][k] W'[m][k] + sum_j lact[t][j] lw[m][j])   (forward)
+//   trans = true : out[t][m] = bf16(sum_k act[t][k] W'[k][m] + sum_j lact[t][j] lw[j][m])   (dX)
+cudaError_t launch_nf4_mma_gemm(const qln_nf4_weight *w, bool trans, const uint16_t *act, int64_t n,
+                                const uint16_t *lact, const uint16_t *lw, int r, uint16_t *out,
+                                int *status, cudaStream_t st, int num_sms);
+
+// nf4_gemm_sm100.cu: fused NF4 decode + tcgen05 GEMM (TMA, TMEM accumulators).
+cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16_t *act, int64_t n,
+                               const uint16_t *lact, const uint16_t *lw, int r, uint16_t *out,
+                               int *status, cudaStream_t st, int num_sms);
+bool nf4_tc_gemm_supported(const qln_nf4_weight *w, bool trans, int64_t n, int r);
+
+}  // namespace qln

@@ -1,0 +1,212 @@
+/*
+ * qlora_nf4.h -- C ABI of libqlora_nf4.so, the sm_100a (B200) hot path of a
+ * QLoRA linear layer:
+ *   (1) blockwise NF4 quantization of a frozen fp32 weight W0,
+ *   (2) double quantization (DQ) of the per-block constants,
+ *   (3) doubleDequant to BF16, and the fused forward / backward of
+ *           Y = X * doubleDequant(W0)^T + s * (X A^T) B^T.
+ *
+ * The method is described on these web pages (cited per entry point):
+ *   "LoRA 与 QLoRA" (whoami-wesleyyou.top): section LoRA, section QLoRA
+ *       "1. NF4" and "2. Double Quantization (DQ)".
+ *   "QLoRA: Efficient Finetuning of Quantized LLMs", deck "3 QLoRA Finetuning"
+ *       (learn.ifs.name), cards 1-4.
+ *   jjjymmm.cn 2024/03 QLoRA post: "4-bit NormalFloat(NF4)", "Double
+ *       Quantization", "QLoRA" (doubleDequant).
+ *   "QLoRA：4-bit 量化与显存账" (finetune.xph.ink kp-007): the
+ *       BitsAndBytesConfig flag set (load_in_4bit, nf4, use_double_quant,
+ *       compute dtype bf16) that this ABI mirrors.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers, owned by the caller.  The library
+ *   never allocates, frees or synchronises; every call enqueues its kernels on
+ *   `stream` (a cudaStream_t passed as void*; NULL = legacy default stream) and
+ *   returns.  Outputs are overwritten, never accumulated into.
+ * - BF16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ * - Layouts are row-major and dense.  Tokens are the leading dimension of the
+ *   activations: X [n][din], Y [n][dout], dY [n][dout], dX [n][din],
+ *   U = X A^T [n][r].  Weights: W0 [dout][din] (rows = dout, cols = din),
+ *   A [r][din], B [dout][r], dA [r][din] fp32, dB [dout][r] fp32.
+ * - NF4 storage of a [rows][cols] weight, numel = rows*cols, flattened
+ *   row-major, blocks of 64 consecutive elements (nb = numel/64):
+ *     codes  uint8 [numel/2]: element 2i in the HIGH nibble of byte i,
+ *                             element 2i+1 in the low nibble;
+ *     absmax fp32  [nb]     : a_j = max |w| over block j (plain NF4);
+ *     qabs   int8  [nb]     : DQ code rhat_j of a_j;
+ *     dq_scale fp32 [ng]    : DQ step b_g per group of 256 blocks,
+ *                             ng = ceil(nb/256);
+ *     dq_mean fp32 [1]      : mu, the mean of all a_j.
+ * - Synchronous argument errors are returned BEFORE anything is launched:
+ *   NULL pointers (QLN_ERR_NULL), bad sizes (QLN_ERR_SHAPE), pointers not
+ *   16-byte aligned (QLN_ERR_ALIGN), workspace too small (QLN_ERR_WORKSPACE),
+ *   current device not sm_100 (QLN_ERR_ARCH).  A failed launch returns
+ *   QLN_ERR_CUDA (cudaGetLastError).  Kernels that wait on on-chip barriers
+ *   give up after a bounded number of polls and write QLN_ERR_TIMEOUT into the
+ *   int32 status word at byte offset 0 of the workspace; read it after the
+ *   stream has synchronised (0 = QLN_OK).
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLN_API __attribute__((visibility("default")))
+#else
+#define QLN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QLN_OK = 0,
+    QLN_ERR_NULL = 1,      /* a required pointer is NULL                       */
+    QLN_ERR_SHAPE = 2,     /* a size is out of range or not a multiple of 64   */
+    QLN_ERR_ALIGN = 3,     /* a pointer is not 16-byte aligned                 */
+    QLN_ERR_WORKSPACE = 4, /* ws_bytes below qln_workspace_bytes(...)          */
+    QLN_ERR_ARCH = 5,      /* current device is not compute capability 10.x    */
+    QLN_ERR_CUDA = 6,      /* a CUDA runtime call or launch failed             */
+    QLN_ERR_TIMEOUT = 7,   /* device side: a bounded barrier wait gave up      */
+    QLN_ERR_INTERNAL = 8   /* device side: an internal consistency check failed*/
+} qln_status;
+
+/* Workspace-sized operations (qln_workspace_bytes `op`). */
+enum { QLN_OP_DOUBLE_QUANT = 1, QLN_OP_LINEAR_FWD = 2, QLN_OP_LINEAR_BWD = 3 };
+
+/* An NF4 weight as stored by nf4_quantize (+ nf4_double_quant).  All pointers
+ * are device pointers owned by the caller.  With qabs != NULL the weight is
+ * double-quantized (qabs, dq_scale, dq_mean are used, absmax is ignored);
+ * with qabs == NULL the plain fp32 absmax is used (bnb_4bit_use_double_quant
+ * off).  cols must be a multiple of 64, so blocks never straddle rows. */
+typedef struct {
+    const uint8_t *codes;
+    const float *absmax;
+    const int8_t *qabs;
+    const float *dq_scale;
+    const float *dq_mean;
+    int64_t rows; /* dout */
+    int64_t cols; /* din  */
+} qln_nf4_weight;
+
+/*
+ * nf4_quantize -- blockwise NF4 quantization.
+ * Defined by: jjjymmm.cn "4-bit NormalFloat(NF4)" (divide by the block
+ * ABSMAX, snap to the nearest quant-book entry); "LoRA 与 QLoRA" section 2
+ * (a_j = max |W_j| per block of 64); deck "3 QLoRA Finetuning" cards 2-3 (the
+ * asymmetric 16-entry NormalFloat book with an exact zero and ends at +-1).
+ *   W      [numel] fp32 in : weights, flattened row-major.
+ *   codes  [numel/2] u8 out, absmax [numel/64] fp32 out.
+ * Per element x = fp32(w / a_j) (IEEE division, round to nearest) and the
+ * code is the nearest of the 16 entries, ties to the lower code; a block with
+ * a_j == 0 gets code 7 (the exact zero) throughout.  Non-finite inputs are
+ * not checked (undefined codes).
+ * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE if numel <= 0 or numel % 64 != 0;
+ * QLN_ERR_ALIGN if W or codes is not 16-byte aligned (absmax: 4-byte).
+ */
+QLN_API qln_status nf4_quantize(const float *W, int64_t numel, uint8_t *codes, float *absmax,
+                        void *stream);
+
+/*
+ * nf4_double_quant -- quantize the block constants to 8 bits.
+ * Defined by: "LoRA 与 QLoRA" section 2 (r_j = (a_j - mu)/b, 8-bit rhat_j,
+ * ahat_j = mu + b rhat_j, mu and b stored in 32 bits); deck card 4 and
+ * jjjymmm.cn "Double Quantization" (blocks of 256 constants).
+ *   absmax   [nb] fp32 in;  qabs [nb] int8 out;  dq_scale [ceil(nb/256)] fp32
+ *   out;  dq_mean [1] fp32 out.
+ * mu = fp32(S / nb), S the binary64 sum of all a_j over a fixed perfect binary
+ * tree (leaves zero-padded to a power of two), so mu is reproducible bit for
+ * bit.  Per group g: d_j = fp32(a_j - mu), b_g = fp32(max|d_j| / 127),
+ * rhat_j = clamp(rint(fp32(d_j / b_g)), -127, 127) (ties to even), 0 when
+ * b_g == 0.  The last group may be partial.
+ *   ws / ws_bytes: device scratch of at least
+ *   qln_workspace_bytes(QLN_OP_DOUBLE_QUANT, nb, 0, 0, 0) bytes, 256-byte
+ *   aligned; contents on entry are ignored.
+ * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE if nb <= 0 or nb > 2^25 (numel above
+ * 2^31); QLN_ERR_WORKSPACE; QLN_ERR_ALIGN if absmax is not 16-byte aligned or
+ * ws is not 256-byte aligned.
+ */
+QLN_API qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale,
+                            float *dq_mean, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * nf4_dequant -- doubleDequant of a whole weight to BF16.
+ * Defined by: jjjymmm.cn "QLoRA" (restore the quantization constant first,
+ * then dequantize the weight with it; a code dequantizes to its quant-book
+ * value); deck card 1 (weights are dequantized to BFloat16 for the matmul).
+ *   out [rows*cols] bf16 (uint16) out:  w' = bf16_RN(fp32(ahat_j * c[q])),
+ *   ahat_j = fp32(mu + fp32(b_g * rhat_j)) with DQ, a_j without.
+ * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE (rows, cols <= 0, cols % 64);
+ * QLN_ERR_ALIGN (codes, out).
+ */
+QLN_API qln_status nf4_dequant(const qln_nf4_weight *w, uint16_t *out, void *stream);
+
+/*
+ * qlora_linear_fwd -- fused QLoRA linear forward.
+ * Defined by: "LoRA 与 QLoRA" section LoRA (y = W0 x + s B(A x); A x is
+ * formed first, BA never is) and section QLoRA "1. NF4" (4-bit weight ->
+ * dequant -> BF16 -> GEMM); jjjymmm.cn "QLoRA" (the forward dequantizes W
+ * twice, from NF4 to BF16, and multiplies with BF16 X).
+ *   X [n][din] bf16 in, A [r][din] bf16 in, B [dout][r] bf16 in, s scale,
+ *   Y [n][dout] bf16 out = bf16_RN(X W'^T + s U B^T) with fp32 accumulation,
+ *   U_out [n][r] bf16 out (nullable): U = bf16_RN(X A^T), unscaled, for reuse
+ *   by qlora_linear_bwd.
+ * W' is decoded tile by tile on chip and never written to HBM.
+ *   ws: at least qln_workspace_bytes(QLN_OP_LINEAR_FWD, dout, din, n, r)
+ *   bytes, 256-byte aligned; byte 0 holds the device status word afterwards.
+ * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE (n < 1; r not a multiple of 8 in
+ * 8..128; rows (dout) or cols (din) not a multiple of 64); QLN_ERR_ALIGN
+ * (16-byte: codes, X, A, B, Y, U_out; ws 256-byte); QLN_ERR_WORKSPACE;
+ * QLN_ERR_ARCH.
+ */
+QLN_API qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t n,
+                            const uint16_t *A, const uint16_t *B, int32_t r, float s,
+                            uint16_t *Y, uint16_t *U_out, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/*
+ * qlora_linear_bwd -- fused QLoRA linear backward.
+ * Defined by: deck card 1 (gradients flow through the dequantized weights;
+ * only the adapters receive updates); "LoRA 与 QLoRA" section LoRA (W0 fixed,
+ * only A and B trained); jjjymmm.cn "QLoRA" (backward updates only the LoRA
+ * factors).  For Y = X W'^T + s (X A^T) B^T and upstream gradient dY:
+ *   G  = dY B                 [n][r]    (kept in the workspace, bf16)
+ *   dX = dY W' + s G A        [n][din]  bf16 out
+ *   dA = s G^T X              [r][din]  fp32 out
+ *   dB = s dY^T U             [dout][r] fp32 out, U = X A^T
+ * U (nullable) is the U_out of the matching forward; when NULL it is
+ * recomputed.  W0 gets no gradient.
+ * ws: at least qln_workspace_bytes(QLN_OP_LINEAR_BWD, dout, din, n, r) bytes.
+ * Errors: as qlora_linear_fwd, plus QLN_ERR_NULL for dY, dX, dA, dB.
+ */
+QLN_API qln_status qlora_linear_bwd(const qln_nf4_weight *w, const uint16_t *X, int64_t n,
+                            const uint16_t *A, const uint16_t *B, int32_t r, float s,
+                            const uint16_t *dY, const uint16_t *U, uint16_t *dX, float *dA,
+                            float *dB, void *ws, size_t ws_bytes, void *stream);
+
+/* Device workspace, in bytes, that `op` needs for these sizes (nb for
+ * QLN_OP_DOUBLE_QUANT is passed as `rows`).  Returns 0 for an unknown op. */
+QLN_API size_t qln_workspace_bytes(int32_t op, int64_t rows, int64_t cols, int64_t n, int32_t r);
+
+/* The 16 NF4 values (fp32, ascending) the kernels snap to and decode with. */
+QLN_API void qln_codebook(float out16[16]);
+
+/* Human-readable name of a status code (static string). */
+QLN_API const char *qln_status_str(qln_status st);
+
+/* ABI version: (major << 16) | minor. */
+QLN_API int32_t qln_version(void);
+
+/* Number of kernels this library has enqueued since it was loaded, over all
+ * threads and devices (a host-side counter; cudaMemsetAsync of the status word
+ * is not counted).  For accounting of launches in benchmarks. */
+QLN_API uint64_t qln_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

@@ -1,0 +1,137 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, carries the oracle's NF4 book bit for bit, and rejects bad
+arguments before touching the device.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from bit_nf4_quantized_07_b200 import api
+from oracle import codec
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        names |= set(re.findall(r"QLN_API\s+[\w\s\*]+?\b(\w+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_nf4_quantized_07_b200 import build
+    build.build()
+    return api.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = _declared_symbols()
+    assert declared == set(api.EXPORTS), declared
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_only_the_abi_is_exported(L):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", api.LIB_PATH], capture_output=True, text=True).stdout
+    text = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert text == set(api.EXPORTS)
+
+
+def test_library_codebook_equals_oracle_construction(L):
+    lib_cb = api.codebook().numpy()
+    _, ora = codec.codebook()
+    assert np.array_equal(lib_cb.view(np.uint32), ora.view(np.uint32))
+
+
+def test_version_and_status_strings(L):
+    assert api.version() >> 16 == 1
+    for code, name in api.STATUS_NAMES.items():
+        assert api.status_str(code) == name
+
+
+def test_workspace_sizes(L):
+    assert api.workspace_bytes(api.OP_DOUBLE_QUANT, 4096) >= 256 + 8
+    assert api.workspace_bytes(api.OP_DOUBLE_QUANT, 3670016) >= 256 + 8 * (3670016 // 8192)
+    f = api.workspace_bytes(api.OP_LINEAR_FWD, 11008, 4096, 2048, 16)
+    assert f >= 256 + 2 * 2048 * 16 * 2
+    b = api.workspace_bytes(api.OP_LINEAR_BWD, 11008, 4096, 2048, 16)
+    assert b >= 256 + 11008 * 16 * 2 + 3 * 2048 * 16 * 2
+    assert api.workspace_bytes(99, 1, 1, 1, 1) == 0
+    for v in (f, b, api.workspace_bytes(api.OP_DOUBLE_QUANT, 1)):
+        assert v % 256 == 0
+
+
+# Argument errors are reported before any CUDA call, so they can be checked
+# with fake, never-dereferenced addresses on a machine without a GPU.
+P = ctypes.c_void_p
+A16 = P(0x10000)          # 16-byte aligned fake device address
+A4 = P(0x10004)           # 4-byte aligned only
+
+
+def _w(codes=A16, absmax=A16, qabs=None, scale=None, mean=None, rows=64, cols=64):
+    return api.CNF4Weight(codes.value if codes else None, absmax.value if absmax else None,
+                          qabs.value if qabs else None, scale.value if scale else None,
+                          mean.value if mean else None, rows, cols)
+
+
+def test_quantize_argument_errors(L):
+    assert L.nf4_quantize(None, 64, A16, A16, None) == 1
+    assert L.nf4_quantize(A16, 0, A16, A16, None) == 2
+    assert L.nf4_quantize(A16, 96, A16, A16, None) == 2
+    assert L.nf4_quantize(A4, 64, A16, A16, None) == 3
+    assert L.nf4_quantize(A16, 64, A4, A16, None) == 3
+
+
+def test_double_quant_argument_errors(L):
+    ws = P(0x20000)
+    need = api.workspace_bytes(api.OP_DOUBLE_QUANT, 100)
+    assert L.nf4_double_quant(None, 100, A16, A16, A16, ws, need, None) == 1
+    assert L.nf4_double_quant(A16, 0, A16, A16, A16, ws, need, None) == 2
+    assert L.nf4_double_quant(A16, (1 << 25) + 1, A16, A16, A16, ws, 1 << 40, None) == 2
+    assert L.nf4_double_quant(A16, 100, A16, A16, A16, P(0x20010), need, None) == 3
+    assert L.nf4_double_quant(A16, 100, A16, A16, A16, ws, need - 1, None) == 4
+
+
+def test_dequant_argument_errors(L):
+    out = A16
+    assert L.nf4_dequant(None, out, None) == 1
+    assert L.nf4_dequant(ctypes.byref(_w(codes=None)), out, None) == 1
+    assert L.nf4_dequant(ctypes.byref(_w(absmax=None)), out, None) == 1         # no DQ and no absmax
+    assert L.nf4_dequant(ctypes.byref(_w(absmax=None, qabs=A16)), out, None) == 1  # DQ without scale/mean
+    assert L.nf4_dequant(ctypes.byref(_w(cols=96)), out, None) == 2
+    assert L.nf4_dequant(ctypes.byref(_w(rows=0)), out, None) == 2
+    assert L.nf4_dequant(ctypes.byref(_w(codes=P(0x10008))), out, None) == 3
+    assert L.nf4_dequant(ctypes.byref(_w()), P(0x10002), None) == 3
+
+
+def test_linear_argument_errors(L):
+    w = _w(rows=128, cols=256)
+    ws = P(0x40000)
+    fwd = lambda **k: L.qlora_linear_fwd(ctypes.byref(k.get("w", w)), k.get("X", A16), k.get("n", 4),
+                                         A16, A16, k.get("r", 16), 1.0, k.get("Y", A16), None,
+                                         k.get("ws", ws), k.get("wsb", 1 << 30), None)
+    assert fwd(X=None) == 1
+    assert fwd(Y=None) == 1
+    assert fwd(n=0) == 2
+    assert fwd(r=12) == 2
+    assert fwd(r=136) == 2
+    assert fwd(w=_w(rows=100, cols=256)) == 2
+    assert fwd(X=P(0x10008)) == 3
+    assert fwd(ws=P(0x40010)) == 3
+    need = api.workspace_bytes(api.OP_LINEAR_FWD, 128, 256, 4, 16)
+    assert fwd(wsb=need - 1) == 4
+    bwd = L.qlora_linear_bwd(ctypes.byref(w), A16, 4, A16, A16, 16, 1.0, None, None, A16, A16, A16, ws, 1 << 30,
+                             None)
+    assert bwd == 1
+    need = api.workspace_bytes(api.OP_LINEAR_BWD, 128, 256, 4, 16)
+    bwd = L.qlora_linear_bwd(ctypes.byref(w), A16, 4, A16, A16, 16, 1.0, A16, None, A16, A16, A16, ws, need - 1,
+                             None)
+    assert bwd == 4

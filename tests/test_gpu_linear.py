@@ -1,0 +1,138 @@
+"""GPU parity of the fused QLoRA linear (forward and backward) against the
+float64 oracle.  Tolerance (the benchmark spec): normwise max relative error
+max|T - T*| / max|T*| <= 2e-2 per output tensor."""
+import numpy as np
+import pytest
+import torch
+
+from bit_nf4_quantized_07_b200 import api, synthetic
+from oracle import linear
+from tests.oracle_ref import (OracleWeight, backward_ref, bf16_to_dev, dev_bf16_bits, f64, forward_ref,
+                              workload)
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+
+def _gpu_weight(w, double_quant=True):
+    return api.quantize_weight(torch.from_numpy(w).cuda(), double_quant=double_quant)
+
+
+def _run(cfg, w, X, A, B, dY, double_quant=True, backward=True):
+    wq = _gpu_weight(w, double_quant)
+    Xd, Ad, Bd = bf16_to_dev(X), bf16_to_dev(A), bf16_to_dev(B)
+    Y, U = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s)
+    out = {"Y": f64(dev_bf16_bits(Y)), "U": f64(dev_bf16_bits(U))}
+    if backward:
+        dX, dA, dB = api.qlora_linear_bwd(wq, Xd, Ad, Bd, cfg.s, bf16_to_dev(dY), U=U)
+        out.update(dX=f64(dev_bf16_bits(dX)), dA=dA.double().cpu().numpy(), dB=dB.double().cpu().numpy())
+    torch.cuda.synchronize()
+    return out
+
+
+def _compare(name, got, ref, tol=TOL):
+    err = linear.normwise_error(got, ref)
+    fro = linear.frobenius_error(got, ref)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), name
+    assert err <= tol, f"{name}: normwise {err:.3e} (frobenius {fro:.3e})"
+    return err
+
+
+SMALL = [
+    synthetic.PR1,
+    synthetic.custom("ragged_192x320_n77_r16", 192, 320, 77, 16, s=2.0, index=11),
+    synthetic.custom("single_token_128x128_n1_r8", 128, 128, 1, 8, s=0.5, index=12),
+    synthetic.custom("tall_256x512_n300_r64", 256, 512, 300, 64, s=1.0, index=13),
+    synthetic.custom("r128_128x256_n33_r128", 128, 256, 33, 128, s=2.0, index=14),
+    synthetic.custom("tokens_tile_512x256_n256_r16", 512, 256, 256, 16, s=2.0, index=15),
+    synthetic.custom("wide_384x1024_n640_r32", 384, 1024, 640, 32, s=1.5, index=16, outlier_rate=0.001),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+@pytest.mark.parametrize("dq", [True, False], ids=["dq", "plain"])
+def test_linear_small_configs(cfg, dq):
+    w, X, A, B, dY = workload(cfg)
+    ow = OracleWeight(w, double_quant=dq)
+    got = _run(cfg, w, X, A, B, dY, double_quant=dq)
+    Y, U = forward_ref(ow, X, A, B, cfg.s)
+    dX, dA, dB = backward_ref(ow, X, A, B, cfg.s, dY)
+    _compare("U", got["U"], U)
+    _compare("Y", got["Y"], Y)
+    _compare("dX", got["dX"], dX)
+    _compare("dA", got["dA"], dA)
+    _compare("dB", got["dB"], dB)
+
+
+@pytest.mark.parametrize("batch", [1, 4, 16])
+def test_decode_forward(batch):
+    cfg = synthetic.DECODE[batch]
+    w, X, A, B, dY = workload(cfg)
+    ow = OracleWeight(w)
+    got = _run(cfg, w, X, A, B, dY, backward=False)
+    Y, U = forward_ref(ow, X, A, B, cfg.s)
+    _compare("U", got["U"], U)
+    _compare("Y", got["Y"], Y)
+
+
+def test_adapter_off_matches_cublas_on_materialised_weight():
+    """B = 0 (or s = 0): the fused forward reduces to X W'^T; cross-check it
+    against torch.matmul (cuBLAS) on nf4_dequant's materialised W'."""
+    cfg = synthetic.custom("b0_512x512_n96", 512, 512, 96, 16, index=17)
+    w, X, A, B, dY = workload(cfg)
+    wq = _gpu_weight(w)
+    Xd, Ad = bf16_to_dev(X), bf16_to_dev(A)
+    Y0, _ = api.qlora_linear_fwd(wq, Xd, Ad, torch.zeros(cfg.dout, cfg.r, dtype=torch.bfloat16, device="cuda"), 2.0)
+    Ys, _ = api.qlora_linear_fwd(wq, Xd, Ad, bf16_to_dev(B), 0.0)
+    ref = torch.matmul(Xd.float(), api.nf4_dequant(wq).float().T)
+    for Y in (Y0, Ys):
+        err = (Y.float() - ref).abs().max().item() / ref.abs().max().item()
+        assert err <= 4e-3, err
+
+
+def test_backward_with_and_without_saved_u_and_determinism():
+    cfg = synthetic.custom("reuse_256x256_n100_r16", 256, 256, 100, 16, index=18)
+    w, X, A, B, dY = workload(cfg)
+    wq = _gpu_weight(w)
+    Xd, Ad, Bd, dYd = bf16_to_dev(X), bf16_to_dev(A), bf16_to_dev(B), bf16_to_dev(dY)
+    Y1, U = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s)
+    Y2, _ = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s)
+    assert torch.equal(Y1, Y2)
+    a = api.qlora_linear_bwd(wq, Xd, Ad, Bd, cfg.s, dYd, U=U)
+    b = api.qlora_linear_bwd(wq, Xd, Ad, Bd, cfg.s, dYd, U=None)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_all_zero_weight_leaves_only_the_adapter():
+    cfg = synthetic.custom("zero_w_128x192_n40_r8", 128, 192, 40, 8, index=19)
+    _, X, A, B, dY = workload(cfg)
+    w = np.zeros((cfg.dout, cfg.din), np.float32)
+    got = _run(cfg, w, X, A, B, dY)
+    U = f64(X) @ f64(A).T
+    _compare("Y", got["Y"], cfg.s * U @ f64(B).T)
+
+
+def _sampled(cfg, ntok=8):
+    w, X, A, B, dY = workload(cfg)
+    ow = OracleWeight(w)
+    got = _run(cfg, w, X, A, B, dY)
+    rng = np.random.Generator(np.random.PCG64(cfg.index))
+    tok = np.unique(np.r_[0, cfg.n - 1, rng.integers(0, cfg.n, ntok)])
+    Y, U = forward_ref(ow, X, A, B, cfg.s, token_idx=tok)
+    _compare("U", got["U"][tok], U)
+    _compare("Y", got["Y"][tok], Y)
+    dX, dA, dB = backward_ref(ow, X, A, B, cfg.s, dY, token_idx=tok)
+    _compare("dX", got["dX"][tok], dX)
+    _compare("dA", got["dA"], dA)
+    _compare("dB", got["dB"], dB)
+
+
+def test_prefill_sampled():
+    _sampled(synthetic.PREFILL)
+
+
+@pytest.mark.slow
+def test_large_sampled():
+    _sampled(synthetic.LARGE)
