@@ -257,7 +257,7 @@ size_t qln_workspace_bytes(int32_t op, int64_t rows, int64_t cols, int64_t n, in
 
 void qln_codebook(float out16[16]) {
     for (int i = 0; i < 16; ++i) {
-        uint32_t b = qln::kNF4Bits[i];
+        uint32_t b = qln::nf4_bits(i);
         memcpy(&out16[i], &b, 4);
     }
 }

@@ -271,46 +271,40 @@ cudaError_t launch_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qab
 }
 
 // ===========================================================================
-// K4: doubleDequant to BF16.  One thread turns 8 codes (one 32-bit word) into
-// 8 BF16 values (one 16-byte store); the 8 threads of a 64-block restore the
-// same ahat.  w' = bf16_RN(fp32(ahat * c[q])).
+// K4: doubleDequant to BF16.  A warp streams 64 code words (512 weights,
+// 8 blocks) per step: lane l decodes words 2l and 2l+1 (16 weights of block
+// l/4) with the register-only table decode and stores 32 contiguous bytes.
+// w' = bf16_RN(fp32(ahat * c[q])).
 // ===========================================================================
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t *__restrict__ codes32,
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint2 *__restrict__ codes64,
                                                           const float *__restrict__ absmax,
                                                           const int8_t *__restrict__ qabs,
                                                           const float *__restrict__ scale,
-                                                          const float *__restrict__ mu_p, int64_t nwords,
+                                                          const float *__restrict__ mu_p, int64_t npairs,
                                                           uint4 *__restrict__ out) {
-    __shared__ float cb[16];
-    if (threadIdx.x < 16) cb[threadIdx.x] = nf4_value(threadIdx.x);
-    __syncthreads();
     const float mu = qabs ? __ldg(mu_p) : 0.f;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nwords; i += stride) {
-        const int64_t j = i >> 3;  // 8 words (64 codes) per block
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < npairs; i += stride) {
+        const int64_t j = i >> 2;  // 4 pairs of words (64 codes) per block
         float ah;
         if (qabs) ah = dq_restore(__ldg(qabs + j), __ldg(scale + (j >> 8)), mu);
         else ah = __ldg(absmax + j);
-        const uint32_t cw = __ldcs(codes32 + i);
-        uint32_t o[4];
-#pragma unroll
-        for (int bi = 0; bi < 4; ++bi) {
-            const uint32_t byte = (cw >> (8 * bi)) & 0xffu;
-            o[bi] = pack_bf16x2(__fmul_rn(ah, cb[byte >> 4]), __fmul_rn(ah, cb[byte & 15u]));
-        }
-        __stcs(out + i, make_uint4(o[0], o[1], o[2], o[3]));
+        const uint2 cw = __ldcs(codes64 + i);
+        const NF4Table t = nf4_table(ah);
+        __stcs(out + 2 * i, nf4_decode8(cw.x, t));
+        __stcs(out + 2 * i + 1, nf4_decode8(cw.y, t));
     }
 }
 
 cudaError_t launch_nf4_dequant(const qln_nf4_weight *w, uint16_t *out, cudaStream_t st, int num_sms) {
     const int64_t numel = w->rows * w->cols;
-    const int64_t nwords = numel / 8;
-    int64_t grid = (nwords + 255) / 256;
+    const int64_t npairs = numel / 16;
+    int64_t grid = (npairs + 255) / 256;
     const int64_t cap = (int64_t)num_sms * 8;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
-    nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint32_t *>(w->codes), w->absmax,
-                                                      w->qabs, w->dq_scale, w->dq_mean, nwords,
+    nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint2 *>(w->codes), w->absmax,
+                                                      w->qabs, w->dq_scale, w->dq_mean, npairs,
                                                       reinterpret_cast<uint4 *>(out));
     note_launch();
     return cudaGetLastError();

@@ -1,15 +1,384 @@
-// Fused NF4 doubleDequant + tcgen05 GEMM (placeholder until the sm_100a
-// kernel lands: reports every shape as unsupported).
+// Fused NF4 doubleDequant + GEMM on the sm_100a tensor cores (tcgen05, TMEM
+// accumulator, TMA operand loads).  W' is decoded tile by tile into shared
+// memory and never reaches HBM.
+//
+// Method: "LoRA 与 QLoRA" section QLoRA 1 (4-bit weight -> dequant -> BF16 ->
+// GEMM) and section LoRA (y = W0 x + s B(A x), A x formed first); jjjymmm.cn
+// "QLoRA" (doubleDequant: restore the block constant, then the weight); deck
+// "3 QLoRA Finetuning" card 1 (the matmul sees the dequantized BF16 weight and
+// gradients flow through it).
+//
+//   forward (TRANS = false): out[t][m] = sum_k X[t][k] W'[m][k]  + sum_j sU[t][j] B[m][j]
+//   dX      (TRANS = true) : out[t][m] = sum_k dY[t][k] W'[k][m] + sum_j sG[t][j] A[j][m]
+//
+// One CTA computes a 128 (m) x BN (tokens, <= 256) tile: D = A_op * B_op^T in
+// TMEM with M = 128 (m), N = BN (tokens), K in steps of 64.
+//   A_op (weights): decoded by 4 warps into the canonical 128-byte-swizzled
+//     layout, K-major for the forward (W' rows along K) and MN-major for dX
+//     (W' rows are the K index, their 128 consecutive columns the M index);
+//   B_op (activations X / dY, K-major): TMA tiles with 128-byte swizzle;
+//   the adapter term is extra K steps whose A_op (B or A, zero-padded to 64)
+//     and B_op (s*U or s*G) both arrive by TMA.
+// Warp roles: warp 0 TMA producer, warp 1 TMEM owner + single-thread MMA
+// issuer, warps 2-5 decoders and then the epilogue (TMEM -> BF16 -> HBM).
+// Every barrier wait is bounded; on give-up the CTA records QLN_ERR_TIMEOUT
+// in the status word, drains its own copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+
 #include "qln_common.cuh"
 #include "qln_internal.h"
+#include "tc_ptx.cuh"
 
 namespace qln {
+namespace tc {
 
-bool nf4_tc_gemm_supported(const qln_nf4_weight *, bool, int64_t, int) { return false; }
+constexpr int kStages = 4;
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kMaxBN = 256;
+constexpr int kThreads = 192;
+constexpr int kDecThreads = 128;
+constexpr uint32_t kABytes = kBM * kBK * 2;      // 16 KB
+constexpr uint32_t kBBytes = kMaxBN * kBK * 2;   // 32 KB
+constexpr uint32_t kCBytes = 4096;               // 128 rows x 32 B (fwd) or 64 rows x 64 B (dX)
+constexpr uint32_t kStageBytes = kABytes + kBBytes + kCBytes;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
 
-cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *, bool, const uint16_t *, int64_t, const uint16_t *,
-                               const uint16_t *, int, uint16_t *, int *, cudaStream_t, int) {
-    return cudaErrorNotSupported;
+// shared-memory map (offsets from a 1024-aligned base)
+constexpr uint32_t kOffA = 0;
+constexpr uint32_t kOffB = kOffA + kStages * kABytes;
+constexpr uint32_t kOffC = kOffB + kStages * kBBytes;
+constexpr uint32_t kOffBar = kOffC + kStages * kCBytes;
+// barriers: tma_full[S], code_full[S], dec_full[S], empty[S], accum_full
+constexpr uint32_t kNumBars = 4 * kStages + 1;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem base (u32), abort flag (int)
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
+
+struct Params {
+    const int8_t *qabs;
+    const float *absmax;
+    const float *dq_scale;
+    const float *dq_mean;
+    int64_t cols;      // W columns (din)
+    int64_t n;         // tokens
+    uint16_t *out;     // [n][out_ld]
+    int64_t out_ld;
+    int *status;
+    int KT;            // weight k-steps
+    int RT;            // adapter k-steps
+    int BN;            // tokens per tile (multiple of 16, <= 256)
+};
+
+template <bool TRANS>
+__global__ void __launch_bounds__(kThreads, 1)
+nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_act,
+                   const __grid_constant__ CUtensorMap tm_lw, const __grid_constant__ CUtensorMap tm_lact,
+                   const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t bar0 = sbase + kOffBar;
+    auto tma_full = [&](int s) { return bar0 + 8u * s; };
+    auto code_full = [&](int s) { return bar0 + 8u * (kStages + s); };
+    auto dec_full = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+    auto empty = [&](int s) { return bar0 + 8u * (3 * kStages + s); };
+    const uint32_t accum_full = bar0 + 8u * (4 * kStages);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t0 = (int64_t)blockIdx.x * p.BN;
+    const int64_t m0 = (int64_t)blockIdx.y * kBM;
+    const int nsteps = p.KT + p.RT;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(tma_full(s), 1);
+            mbar_init(code_full(s), 1);
+            mbar_init(dec_full(s), kDecThreads);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(accum_full, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+        tma_prefetch_map(&tm_codes);
+        tma_prefetch_map(&tm_act);
+        tma_prefetch_map(&tm_lw);
+        tma_prefetch_map(&tm_lact);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = *tmem_slot;
+
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        atomicExch(p.status, (int)QLN_ERR_TIMEOUT);
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint32_t bbytes = (uint32_t)p.BN * kBK * 2;
+            int issued = 0;
+            for (int kt = 0; kt < nsteps; ++kt) {
+                const int s = kt % kStages;
+                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                if (!mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, kWaitLimitNs)) {
+                    give_up();
+                    break;
+                }
+                const uint32_t sA = sbase + kOffA + s * kABytes;
+                const uint32_t sB = sbase + kOffB + s * kBBytes;
+                const uint32_t sC = sbase + kOffC + s * kCBytes;
+                if (kt < p.KT) {
+                    mbar_arrive_expect_tx(code_full(s), kCBytes);
+                    if (!TRANS) tma_load_2d(sC, &tm_codes, kt * 32, (int32_t)m0, code_full(s));
+                    else tma_load_2d(sC, &tm_codes, (int32_t)(m0 / 2), kt * kBK, code_full(s));
+                    mbar_arrive_expect_tx(tma_full(s), bbytes);
+                    tma_load_2d(sB, &tm_act, kt * kBK, (int32_t)t0, tma_full(s));
+                } else {
+                    const int a = kt - p.KT;
+                    mbar_arrive_expect_tx(tma_full(s), kABytes + bbytes);
+                    if (!TRANS) {
+                        tma_load_2d(sA, &tm_lw, a * kBK, (int32_t)m0, tma_full(s));
+                    } else {
+                        tma_load_2d(sA, &tm_lw, (int32_t)m0, a * kBK, tma_full(s));
+                        tma_load_2d(sA + 8192, &tm_lw, (int32_t)m0 + 64, a * kBK, tma_full(s));
+                    }
+                    tma_load_2d(sB, &tm_lact, a * kBK, (int32_t)t0, tma_full(s));
+                }
+                issued = kt + 1;
+            }
+            // Drain: every issued copy has landed before the CTA may exit.
+            for (int kt = (issued > kStages ? issued - kStages : 0); kt < issued; ++kt) {
+                const int s = kt % kStages;
+                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                if (!mbar_wait_bounded(tma_full(s), ph, nullptr, kWaitLimitNs)) give_up();
+                if (kt < p.KT && !mbar_wait_bounded(code_full(s), ph, nullptr, kWaitLimitNs)) give_up();
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(kBM, p.BN, TRANS, false);
+            for (int kt = 0; kt < nsteps; ++kt) {
+                const int s = kt % kStages;
+                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                if (!mbar_wait_bounded(tma_full(s), ph, abort_flag, kWaitLimitNs) ||
+                    !mbar_wait_bounded(dec_full(s), ph, abort_flag, kWaitLimitNs)) {
+                    give_up();
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sA = sbase + kOffA + s * kABytes;
+                const uint32_t sB = sbase + kOffB + s * kBBytes;
+#pragma unroll
+                for (int k = 0; k < kBK / 16; ++k) {
+                    // K-major: next 16 K elements are 32 bytes further inside the
+                    // swizzled 128-byte rows.  MN-major: next two 8-row K groups.
+                    const uint64_t adesc = TRANS ? smem_desc_sw128(sA + k * 2048, 8192, 1024)
+                                                 : smem_desc_sw128(sA + k * 32, 16, 1024);
+                    const uint64_t bdesc = smem_desc_sw128(sB + k * 32, 16, 1024);
+                    tc_mma_ss(tmem_d, adesc, bdesc, idesc, (kt | k) != 0 ? 1u : 0u);
+                }
+                tc_commit(empty(s));
+            }
+            tc_commit(accum_full);
+        }
+    } else {
+        // ------------------------------------------------------------ decoders
+        const int dt = threadIdx.x - 64;  // 0..127
+        // fwd: thread = W row m0+dt, block column kt.  dX: thread = W row
+        // 64*kt + (dt % 64), block column m0/64 + dt/64.
+        const int64_t bpr = p.cols / 64;
+        const int drow = TRANS ? (dt & 63) : dt;
+        const int dcol = TRANS ? (dt >> 6) : 0;
+        const float mu = p.qabs ? __ldg(p.dq_mean) : 0.f;
+        auto block_index = [&](int kt) -> int64_t {
+            return TRANS ? ((int64_t)kt * kBK + drow) * bpr + (m0 / 64) + dcol : (m0 + drow) * bpr + kt;
+        };
+        auto load_const = [&](int kt) -> float {
+            const int64_t jb = block_index(kt);
+            if (p.qabs) return dq_restore(__ldg(p.qabs + jb), __ldg(p.dq_scale + (jb >> 8)), mu);
+            return __ldg(p.absmax + jb);
+        };
+        float ah_next = p.KT > 0 ? load_const(0) : 0.f;
+        for (int kt = 0; kt < nsteps; ++kt) {
+            const int s = kt % kStages;
+            const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+            const float ah = ah_next;
+            if (kt + 1 < p.KT) ah_next = load_const(kt + 1);
+            if (!mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, kWaitLimitNs)) {
+                give_up();
+                break;
+            }
+            if (kt < p.KT) {
+                if (!mbar_wait_bounded(code_full(s), ph, abort_flag, kWaitLimitNs)) {
+                    give_up();
+                    break;
+                }
+                const uint8_t *cptr = smem + kOffC + s * kCBytes + (TRANS ? (drow * 64 + dcol * 32) : drow * 32);
+                const uint4 c0 = *reinterpret_cast<const uint4 *>(cptr);
+                const uint4 c1 = *reinterpret_cast<const uint4 *>(cptr + 16);
+                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                const NF4Table tab = nf4_table(ah);
+                uint8_t *abase = smem + kOffA + s * kABytes;
+                const int r8 = drow & 7;
+                // fwd (K-major): row drow at (drow/8)*1024 + (drow%8)*128, chunk c (K 8c..8c+7)
+                // dX (MN-major): atom (dcol, drow/8) at dcol*8192 + (drow/8)*1024, K-row drow%8,
+                //   chunk c = M elements 8c..8c+7.  Both: chunk position c ^ (row % 8).
+                uint8_t *rowp = abase + (TRANS ? dcol * 8192 : 0) + (drow >> 3) * 1024 + r8 * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(rowp + ((c ^ r8) << 4)) = nf4_decode8(cw[c], tab);
+                fence_proxy_async_smem();
+            }
+            mbar_arrive(dec_full(s));
+        }
+
+        // ------------------------------------------------------------ epilogue
+        // The go / no-go decision is made uniform across the 128 decoder
+        // threads (tcgen05.ld is warp-collective, bar 1 counts all of them).
+        if (*abort_flag || !mbar_wait_bounded(accum_full, 0, abort_flag, kWaitLimitNs)) give_up();
+        volatile int *epi_go = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (dt == 0) *epi_go = *abort_flag ? 0 : 1;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (*epi_go) {
+            tc_fence_after();
+            const int q = warp & 3;  // TMEM lane quadrant of this warp
+            uint16_t *Os = reinterpret_cast<uint16_t *>(smem + kOffA);  // [BN][128] bf16, all MMAs are done
+            const int m = q * 32 + lane;
+            for (int c0 = 0; c0 < p.BN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    Os[(c0 + j) * kBM + m] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            const int chunks = p.BN * (kBM / 8);
+            for (int idx = dt; idx < chunks; idx += kDecThreads) {
+                const int row = idx >> 4, ch = idx & 15;
+                const int64_t t = t0 + row;
+                if (t < p.n)
+                    *reinterpret_cast<uint4 *>(p.out + t * p.out_ld + m0 + 8 * ch) =
+                        *reinterpret_cast<const uint4 *>(Os + row * kBM + 8 * ch);
+            }
+        }
+    }
+
+    // Teardown: all MMAs must have retired before TMEM is released.
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        if (lane == 0 && !mbar_wait_bounded(accum_full, 0, nullptr, kWaitLimitNs)) give_up();
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_d, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps (driver entry point fetched through the runtime, so
+// the library does not link libcuda), launch.
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2D map over a row-major [outer][inner] array.
+static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t inner,
+                     uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * (uint64_t)esize};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+bool nf4_tc_gemm_supported(const qln_nf4_weight *w, bool trans, int64_t n, int r) {
+    const int64_t M = trans ? w->cols : w->rows;
+    const int64_t K = trans ? w->rows : w->cols;
+    return n >= 64 && (M % tc::kBM) == 0 && (K % tc::kBK) == 0 && r >= 8 && r <= 128 && (r % 8) == 0 &&
+           tc::encode_fn() != nullptr;
+}
+
+cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16_t *act, int64_t n,
+                               const uint16_t *lact, const uint16_t *lw, int r, uint16_t *out, int *status,
+                               cudaStream_t st, int num_sms) {
+    (void)num_sms;
+    using namespace tc;
+    const int64_t rows = w->rows, cols = w->cols;
+    const int64_t M = trans ? cols : rows;
+    const int64_t K = trans ? rows : cols;
+    int BN = n >= kMaxBN ? kMaxBN : (int)((n + 15) / 16 * 16);
+    CUtensorMap m_codes, m_act, m_lw, m_lact;
+    bool ok = true;
+    // codes as bytes [rows][cols/2]
+    if (!trans) ok &= make_map(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, cols / 2, rows, 32, kBM,
+                               CU_TENSOR_MAP_SWIZZLE_NONE);
+    else ok &= make_map(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, cols / 2, rows, 64, kBK,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok &= make_map(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, K, n, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!trans) ok &= make_map(&m_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lw, r, rows, kBK, kBM,
+                               CU_TENSOR_MAP_SWIZZLE_128B);                       // B [rows][r]
+    else ok &= make_map(&m_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lw, cols, r, 64, kBK,
+                        CU_TENSOR_MAP_SWIZZLE_128B);                               // A [r][cols]
+    ok &= make_map(&m_lact, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lact, r, n, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
+
+    Params p;
+    p.qabs = w->qabs;
+    p.absmax = w->absmax;
+    p.dq_scale = w->dq_scale;
+    p.dq_mean = w->dq_mean;
+    p.cols = cols;
+    p.n = n;
+    p.out = out;
+    p.out_ld = M;
+    p.status = status;
+    p.KT = (int)(K / kBK);
+    p.RT = (r + kBK - 1) / kBK;
+    p.BN = BN;
+    dim3 grid((unsigned)((n + BN - 1) / BN), (unsigned)(M / kBM));
+    cudaError_t e;
+    if (trans) {
+        e = cudaFuncSetAttribute(nf4_tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        nf4_tc_gemm_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(m_codes, m_act, m_lw, m_lact, p);
+        note_launch();
+    } else {
+        e = cudaFuncSetAttribute(nf4_tc_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        nf4_tc_gemm_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(m_codes, m_act, m_lw, m_lact, p);
+        note_launch();
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace qln

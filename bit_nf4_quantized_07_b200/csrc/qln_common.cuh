@@ -20,15 +20,29 @@ namespace qln {
 // jjjymmm.cn post ("4-bit NormalFloat(NF4)").  Stored as bit patterns so the
 // values are exact; a CPU test compares them with an independent recomputation.
 // ---------------------------------------------------------------------------
-__host__ __device__ constexpr uint32_t kNF4Bits[16] = {
-    0xbf800000u, 0xbf3239b1u, 0xbf066b2eu, 0xbeca329eu, 0xbe91a24bu, 0xbe3d353du,
-    0xbdba7869u, 0x00000000u, 0x3da2fb01u, 0x3e24cadfu, 0x3e7c04dau, 0x3ead0336u,
-    0x3ee1a4b5u, 0x3f1007a9u, 0x3f3913b0u, 0x3f800000u};
+__host__ __device__ constexpr uint32_t nf4_bits(int q) {
+    return q == 0    ? 0xbf800000u
+           : q == 1  ? 0xbf3239b1u
+           : q == 2  ? 0xbf066b2eu
+           : q == 3  ? 0xbeca329eu
+           : q == 4  ? 0xbe91a24bu
+           : q == 5  ? 0xbe3d353du
+           : q == 6  ? 0xbdba7869u
+           : q == 7  ? 0x00000000u
+           : q == 8  ? 0x3da2fb01u
+           : q == 9  ? 0x3e24cadfu
+           : q == 10 ? 0x3e7c04dau
+           : q == 11 ? 0x3ead0336u
+           : q == 12 ? 0x3ee1a4b5u
+           : q == 13 ? 0x3f1007a9u
+           : q == 14 ? 0x3f3913b0u
+                     : 0x3f800000u;
+}
 
 constexpr int kBlock = 64;     // weights per absmax block
 constexpr int kDqGroup = 256;  // block constants per DQ scale
 
-__device__ __forceinline__ float nf4_value(int q) { return __uint_as_float(kNF4Bits[q]); }
+__device__ __forceinline__ float nf4_value(int q) { return __uint_as_float(nf4_bits(q)); }
 
 // Snap thresholds: t_k = the largest fp32 value <= (c_k + c_{k+1}) / 2.
 // For an fp32 x, x > t_k  <=>  x is strictly closer to c_{k+1} than to c_k,
@@ -111,5 +125,61 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 }
 
 __host__ __device__ constexpr int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+}  // namespace qln
+
+namespace qln {
+
+// ---------------------------------------------------------------------------
+// Register-only NF4 decode.  For one block constant ahat the 16 products
+// P[q] = bf16_RN(fp32(ahat * c[q])) are formed once and split into a table of
+// low bytes L[0..3] and high bytes H[0..3] (4 entries per register); a byte
+// permute (prmt) then looks up 4 codes at a time: the low 3 bits of each code
+// pick a byte within an 8-entry half-table, bit 3 picks the half.  Exactly the
+// doubleDequant value w' = bf16_RN(fp32(ahat * c[q])), with no shared-memory
+// traffic.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+struct NF4Table {
+    uint32_t L[4], H[4];
+};
+
+__device__ __forceinline__ NF4Table nf4_table(float ah) {
+    uint32_t T[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) T[i] = pack_bf16x2(__fmul_rn(ah, nf4_value(2 * i)), __fmul_rn(ah, nf4_value(2 * i + 1)));
+    NF4Table t;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        t.L[j] = prmt(T[2 * j], T[2 * j + 1], 0x6420u);  // low bytes of P[4j..4j+3]
+        t.H[j] = prmt(T[2 * j], T[2 * j + 1], 0x7531u);  // high bytes
+    }
+    return t;
+}
+
+// Four codes held in the low 16 bits of s (nibble order: element 1, 0, 3, 2 of
+// the two bytes) -> BF16 pairs (elements 0,1) and (2,3).
+__device__ __forceinline__ void nf4_decode4(uint32_t s, const NF4Table &t, uint32_t &e01, uint32_t &e23) {
+    const uint32_t i3 = s & 0x7777u;
+    const uint32_t sel = ((s >> 1) & 0x4444u) | 0x3210u;
+    const uint32_t lo = prmt(prmt(t.L[0], t.L[1], i3), prmt(t.L[2], t.L[3], i3), sel);
+    const uint32_t hi = prmt(prmt(t.H[0], t.H[1], i3), prmt(t.H[2], t.H[3], i3), sel);
+    e01 = prmt(lo, hi, 0x4051u);
+    e23 = prmt(lo, hi, 0x6273u);
+}
+
+// One 32-bit word of packed codes (8 weights, first in the high nibble of the
+// lowest byte) -> 8 BF16 values in memory order.
+__device__ __forceinline__ uint4 nf4_decode8(uint32_t w, const NF4Table &t) {
+    uint4 o;
+    nf4_decode4(w & 0xFFFFu, t, o.x, o.y);
+    nf4_decode4(w >> 16, t, o.z, o.w);
+    return o;
+}
 
 }  // namespace qln
