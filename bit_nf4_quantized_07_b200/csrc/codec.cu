@@ -15,22 +15,48 @@ namespace qln {
 // K1: quantize.  One warp streams 256 consecutive weights (4 blocks) per step:
 // lane l holds float4 #l and #(l+32), i.e. elements 4l..4l+3 of block l/16 and
 // of block 2 + l/16.  Each 16-lane half reduces its block's absmax with four
-// xor-shuffles; every element is divided by the absmax (IEEE fp32 division)
-// and snapped by counting the 15 thresholds it exceeds.
+// xor-shuffles and every element is divided by it (IEEE fp32 division, x in
+// [-1, 1]).
+// Snap without a 15-way compare: the top 12 bits of x (sign, exponent, three
+// mantissa bits) name an interval of fp32 values that contains at most one
+// snap threshold (the narrowest gap between thresholds, 0.08, is wider than
+// any such interval below 1 in magnitude).  A per-CTA table gives, for each
+// key, the code of the interval's smallest value and that one threshold (or
+// +inf), so  q = base[key] + (x > thr[key])  -- exactly #{k : x > t_k}.
 // ===========================================================================
-__device__ __forceinline__ uint32_t snap_pair(float w0, float w1, float a, const float (&t)[15]) {
+constexpr int kSnapKeys = 4096;
+
+__device__ __forceinline__ uint32_t snap_lut(float x, const uint2 *lut) {
+    const uint2 e = lut[__float_as_uint(x) >> 20];
+    return e.y + ((x > __uint_as_float(e.x)) ? 1u : 0u);
+}
+
+__device__ void build_snap_lut(uint2 *lut) {
+    float t[15];
+#pragma unroll
+    for (int k = 0; k < 15; ++k) t[k] = nf4_threshold(k);
+    for (int key = threadIdx.x; key < kSnapKeys; key += blockDim.x) {
+        const float a = __uint_as_float((uint32_t)key << 20);
+        const float b = __uint_as_float(((uint32_t)key << 20) | 0xFFFFFu);
+        const bool neg = (key & 0x800) != 0;
+        const float lo = neg ? b : a, hi = neg ? a : b;  // the interval [lo, hi] in value order
+        uint32_t base = 0, thr = 0x7f800000u;            // +inf: no threshold inside
+#pragma unroll
+        for (int k = 0; k < 15; ++k) {
+            if (lo > t[k]) ++base;
+            else if (t[k] < hi && thr == 0x7f800000u) thr = __float_as_uint(t[k]);
+        }
+        lut[key] = make_uint2(thr, base);
+    }
+}
+
+__device__ __forceinline__ uint32_t snap_pair(float w0, float w1, float a, const uint2 *lut) {
     float x0 = 0.f, x1 = 0.f;
     if (a > 0.f) {
         x0 = __fdiv_rn(w0, a);
         x1 = __fdiv_rn(w1, a);
     }
-    uint32_t q0 = 0, q1 = 0;
-#pragma unroll
-    for (int k = 0; k < 15; ++k) {
-        q0 += (x0 > t[k]) ? 1u : 0u;
-        q1 += (x1 > t[k]) ? 1u : 0u;
-    }
-    return (q0 << 4) | q1;  // first element in the high nibble
+    return (snap_lut(x0, lut) << 4) | snap_lut(x1, lut);  // first element in the high nibble
 }
 
 __device__ __forceinline__ float absmax4(float4 v) {
@@ -40,9 +66,9 @@ __device__ __forceinline__ float absmax4(float4 v) {
 __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float4 *__restrict__ W, int64_t nb,
                                                            uint16_t *__restrict__ codes16,
                                                            float *__restrict__ absmax) {
-    float t[15];
-#pragma unroll
-    for (int k = 0; k < 15; ++k) t[k] = nf4_threshold(k);
+    __shared__ uint2 lut[kSnapKeys];
+    build_snap_lut(lut);
+    __syncthreads();
 
     const int lane = threadIdx.x & 31;
     const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -62,12 +88,12 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float4 *__restr
             m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
         }
         if (b0 < nb) {
-            uint32_t p = snap_pair(v0.x, v0.y, m0, t) | (snap_pair(v0.z, v0.w, m0, t) << 8);
+            uint32_t p = snap_pair(v0.x, v0.y, m0, lut) | (snap_pair(v0.z, v0.w, m0, lut) << 8);
             __stcs(codes16 + 64 * c + lane, (uint16_t)p);
             if ((lane & 15) == 0) absmax[b0] = m0;
         }
         if (b1 < nb) {
-            uint32_t p = snap_pair(v1.x, v1.y, m1, t) | (snap_pair(v1.z, v1.w, m1, t) << 8);
+            uint32_t p = snap_pair(v1.x, v1.y, m1, lut) | (snap_pair(v1.z, v1.w, m1, lut) << 8);
             __stcs(codes16 + 64 * c + 32 + lane, (uint16_t)p);
             if ((lane & 15) == 0) absmax[b1] = m1;
         }
@@ -80,7 +106,7 @@ cudaError_t launch_nf4_quantize(const float *W, int64_t numel, uint8_t *codes, f
     const int64_t nchunks = (nb + 3) / 4;
     const int threads = 256;
     int64_t grid = (nchunks + 7) / 8;
-    const int64_t cap = (int64_t)num_sms * 8;  // 8 CTAs of 256 threads per SM
+    const int64_t cap = (int64_t)num_sms * 4;  // persistent-ish: the table is built once per CTA
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
     nf4_quantize_kernel<<<(unsigned)grid, threads, 0, st>>>(reinterpret_cast<const float4 *>(W), nb,

@@ -40,7 +40,7 @@ constexpr int kThreads = 192;
 constexpr int kDecThreads = 128;
 constexpr uint32_t kABytes = kBM * kBK * 2;      // 16 KB
 constexpr uint32_t kBBytes = kMaxBN * kBK * 2;   // 32 KB
-constexpr uint32_t kCBytes = 4096;               // 128 rows x 32 B (fwd) or 64 rows x 64 B (dX)
+constexpr uint32_t kCBytes = 4096;               // 128 rows x 32 B (fwd) or 2 x 64 rows x 32 B (dX)
 constexpr uint32_t kStageBytes = kABytes + kBBytes + kCBytes;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
@@ -138,8 +138,12 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 const uint32_t sC = sbase + kOffC + s * kCBytes;
                 if (kt < p.KT) {
                     mbar_arrive_expect_tx(code_full(s), kCBytes);
-                    if (!TRANS) tma_load_2d(sC, &tm_codes, kt * 32, (int32_t)m0, code_full(s));
-                    else tma_load_2d(sC, &tm_codes, (int32_t)(m0 / 2), kt * kBK, code_full(s));
+                    if (!TRANS) {
+                        tma_load_2d(sC, &tm_codes, kt * 32, (int32_t)m0, code_full(s));
+                    } else {  // two 64-row x 32-byte boxes: [column block][row][32 B]
+                        tma_load_2d(sC, &tm_codes, (int32_t)(m0 / 2), kt * kBK, code_full(s));
+                        tma_load_2d(sC + 2048, &tm_codes, (int32_t)(m0 / 2) + 32, kt * kBK, code_full(s));
+                    }
                     mbar_arrive_expect_tx(tma_full(s), bbytes);
                     tma_load_2d(sB, &tm_act, kt * kBK, (int32_t)t0, tma_full(s));
                 } else {
@@ -203,17 +207,35 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         auto block_index = [&](int kt) -> int64_t {
             return TRANS ? ((int64_t)kt * kBK + drow) * bpr + (m0 / 64) + dcol : (m0 + drow) * bpr + kt;
         };
-        auto load_const = [&](int kt) -> float {
-            const int64_t jb = block_index(kt);
-            if (p.qabs) return dq_restore(__ldg(p.qabs + jb), __ldg(p.dq_scale + (jb >> 8)), mu);
-            return __ldg(p.absmax + jb);
+        // Raw block constants are fetched two k-steps before use so that their
+        // L2 latency hides behind the decode of the steps in between.
+        struct Raw {
+            float v;     // absmax (plain) or DQ scale b_g
+            int32_t q;   // DQ code rhat_j
         };
-        float ah_next = p.KT > 0 ? load_const(0) : 0.f;
+        auto fetch = [&](int kt) -> Raw {
+            Raw r{0.f, 0};
+            if (kt < p.KT) {
+                const int64_t jb = block_index(kt);
+                if (p.qabs) {
+                    r.q = __ldg(p.qabs + jb);
+                    r.v = __ldg(p.dq_scale + (jb >> 8));
+                } else {
+                    r.v = __ldg(p.absmax + jb);
+                }
+            }
+            return r;
+        };
+        Raw r0 = fetch(0), r1 = fetch(1);
+        // code bytes of this thread: 32 B at a 32 B stride; the two 16 B halves
+        // are read in an order that keeps each 8-thread phase on distinct banks
+        const int cfirst = (drow >> 2) & 1;
         for (int kt = 0; kt < nsteps; ++kt) {
             const int s = kt % kStages;
             const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
-            const float ah = ah_next;
-            if (kt + 1 < p.KT) ah_next = load_const(kt + 1);
+            const float ah = p.qabs ? dq_restore((int8_t)r0.q, r0.v, mu) : r0.v;
+            r0 = r1;
+            r1 = fetch(kt + 2);
             if (!mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, kWaitLimitNs)) {
                 give_up();
                 break;
@@ -223,9 +245,10 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                     give_up();
                     break;
                 }
-                const uint8_t *cptr = smem + kOffC + s * kCBytes + (TRANS ? (drow * 64 + dcol * 32) : drow * 32);
-                const uint4 c0 = *reinterpret_cast<const uint4 *>(cptr);
-                const uint4 c1 = *reinterpret_cast<const uint4 *>(cptr + 16);
+                const uint8_t *cptr = smem + kOffC + s * kCBytes + (TRANS ? (dcol * 2048 + drow * 32) : drow * 32);
+                const uint4 ca = *reinterpret_cast<const uint4 *>(cptr + 16 * cfirst);
+                const uint4 cb = *reinterpret_cast<const uint4 *>(cptr + 16 * (cfirst ^ 1));
+                const uint4 c0 = cfirst ? cb : ca, c1 = cfirst ? ca : cb;
                 const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                 const NF4Table tab = nf4_table(ah);
                 uint8_t *abase = smem + kOffA + s * kABytes;
@@ -342,7 +365,7 @@ cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16
     // codes as bytes [rows][cols/2]
     if (!trans) ok &= make_map(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, cols / 2, rows, 32, kBM,
                                CU_TENSOR_MAP_SWIZZLE_NONE);
-    else ok &= make_map(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, cols / 2, rows, 64, kBK,
+    else ok &= make_map(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, cols / 2, rows, 32, kBK,
                         CU_TENSOR_MAP_SWIZZLE_NONE);
     ok &= make_map(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, K, n, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!trans) ok &= make_map(&m_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lw, r, rows, kBK, kBM,
