@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "QLN_OK", 1: "QLN_ERR_NULL", 2: "QLN_ERR_SHAPE", 3: "QLN_ERR_
 OP_DOUBLE_QUANT, OP_LINEAR_FWD, OP_LINEAR_BWD = 1, 2, 3
 
 #: Every symbol include/qlora_nf4.h declares.
-EXPORTS = ("nf4_quantize", "nf4_double_quant", "nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd",
+EXPORTS = ("nf4_quantize", "nf4_double_quant", "nf4_double_quant_noalloc", "nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd",
            "qln_workspace_bytes", "qln_codebook", "qln_status_str", "qln_version", "qln_launch_count")
 
 
@@ -56,6 +56,7 @@ def lib():
         sig = {
             "nf4_quantize": ([P, I64, P, P, P], I32),
             "nf4_double_quant": ([P, I64, P, P, P, P, SZ, P], I32),
+            "nf4_double_quant_noalloc": ([P, I64, P, P, P, P], I32),
             "nf4_dequant": ([WP, P, P], I32),
             "qlora_linear_fwd": ([WP, P, I64, P, P, I32, F, P, P, P, SZ, P], I32),
             "qlora_linear_bwd": ([WP, P, I64, P, P, I32, F, P, P, P, P, P, P, SZ, P], I32),
@@ -168,6 +169,16 @@ def nf4_double_quant(absmax: torch.Tensor, qabs=None, dq_scale=None, dq_mean=Non
     _need_cuda(absmax, qabs, dq_scale, dq_mean, ws)
     _check("nf4_double_quant", lib().nf4_double_quant(_p(absmax), nb, _p(qabs), _p(dq_scale), _p(dq_mean), _p(ws),
                                                       ws.numel(), _stream()))
+    return qabs, dq_scale, dq_mean
+
+
+def nf4_double_quant_noalloc(absmax: torch.Tensor, qabs, dq_scale, dq_mean):
+    """nf4_double_quant into caller-provided outputs, with no device workspace:
+    for callers that cannot allocate device memory (see the header)."""
+    nb = absmax.numel()
+    _need_cuda(absmax, qabs, dq_scale, dq_mean)
+    _check("nf4_double_quant_noalloc", lib().nf4_double_quant_noalloc(_p(absmax), nb, _p(qabs), _p(dq_scale),
+                                                                      _p(dq_mean), _stream()))
     return qabs, dq_scale, dq_mean
 
 

@@ -156,6 +156,18 @@ qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float
     return from_cuda(qln::launch_nf4_double_quant(absmax, nb, qabs, dq_scale, dq_mean, ws, (cudaStream_t)stream));
 }
 
+qln_status nf4_double_quant_noalloc(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale,
+                                    float *dq_mean, void *stream) {
+    if (!absmax || !qabs || !dq_scale || !dq_mean) return QLN_ERR_NULL;
+    if (nb <= 0 || nb > qln::dq_static_max_blocks()) return QLN_ERR_SHAPE;
+    if (!aligned(absmax, 16) || !aligned(qabs, 4) || !aligned(dq_scale, 4) || !aligned(dq_mean, 4))
+        return QLN_ERR_ALIGN;
+    int sms = 0;
+    qln_status s = check_device(&sms);
+    if (s != QLN_OK) return s;
+    return from_cuda(qln::launch_nf4_double_quant_static(absmax, nb, qabs, dq_scale, dq_mean, (cudaStream_t)stream));
+}
+
 qln_status nf4_dequant(const qln_nf4_weight *w, uint16_t *out, void *stream) {
     qln_status s = check_weight(w);
     if (s != QLN_OK) return s;

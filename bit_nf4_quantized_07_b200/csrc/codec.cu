@@ -6,6 +6,8 @@
 // "Double Quantization" and "QLoRA" (doubleDequant: constants first);
 // "LoRA 与 QLoRA" section QLoRA 2 (a_j = max|W_j| per 64 weights,
 // r_j = (a_j - mu)/b, 8-bit rhat_j, ahat_j = mu + b rhat_j).
+#include <atomic>
+
 #include "qln_common.cuh"
 #include "qln_internal.h"
 
@@ -288,6 +290,63 @@ cudaError_t launch_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qab
     dq_partial_kernel<<<np, kMeanThreads, 0, st>>>(absmax, nb, partial);
     note_launch();
     cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
+    const int64_t grid = (ng + (kDqThreads / 32) - 1) / (kDqThreads / 32);
+    dq_quant_kernel<<<(unsigned)grid, kDqThreads, 0, st>>>(absmax, nb, partial, np, np2, qabs, scale, mu);
+    note_launch();
+    return cudaGetLastError();
+}
+
+// ===========================================================================
+// Allocation-free double quantization.  The only scratch K2/K3 need is the
+// binary64 partial sums of mu, one per 8192 block constants.  This variant
+// keeps them in a fixed, file-scope device array instead of a caller
+// workspace, so a caller that cannot allocate device memory can still run the
+// path.  The array is 8 KB (1024 partials), which caps nb at 1024 * 8192 =
+// 8,388,608 blocks (536,870,912 weights); every GPU that loads the library
+// holds it until the process exits.  Each call overwrites every partial it
+// reads before reading it, so nothing has to be cleared between calls; two
+// calls that overlap on the GPU (different streams, no ordering) share the
+// array and race.
+// ===========================================================================
+constexpr int kStaticPartials = 1024;
+static __device__ __align__(256) double g_dq_static_partials[kStaticPartials];
+static std::atomic<double *> g_dq_static_ptr[64];
+
+int64_t dq_static_max_blocks() { return (int64_t)kStaticPartials * kMeanChunk; }
+
+// Device address of the array on the current device.  In host code the
+// symbol names a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+static cudaError_t dq_static_partials(double **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    double *p = g_dq_static_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        void *addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, g_dq_static_partials);
+        if (e != cudaSuccess) return e;
+        p = static_cast<double *>(addr);
+        g_dq_static_ptr[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return cudaSuccess;
+}
+
+cudaError_t launch_nf4_double_quant_static(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,
+                                           cudaStream_t st) {
+    double *partial = nullptr;
+    cudaError_t e = dq_static_partials(&partial);
+    if (e != cudaSuccess) return e;
+    const int np = (int)((nb + kMeanChunk - 1) / kMeanChunk);
+    int np2 = 1;
+    while (np2 < np) np2 <<= 1;
+    dq_partial_kernel<<<np, kMeanThreads, 0, st>>>(absmax, nb, partial);
+    note_launch();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
     const int64_t grid = (ng + (kDqThreads / 32) - 1) / (kDqThreads / 32);

@@ -19,6 +19,10 @@ cudaError_t launch_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qab
                                     void *ws, cudaStream_t st);
 cudaError_t launch_nf4_dequant(const qln_nf4_weight *w, uint16_t *out, cudaStream_t st, int num_sms);
 size_t dq_workspace_bytes(int64_t nb);
+// allocation-free variant: scratch in a file-scope device array (codec.cu)
+cudaError_t launch_nf4_double_quant_static(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,
+                                           cudaStream_t st);
+int64_t dq_static_max_blocks();
 int64_t dq_max_blocks();
 
 // lora_small.cu: skinny products around the adapters.

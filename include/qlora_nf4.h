@@ -133,6 +133,32 @@ QLN_API qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qab
                             float *dq_mean, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * nf4_double_quant_noalloc -- nf4_double_quant without a caller workspace.
+ * The pages describe nothing like it: it exists for callers that cannot
+ * allocate device memory at the point where they quantize -- for example a
+ * runtime that reserves all device memory up front in its own pool and
+ * forbids further cudaMalloc, or a plugin that only receives tensors from a
+ * host framework and has no allocator of its own.  It computes exactly what
+ * nf4_double_quant computes (same kernels, same bits) and allocates nothing:
+ * it calls no cudaMalloc, cudaFree or other allocating routine.
+ *   Scratch: an 8 KB array of binary64 partial sums at file scope in the
+ *   library, present on every GPU that loads it until the process exits.
+ *   Limit: nb <= 8,388,608 block constants (weights <= 536,870,912); larger
+ *   nb returns QLN_ERR_SHAPE before anything is launched.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture on that device.
+ *   Sharing: every call uses the same array.  Each call rewrites all of it
+ *   that it reads, so nothing carries over, but calls that overlap on the GPU
+ *   (e.g. on two unordered streams) race on it and must be serialised by the
+ *   caller.
+ * Arguments and outputs as nf4_double_quant.  Errors: QLN_ERR_NULL,
+ * QLN_ERR_SHAPE, QLN_ERR_ALIGN, QLN_ERR_ARCH, QLN_ERR_CUDA.
+ */
+QLN_API qln_status nf4_double_quant_noalloc(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale,
+                                            float *dq_mean, void *stream);
+
+/*
  * nf4_dequant -- doubleDequant of a whole weight to BF16.
  * Defined by: jjjymmm.cn "QLoRA" (restore the quantization constant first,
  * then dequantize the weight with it; a code dequantizes to its quant-book
