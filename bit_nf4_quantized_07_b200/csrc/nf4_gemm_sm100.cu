@@ -1,5 +1,5 @@
 // Fused NF4 doubleDequant + GEMM on the sm_100a tensor cores (tcgen05, TMEM
-// accumulator, TMA operand loads).  W' is decoded tile by tile into shared
+// accumulators, TMA operand loads).  W' is decoded tile by tile into shared
 // memory and never reaches HBM.
 //
 // Method: "LoRA 与 QLoRA" section QLoRA 1 (4-bit weight -> dequant -> BF16 ->
@@ -11,16 +11,19 @@
 //   forward (TRANS = false): out[t][m] = sum_k X[t][k] W'[m][k]  + sum_j sU[t][j] B[m][j]
 //   dX      (TRANS = true) : out[t][m] = sum_k dY[t][k] W'[k][m] + sum_j sG[t][j] A[j][m]
 //
-// One CTA computes a 128 (m) x BN (tokens, <= 256) tile: D = A_op * B_op^T in
-// TMEM with M = 128 (m), N = BN (tokens), K in steps of 64.
-//   A_op (weights): decoded by 4 warps into the canonical 128-byte-swizzled
-//     layout, K-major for the forward (W' rows along K) and MN-major for dX
-//     (W' rows are the K index, their 128 consecutive columns the M index);
+// One CTA computes a (128*MT) (m) x BN (tokens, <= 256) tile as MT
+// accumulators of 128 TMEM lanes x BN columns, K in steps of 64.  MT = 2 lets
+// two 128-row weight tiles share every activation tile, halving the
+// activation bytes each FLOP pulls from L2.
+//   A_op (weights): decoded by 128*MT threads (one 64-wide row block each)
+//     into the canonical 128-byte-swizzled layout, K-major for the forward
+//     (W' rows along K) and MN-major for dX (W' rows are the K index, their
+//     consecutive columns the M index);
 //   B_op (activations X / dY, K-major): TMA tiles with 128-byte swizzle;
 //   the adapter term is extra K steps whose A_op (B or A, zero-padded to 64)
 //     and B_op (s*U or s*G) both arrive by TMA.
 // Warp roles: warp 0 TMA producer, warp 1 TMEM owner + single-thread MMA
-// issuer, warps 2-5 decoders and then the epilogue (TMEM -> BF16 -> HBM).
+// issuer, warps 2.. decoders and then the epilogue (TMEM -> BF16 -> HBM).
 // Every barrier wait is bounded; on give-up the CTA records QLN_ERR_TIMEOUT
 // in the status word, drains its own copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -32,28 +35,29 @@
 namespace qln {
 namespace tc {
 
-constexpr int kStages = 4;
-constexpr int kBM = 128;
+constexpr int kBM = 128;   // rows per accumulator (TMEM lanes)
 constexpr int kBK = 64;
 constexpr int kMaxBN = 256;
-constexpr int kThreads = 192;
-constexpr int kDecThreads = 128;
-constexpr uint32_t kABytes = kBM * kBK * 2;      // 16 KB
-constexpr uint32_t kBBytes = kMaxBN * kBK * 2;   // 32 KB
-constexpr uint32_t kCBytes = 4096;               // 128 rows x 32 B (fwd) or 2 x 64 rows x 32 B (dX)
-constexpr uint32_t kStageBytes = kABytes + kBBytes + kCBytes;
-constexpr uint32_t kTmemCols = 256;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
 
-// shared-memory map (offsets from a 1024-aligned base)
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + kStages * kABytes;
-constexpr uint32_t kOffC = kOffB + kStages * kBBytes;
-constexpr uint32_t kOffBar = kOffC + kStages * kCBytes;
-// barriers: tma_full[S], code_full[S], dec_full[S], empty[S], accum_full
-constexpr uint32_t kNumBars = 4 * kStages + 1;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem base (u32), abort flag (int)
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
+template <int MT>
+struct Cfg {
+    static constexpr int kStages = MT == 1 ? 4 : 3;
+    static constexpr int kDecThreads = 128 * MT;
+    static constexpr int kThreads = 64 + kDecThreads;
+    static constexpr uint32_t kABytes = 16384u * MT;       // MT x (128 rows x 64 K) bf16
+    static constexpr uint32_t kBBytes = kMaxBN * kBK * 2;  // 32 KB
+    static constexpr uint32_t kCBytes = 4096u * MT;        // codes of the A tile
+    static constexpr uint32_t kTmemCols = 256u * MT;
+    static constexpr uint32_t kOffA = 0;
+    static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
+    static constexpr uint32_t kOffC = kOffB + kStages * kBBytes;
+    static constexpr uint32_t kOffBar = kOffC + kStages * kCBytes;
+    // barriers: tma_full[S], code_full[S], dec_full[S], empty[S], accum_full
+    static constexpr uint32_t kNumBars = 4 * kStages + 1;
+    static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag, epilogue go
+    static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+};
 
 struct Params {
     const int8_t *qabs;
@@ -70,33 +74,37 @@ struct Params {
     int BN;            // tokens per tile (multiple of 16, <= 256)
 };
 
-template <bool TRANS>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool TRANS, int MT>
+__global__ void __launch_bounds__(Cfg<MT>::kThreads, 1)
 nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_act,
                    const __grid_constant__ CUtensorMap tm_lw, const __grid_constant__ CUtensorMap tm_lact,
                    const Params p) {
+    using C = Cfg<MT>;
+    constexpr int S = C::kStages;
+    constexpr int TM = kBM * MT;  // rows of the CTA tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
-    const uint32_t bar0 = sbase + kOffBar;
+    const uint32_t bar0 = sbase + C::kOffBar;
     auto tma_full = [&](int s) { return bar0 + 8u * s; };
-    auto code_full = [&](int s) { return bar0 + 8u * (kStages + s); };
-    auto dec_full = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
-    auto empty = [&](int s) { return bar0 + 8u * (3 * kStages + s); };
-    const uint32_t accum_full = bar0 + 8u * (4 * kStages);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+    auto code_full = [&](int s) { return bar0 + 8u * (S + s); };
+    auto dec_full = [&](int s) { return bar0 + 8u * (2 * S + s); };
+    auto empty = [&](int s) { return bar0 + 8u * (3 * S + s); };
+    const uint32_t accum_full = bar0 + 8u * (4 * S);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 4);
+    volatile int *epi_go = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * p.BN;
-    const int64_t m0 = (int64_t)blockIdx.y * kBM;
+    const int64_t m0 = (int64_t)blockIdx.y * TM;
     const int nsteps = p.KT + p.RT;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(tma_full(s), 1);
             mbar_init(code_full(s), 1);
-            mbar_init(dec_full(s), kDecThreads);
+            mbar_init(dec_full(s), C::kDecThreads);
             mbar_init(empty(s), 1);
         }
         mbar_init(accum_full, 1);
@@ -108,7 +116,7 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         tma_prefetch_map(&tm_lact);
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+        tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -127,42 +135,44 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             const uint32_t bbytes = (uint32_t)p.BN * kBK * 2;
             int issued = 0;
             for (int kt = 0; kt < nsteps; ++kt) {
-                const int s = kt % kStages;
-                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                const int s = kt % S;
+                const uint32_t ph = (uint32_t)(kt / S) & 1u;
                 if (!mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, kWaitLimitNs)) {
                     give_up();
                     break;
                 }
-                const uint32_t sA = sbase + kOffA + s * kABytes;
-                const uint32_t sB = sbase + kOffB + s * kBBytes;
-                const uint32_t sC = sbase + kOffC + s * kCBytes;
+                const uint32_t sA = sbase + C::kOffA + s * C::kABytes;
+                const uint32_t sB = sbase + C::kOffB + s * C::kBBytes;
+                const uint32_t sC = sbase + C::kOffC + s * C::kCBytes;
                 if (kt < p.KT) {
-                    mbar_arrive_expect_tx(code_full(s), kCBytes);
-                    if (!TRANS) {
+                    mbar_arrive_expect_tx(code_full(s), C::kCBytes);
+                    if (!TRANS) {  // TM rows x 32 bytes
                         tma_load_2d(sC, &tm_codes, kt * 32, (int32_t)m0, code_full(s));
-                    } else {  // two 64-row x 32-byte boxes: [column block][row][32 B]
-                        tma_load_2d(sC, &tm_codes, (int32_t)(m0 / 2), kt * kBK, code_full(s));
-                        tma_load_2d(sC + 2048, &tm_codes, (int32_t)(m0 / 2) + 32, kt * kBK, code_full(s));
+                    } else {       // 2*MT boxes of 64 rows x 32 bytes: [column block][row][32 B]
+#pragma unroll
+                        for (int d = 0; d < 2 * MT; ++d)
+                            tma_load_2d(sC + 2048 * d, &tm_codes, (int32_t)(m0 / 2) + 32 * d, kt * kBK, code_full(s));
                     }
                     mbar_arrive_expect_tx(tma_full(s), bbytes);
                     tma_load_2d(sB, &tm_act, kt * kBK, (int32_t)t0, tma_full(s));
                 } else {
                     const int a = kt - p.KT;
-                    mbar_arrive_expect_tx(tma_full(s), kABytes + bbytes);
+                    mbar_arrive_expect_tx(tma_full(s), C::kABytes + bbytes);
                     if (!TRANS) {
-                        tma_load_2d(sA, &tm_lw, a * kBK, (int32_t)m0, tma_full(s));
+                        tma_load_2d(sA, &tm_lw, a * kBK, (int32_t)m0, tma_full(s));  // TM rows x 64
                     } else {
-                        tma_load_2d(sA, &tm_lw, (int32_t)m0, a * kBK, tma_full(s));
-                        tma_load_2d(sA + 8192, &tm_lw, (int32_t)m0 + 64, a * kBK, tma_full(s));
+#pragma unroll
+                        for (int d = 0; d < 2 * MT; ++d)
+                            tma_load_2d(sA + 8192 * d, &tm_lw, (int32_t)m0 + 64 * d, a * kBK, tma_full(s));
                     }
                     tma_load_2d(sB, &tm_lact, a * kBK, (int32_t)t0, tma_full(s));
                 }
                 issued = kt + 1;
             }
             // Drain: every issued copy has landed before the CTA may exit.
-            for (int kt = (issued > kStages ? issued - kStages : 0); kt < issued; ++kt) {
-                const int s = kt % kStages;
-                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+            for (int kt = (issued > S ? issued - S : 0); kt < issued; ++kt) {
+                const int s = kt % S;
+                const uint32_t ph = (uint32_t)(kt / S) & 1u;
                 if (!mbar_wait_bounded(tma_full(s), ph, nullptr, kWaitLimitNs)) give_up();
                 if (kt < p.KT && !mbar_wait_bounded(code_full(s), ph, nullptr, kWaitLimitNs)) give_up();
             }
@@ -172,24 +182,28 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(kBM, p.BN, TRANS, false);
             for (int kt = 0; kt < nsteps; ++kt) {
-                const int s = kt % kStages;
-                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                const int s = kt % S;
+                const uint32_t ph = (uint32_t)(kt / S) & 1u;
                 if (!mbar_wait_bounded(tma_full(s), ph, abort_flag, kWaitLimitNs) ||
                     !mbar_wait_bounded(dec_full(s), ph, abort_flag, kWaitLimitNs)) {
                     give_up();
                     break;
                 }
                 tc_fence_after();
-                const uint32_t sA = sbase + kOffA + s * kABytes;
-                const uint32_t sB = sbase + kOffB + s * kBBytes;
+                const uint32_t sA = sbase + C::kOffA + s * C::kABytes;
+                const uint32_t sB = sbase + C::kOffB + s * C::kBBytes;
 #pragma unroll
-                for (int k = 0; k < kBK / 16; ++k) {
-                    // K-major: next 16 K elements are 32 bytes further inside the
-                    // swizzled 128-byte rows.  MN-major: next two 8-row K groups.
-                    const uint64_t adesc = TRANS ? smem_desc_sw128(sA + k * 2048, 8192, 1024)
-                                                 : smem_desc_sw128(sA + k * 32, 16, 1024);
-                    const uint64_t bdesc = smem_desc_sw128(sB + k * 32, 16, 1024);
-                    tc_mma_ss(tmem_d, adesc, bdesc, idesc, (kt | k) != 0 ? 1u : 0u);
+                for (int sub = 0; sub < MT; ++sub) {
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        // K-major: next 16 K elements are 32 bytes further inside the
+                        // swizzled 128-byte rows.  MN-major: next two 8-row K groups.
+                        const uint32_t aS = sA + sub * 16384;
+                        const uint64_t adesc = TRANS ? smem_desc_sw128(aS + k * 2048, 8192, 1024)
+                                                     : smem_desc_sw128(aS + k * 32, 16, 1024);
+                        const uint64_t bdesc = smem_desc_sw128(sB + k * 32, 16, 1024);
+                        tc_mma_ss(tmem_d + sub * 256, adesc, bdesc, idesc, (kt | k) != 0 ? 1u : 0u);
+                    }
                 }
                 tc_commit(empty(s));
             }
@@ -197,9 +211,10 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         }
     } else {
         // ------------------------------------------------------------ decoders
-        const int dt = threadIdx.x - 64;  // 0..127
-        // fwd: thread = W row m0+dt, block column kt.  dX: thread = W row
-        // 64*kt + (dt % 64), block column m0/64 + dt/64.
+        // One thread per 64-wide row block of the A tile.
+        //   fwd: block = W row m0 + dt, column block kt.
+        //   dX : block = W row 64*kt + dt%64, column block m0/64 + dt/64.
+        const int dt = threadIdx.x - 64;
         const int64_t bpr = p.cols / 64;
         const int drow = TRANS ? (dt & 63) : dt;
         const int dcol = TRANS ? (dt >> 6) : 0;
@@ -227,12 +242,19 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             return r;
         };
         Raw r0 = fetch(0), r1 = fetch(1);
-        // code bytes of this thread: 32 B at a 32 B stride; the two 16 B halves
-        // are read in an order that keeps each 8-thread phase on distinct banks
+        // This thread's 32 code bytes sit at a 32-byte stride; the two 16-byte
+        // halves are read in an order that keeps each 8-thread phase on
+        // distinct banks.
         const int cfirst = (drow >> 2) & 1;
+        const uint32_t code_off = (TRANS ? dcol * 2048 : 0) + drow * 32;
+        const int r8 = drow & 7;
+        // fwd (K-major): row drow at (drow/8)*1024 + (drow%8)*128, chunk c (K 8c..8c+7).
+        // dX (MN-major): atom (dcol, drow/8) at dcol*8192 + (drow/8)*1024, K-row drow%8,
+        //   chunk c = M elements 8c..8c+7.  Both: chunk position c ^ (row % 8).
+        const uint32_t row_off = (TRANS ? dcol * 8192 : 0) + (drow >> 3) * 1024 + r8 * 128;
         for (int kt = 0; kt < nsteps; ++kt) {
-            const int s = kt % kStages;
-            const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+            const int s = kt % S;
+            const uint32_t ph = (uint32_t)(kt / S) & 1u;
             const float ah = p.qabs ? dq_restore((int8_t)r0.q, r0.v, mu) : r0.v;
             r0 = r1;
             r1 = fetch(kt + 2);
@@ -245,18 +267,13 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                     give_up();
                     break;
                 }
-                const uint8_t *cptr = smem + kOffC + s * kCBytes + (TRANS ? (dcol * 2048 + drow * 32) : drow * 32);
+                const uint8_t *cptr = smem + C::kOffC + s * C::kCBytes + code_off;
                 const uint4 ca = *reinterpret_cast<const uint4 *>(cptr + 16 * cfirst);
                 const uint4 cb = *reinterpret_cast<const uint4 *>(cptr + 16 * (cfirst ^ 1));
                 const uint4 c0 = cfirst ? cb : ca, c1 = cfirst ? ca : cb;
                 const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                 const NF4Table tab = nf4_table(ah);
-                uint8_t *abase = smem + kOffA + s * kABytes;
-                const int r8 = drow & 7;
-                // fwd (K-major): row drow at (drow/8)*1024 + (drow%8)*128, chunk c (K 8c..8c+7)
-                // dX (MN-major): atom (dcol, drow/8) at dcol*8192 + (drow/8)*1024, K-row drow%8,
-                //   chunk c = M elements 8c..8c+7.  Both: chunk position c ^ (row % 8).
-                uint8_t *rowp = abase + (TRANS ? dcol * 8192 : 0) + (drow >> 3) * 1024 + r8 * 128;
+                uint8_t *rowp = smem + C::kOffA + s * C::kABytes + row_off;
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
                     *reinterpret_cast<uint4 *>(rowp + ((c ^ r8) << 4)) = nf4_decode8(cw[c], tab);
@@ -266,34 +283,36 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         }
 
         // ------------------------------------------------------------ epilogue
-        // The go / no-go decision is made uniform across the 128 decoder
-        // threads (tcgen05.ld is warp-collective, bar 1 counts all of them).
+        // The go / no-go decision is made uniform across the decoder threads
+        // (tcgen05.ld is warp-collective, named barrier 1 counts all of them).
         if (*abort_flag || !mbar_wait_bounded(accum_full, 0, abort_flag, kWaitLimitNs)) give_up();
-        volatile int *epi_go = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(C::kDecThreads) : "memory");
         if (dt == 0) *epi_go = *abort_flag ? 0 : 1;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(C::kDecThreads) : "memory");
         if (*epi_go) {
             tc_fence_after();
-            const int q = warp & 3;  // TMEM lane quadrant of this warp
-            uint16_t *Os = reinterpret_cast<uint16_t *>(smem + kOffA);  // [BN][128] bf16, all MMAs are done
-            const int m = q * 32 + lane;
+            const int q = warp & 3;              // TMEM lane quadrant of this warp
+            const int sub = (warp - 2) >> 2;     // accumulator of this warp
+            uint16_t *Os = reinterpret_cast<uint16_t *>(smem);  // [BN][TM] bf16; all MMAs are done
+            const int m = sub * kBM + q * 32 + lane;
             for (int c0 = 0; c0 < p.BN; c0 += 32) {
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+                tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)(sub * 256 + c0), v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                    Os[(c0 + j) * kBM + m] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+                    if (c0 + j < p.BN)
+                        Os[(c0 + j) * TM + m] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            const int chunks = p.BN * (kBM / 8);
-            for (int idx = dt; idx < chunks; idx += kDecThreads) {
-                const int row = idx >> 4, ch = idx & 15;
+            asm volatile("bar.sync 1, %0;" ::"n"(C::kDecThreads) : "memory");
+            constexpr int kChunksPerRow = TM / 8;
+            const int chunks = p.BN * kChunksPerRow;
+            for (int idx = dt; idx < chunks; idx += C::kDecThreads) {
+                const int row = idx / kChunksPerRow, ch = idx % kChunksPerRow;
                 const int64_t t = t0 + row;
                 if (t < p.n)
                     *reinterpret_cast<uint4 *>(p.out + t * p.out_ld + m0 + 8 * ch) =
-                        *reinterpret_cast<const uint4 *>(Os + row * kBM + 8 * ch);
+                        *reinterpret_cast<const uint4 *>(Os + row * TM + 8 * ch);
             }
         }
     }
@@ -305,13 +324,13 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         if (lane == 0 && !mbar_wait_bounded(accum_full, 0, nullptr, kWaitLimitNs)) give_up();
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem_d, kTmemCols);
+        tmem_dealloc(tmem_d, C::kTmemCols);
     }
 }
 
 // ---------------------------------------------------------------------------
 // Host side: tensor maps (driver entry point fetched through the runtime, so
-// the library does not link libcuda), launch.
+// the library does not link libcuda), tile-shape choice, launch.
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -342,6 +361,41 @@ static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const vo
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tokens per tile: a multiple of 16 in [128, 256] (or all of n when n <= 256)
+// chosen to waste the least on the last partial wave of CTAs (one CTA per SM)
+// and on padding the last token tile, preferring wide tiles.
+static int choose_bn(int64_t n, int64_t mtiles, int num_sms) {
+    const int64_t n16 = (n + 15) / 16 * 16;
+    if (n16 <= kMaxBN) return (int)n16;
+    int best = kMaxBN;
+    double best_eff = -1.0;
+    for (int bn = kMaxBN; bn >= 128; bn -= 16) {
+        const int64_t ttiles = (n + bn - 1) / bn;
+        const int64_t tiles = ttiles * mtiles;
+        const int64_t rounds = (tiles + num_sms - 1) / num_sms;
+        // narrower tiles decode each weight for fewer tokens: a mild penalty
+        const double eff = ((double)tiles / (double)(rounds * num_sms)) * ((double)n / (double)(ttiles * bn)) -
+                           0.1 * (double)(kMaxBN - bn) / 128.0;
+        if (eff > best_eff + 1e-3) {
+            best_eff = eff;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+template <bool TRANS, int MT>
+static cudaError_t launch_t(const CUtensorMap &m_codes, const CUtensorMap &m_act, const CUtensorMap &m_lw,
+                            const CUtensorMap &m_lact, const Params &p, dim3 grid, cudaStream_t st) {
+    using C = Cfg<MT>;
+    cudaError_t e = cudaFuncSetAttribute(nf4_tc_gemm_kernel<TRANS, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    nf4_tc_gemm_kernel<TRANS, MT><<<grid, C::kThreads, C::kSmemBytes, st>>>(m_codes, m_act, m_lw, m_lact, p);
+    note_launch();
+    return cudaGetLastError();
+}
+
 }  // namespace tc
 
 bool nf4_tc_gemm_supported(const qln_nf4_weight *w, bool trans, int64_t n, int r) {
@@ -354,21 +408,22 @@ bool nf4_tc_gemm_supported(const qln_nf4_weight *w, bool trans, int64_t n, int r
 cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16_t *act, int64_t n,
                                const uint16_t *lact, const uint16_t *lw, int r, uint16_t *out, int *status,
                                cudaStream_t st, int num_sms) {
-    (void)num_sms;
     using namespace tc;
     const int64_t rows = w->rows, cols = w->cols;
     const int64_t M = trans ? cols : rows;
     const int64_t K = trans ? rows : cols;
-    int BN = n >= kMaxBN ? kMaxBN : (int)((n + 15) / 16 * 16);
+    const int MT = (M % 256) == 0 ? 2 : 1;
+    const int TM = kBM * MT;
+    const int BN = choose_bn(n, M / TM, num_sms > 0 ? num_sms : 148);
     CUtensorMap m_codes, m_act, m_lw, m_lact;
     bool ok = true;
     // codes as bytes [rows][cols/2]
-    if (!trans) ok &= make_map(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, cols / 2, rows, 32, kBM,
+    if (!trans) ok &= make_map(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, cols / 2, rows, 32, TM,
                                CU_TENSOR_MAP_SWIZZLE_NONE);
     else ok &= make_map(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, cols / 2, rows, 32, kBK,
                         CU_TENSOR_MAP_SWIZZLE_NONE);
     ok &= make_map(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, K, n, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (!trans) ok &= make_map(&m_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lw, r, rows, kBK, kBM,
+    if (!trans) ok &= make_map(&m_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lw, r, rows, kBK, TM,
                                CU_TENSOR_MAP_SWIZZLE_128B);                       // B [rows][r]
     else ok &= make_map(&m_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lw, cols, r, 64, kBK,
                         CU_TENSOR_MAP_SWIZZLE_128B);                               // A [r][cols]
@@ -388,20 +443,11 @@ cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16
     p.KT = (int)(K / kBK);
     p.RT = (r + kBK - 1) / kBK;
     p.BN = BN;
-    dim3 grid((unsigned)((n + BN - 1) / BN), (unsigned)(M / kBM));
-    cudaError_t e;
-    if (trans) {
-        e = cudaFuncSetAttribute(nf4_tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        nf4_tc_gemm_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(m_codes, m_act, m_lw, m_lact, p);
-        note_launch();
-    } else {
-        e = cudaFuncSetAttribute(nf4_tc_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        nf4_tc_gemm_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(m_codes, m_act, m_lw, m_lact, p);
-        note_launch();
-    }
-    return cudaGetLastError();
+    dim3 grid((unsigned)((n + BN - 1) / BN), (unsigned)(M / TM));
+    if (trans) return MT == 2 ? launch_t<true, 2>(m_codes, m_act, m_lw, m_lact, p, grid, st)
+                              : launch_t<true, 1>(m_codes, m_act, m_lw, m_lact, p, grid, st);
+    return MT == 2 ? launch_t<false, 2>(m_codes, m_act, m_lw, m_lact, p, grid, st)
+                   : launch_t<false, 1>(m_codes, m_act, m_lw, m_lact, p, grid, st);
 }
 
 }  // namespace qln
