@@ -244,14 +244,18 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         Raw r0 = fetch(0), r1 = fetch(1);
         // This thread's 32 code bytes sit at a 32-byte stride; the two 16-byte
         // halves are read in an order that keeps each 8-thread phase on
-        // distinct banks.
-        const int cfirst = (drow >> 2) & 1;
+        // distinct banks (half `cfirst` first).
+        const uint32_t cfirst = (drow >> 2) & 1;
         const uint32_t code_off = (TRANS ? dcol * 2048 : 0) + drow * 32;
-        const int r8 = drow & 7;
+        const uint32_t r8 = drow & 7;
         // fwd (K-major): row drow at (drow/8)*1024 + (drow%8)*128, chunk c (K 8c..8c+7).
         // dX (MN-major): atom (dcol, drow/8) at dcol*8192 + (drow/8)*1024, K-row drow%8,
-        //   chunk c = M elements 8c..8c+7.  Both: chunk position c ^ (row % 8).
+        //   chunk c = M elements 8c..8c+7.  Both: chunk c at byte (c ^ (row % 8)) * 16
+        // of the row.  Bits 4-6 of the row's address are zero, so the chunk
+        // address is (row address + 16*r8) XOR 16*c; the half read first
+        // holds chunks 4*cfirst.. , folded into the XOR base as well.
         const uint32_t row_off = (TRANS ? dcol * 8192 : 0) + (drow >> 3) * 1024 + r8 * 128;
+        const uint32_t sA0 = smem_addr(smem + C::kOffA) + row_off + (r8 << 4);
         for (int kt = 0; kt < nsteps; ++kt) {
             const int s = kt % S;
             const uint32_t ph = (uint32_t)(kt / S) & 1u;
@@ -270,13 +274,17 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 const uint8_t *cptr = smem + C::kOffC + s * C::kCBytes + code_off;
                 const uint4 ca = *reinterpret_cast<const uint4 *>(cptr + 16 * cfirst);
                 const uint4 cb = *reinterpret_cast<const uint4 *>(cptr + 16 * (cfirst ^ 1));
-                const uint4 c0 = cfirst ? cb : ca, c1 = cfirst ? ca : cb;
-                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                 const NF4Table tab = nf4_table(ah);
-                uint8_t *rowp = smem + C::kOffA + s * C::kABytes + row_off;
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(rowp + ((c ^ r8) << 4)) = nf4_decode8(cw[c], tab);
+                const uint32_t xa = (sA0 + s * C::kABytes) ^ (cfirst << 6);  // chunks of ca: 4*cfirst + i
+                const uint32_t xb = xa ^ 64u;                                  // chunks of cb
+                st_shared_v4(xa ^ 0u, nf4_decode8(ca.x, tab));
+                st_shared_v4(xa ^ 16u, nf4_decode8(ca.y, tab));
+                st_shared_v4(xa ^ 32u, nf4_decode8(ca.z, tab));
+                st_shared_v4(xa ^ 48u, nf4_decode8(ca.w, tab));
+                st_shared_v4(xb ^ 0u, nf4_decode8(cb.x, tab));
+                st_shared_v4(xb ^ 16u, nf4_decode8(cb.y, tab));
+                st_shared_v4(xb ^ 32u, nf4_decode8(cb.z, tab));
+                st_shared_v4(xb ^ 48u, nf4_decode8(cb.w, tab));
                 fence_proxy_async_smem();
             }
             mbar_arrive(dec_full(s));

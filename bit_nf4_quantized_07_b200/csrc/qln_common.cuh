@@ -174,11 +174,26 @@ __device__ __forceinline__ void nf4_decode4(uint32_t s, const NF4Table &t, uint3
 }
 
 // One 32-bit word of packed codes (8 weights, first in the high nibble of the
-// lowest byte) -> 8 BF16 values in memory order.
+// lowest byte) -> 8 BF16 values in memory order.  The selectors of both
+// 16-bit halves come from one mask and one shifted mask of the whole word
+// (prmt reads only the low 16 bits of its selector).
 __device__ __forceinline__ uint4 nf4_decode8(uint32_t w, const NF4Table &t) {
+    const uint32_t i3 = w & 0x77777777u;                           // code & 7, all 8 codes
+    const uint32_t sel = ((w >> 1) & 0x44444444u) | 0x32103210u;   // byte j of x0 or of x1 by bit 3
+    const uint32_t i3h = i3 >> 16, selh = sel >> 16;
     uint4 o;
-    nf4_decode4(w & 0xFFFFu, t, o.x, o.y);
-    nf4_decode4(w >> 16, t, o.z, o.w);
+    {
+        const uint32_t lo = prmt(prmt(t.L[0], t.L[1], i3), prmt(t.L[2], t.L[3], i3), sel);
+        const uint32_t hi = prmt(prmt(t.H[0], t.H[1], i3), prmt(t.H[2], t.H[3], i3), sel);
+        o.x = prmt(lo, hi, 0x4051u);
+        o.y = prmt(lo, hi, 0x6273u);
+    }
+    {
+        const uint32_t lo = prmt(prmt(t.L[0], t.L[1], i3h), prmt(t.L[2], t.L[3], i3h), selh);
+        const uint32_t hi = prmt(prmt(t.H[0], t.H[1], i3h), prmt(t.H[2], t.H[3], i3h), selh);
+        o.z = prmt(lo, hi, 0x4051u);
+        o.w = prmt(lo, hi, 0x6273u);
+    }
     return o;
 }
 
