@@ -200,6 +200,110 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# Secondary measurements (reported under "parts", not part of the step)
+# ---------------------------------------------------------------------------
+def measure_decode(api, dev, copies=64, reps=3):
+    """Decode-shaped forward (4096 x 4096, r = 16, n in {1, 4, 16}) over
+    `copies` distinct NF4 + DQ weights (~553 MB, far above L2), one call per
+    weight, CUDA events around each sweep.  GB/s counts the algorithmic bytes
+    of a call: codes, DQ constants, X, A, B, U and Y."""
+    import torch
+    from bit_nf4_quantized_07_b200 import synthetic
+    cfg = synthetic.DECODE[1]
+    rows, cols, r = cfg.dout, cfg.din, cfg.r
+    gen = torch.Generator(device=dev)
+    weights = []
+    for i in range(copies):
+        gen.manual_seed(7000 + i)
+        W = torch.randn(rows, cols, generator=gen, device=dev) * cfg.w_sigma
+        weights.append(api.quantize_weight(W))
+        del W
+    A = (torch.randn(r, cols, generator=gen, device=dev) * cfg.ab_sigma).to(torch.bfloat16)
+    B = (torch.randn(rows, r, generator=gen, device=dev) * cfg.ab_sigma).to(torch.bfloat16)
+    out = {}
+    stream = torch.cuda.current_stream()
+    for n in (1, 4, 16):
+        X = torch.randn(n, cols, generator=gen, device=dev).to(torch.bfloat16)
+        Y = torch.empty(n, rows, dtype=torch.bfloat16, device=dev)
+        U = torch.empty(n, r, dtype=torch.bfloat16, device=dev)
+        ws = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_FWD, rows, cols, n, r), dev)
+        for w in weights[:4]:
+            api.qlora_linear_fwd(w, X, A, B, 2.0, Y=Y, U_out=U, ws=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            for w in weights:
+                api.qlora_linear_fwd(w, X, A, B, 2.0, Y=Y, U_out=U, ws=ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per_call = e0.elapsed_time(e1) / (reps * copies) * 1e-3
+        nb = rows * cols // 64
+        wbytes = rows * cols // 2 + nb + 4 * ((nb + 255) // 256) + 4
+        bytes_call = wbytes + 2 * n * cols + 2 * r * cols + 2 * rows * r + 2 * n * r + 2 * n * rows
+        out[f"n{n}"] = {"us_per_call": per_call * 1e6, "GBs": bytes_call / per_call / 1e9,
+                        "TFLOPs": 2 * n * (rows * cols + r * cols + rows * r) / per_call / 1e12}
+    del weights
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_sweep(api, dev):
+    """Quantize + DQ and dequant of every linear of a 32-layer d=4096,
+    ffn=11008 decoder (6.48 B parameters, generated on the device), one pass
+    each, CUDA events around each pass."""
+    import torch
+    from bit_nf4_quantized_07_b200 import synthetic
+    gen = torch.Generator(device=dev)
+    mats = []
+    for layer in range(synthetic.SWEEP_LAYERS):
+        for i, (_, rr, cc) in enumerate(synthetic.SWEEP_SHAPES):
+            gen.manual_seed(5000 + 7 * layer + i)
+            W = torch.randn(rr, cc, generator=gen, device=dev) * synthetic.SWEEP_SIGMA
+            nb = rr * cc // 64
+            mats.append((W, torch.empty(rr * cc // 2, dtype=torch.uint8, device=dev),
+                         torch.empty(nb, dtype=torch.float32, device=dev),
+                         torch.empty(nb, dtype=torch.int8, device=dev),
+                         torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev),
+                         torch.empty(1, dtype=torch.float32, device=dev)))
+    maxnb = max(m[2].numel() for m in mats)
+    ws = api.alloc_workspace(api.workspace_bytes(api.OP_DOUBLE_QUANT, maxnb), dev)
+    outbuf = {}
+    for W, *_ in mats:
+        outbuf.setdefault(tuple(W.shape), torch.empty(W.shape, dtype=torch.bfloat16, device=dev))
+    wq = [api.NF4Weight(codes=c, rows=W.shape[0], cols=W.shape[1], absmax=a, qabs=q, dq_scale=sc, dq_mean=mu)
+          for (W, c, a, q, sc, mu) in mats]
+
+    def quant_pass():
+        for (W, c, a, q, sc, mu) in mats:
+            api.nf4_quantize(W, c, a)
+            api.nf4_double_quant(a, q, sc, mu, ws=ws)
+
+    def deq_pass():
+        for w in wq:
+            api.nf4_dequant(w, outbuf[(w.rows, w.cols)])
+
+    stream = torch.cuda.current_stream()
+    quant_pass()
+    deq_pass()
+    torch.cuda.synchronize()
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    e[0].record(stream)
+    quant_pass()
+    e[1].record(stream)
+    deq_pass()
+    e[2].record(stream)
+    torch.cuda.synchronize()
+    params = synthetic.sweep_params()
+    qb, db = codec_bytes_per_param()
+    tq, td = e[0].elapsed_time(e[1]) * 1e-3, e[1].elapsed_time(e[2]) * 1e-3
+    del mats, wq, outbuf
+    torch.cuda.empty_cache()
+    return {"params": params, "quantize_dq_ms": tq * 1e3, "quantize_dq_GBs": params * qb / tq / 1e9,
+            "dequant_ms": td * 1e3, "dequant_GBs": params * db / td / 1e9}
+
+
+# ---------------------------------------------------------------------------
 # GPU leg
 # ---------------------------------------------------------------------------
 def run_ours(args):
@@ -380,6 +484,16 @@ def run_ours(args):
                       "l2": "3 rotating input sets (W0 fp32 alone 180 MB > 126 MB L2)"},
            "gpu_launches": launches, "roofline": roof, "parts": parts, "clocks": clk.summary(),
            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}}
+    if not args.no_extra:
+        del sets
+        torch.cuda.empty_cache()
+        parts["decode_4096x4096_r16"] = measure_decode(api, dev)
+        for k, v in parts["decode_4096x4096_r16"].items():
+            v["frac_hbm"] = v["GBs"] / peaks["hbm_gbs"]
+        sw = measure_sweep(api, dev)
+        sw["quantize_dq_frac_hbm"] = sw["quantize_dq_GBs"] / peaks["hbm_gbs"]
+        sw["dequant_frac_hbm"] = sw["dequant_GBs"] / peaks["hbm_gbs"]
+        parts["sweep_6.48B"] = sw
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         step_s, info = oracle_sample(cfg)
         out["cpu_baseline"] = {"value": flops / step_s / 1e12, "unit": "TFLOP/s", "cores": info["cores"],
@@ -399,6 +513,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["prefill", "large", "pr1"], default="prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the decode-shape and codec-sweep measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

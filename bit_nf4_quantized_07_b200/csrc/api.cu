@@ -39,29 +39,34 @@ qln_status check_device(int *num_sms) {
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Split-K choice for the token reductions: sized for a fixed target grid so
-// that the workspace size does not depend on the device queried.
+// Split-K plans are made for this SM count (B200) on every device, so the
+// workspace size never depends on the device queried.
 constexpr int kSplitTargetSms = 148;
 
 // Workspace layout of the linear calls (all offsets 256-byte aligned):
 //   [0, 256)        int32 device status word (0 = QLN_OK) + reserved
-//   fwd: sU [n][r] bf16, U [n][r] bf16 (used when U_out is NULL)
+//   fwd: sU [n][r] bf16, U [n][r] bf16 (used when U_out is NULL),
+//        split-K partials of U (fp32)
 //   bwd: Bt [r][dout] bf16, G [n][r] bf16, sG [n][r] bf16, U [n][r] bf16,
-//        dA partials, dB partials (fp32, split-K)
+//        split-K partials of G / U (fp32, reused), dA partials, dB partials
+// Split counts are planned for a fixed SM count so that the workspace size
+// does not depend on the device queried.
 struct FwdWs {
-    size_t sU, U, total;
+    size_t sU, U, pU, total;
 };
 struct BwdWs {
-    size_t Bt, G, sG, U, pA, pB, total;
+    size_t Bt, G, sG, U, pGU, pA, pB, total;
     int splitA, splitB;
 };
 
-FwdWs fwd_layout(int64_t n, int r) {
+FwdWs fwd_layout(int64_t rows, int64_t cols, int64_t n, int r) {
+    (void)rows;
     FwdWs L;
     const size_t nr = round256((size_t)n * r * 2);
     L.sU = 256;
     L.U = L.sU + nr;
-    L.total = L.U + nr;
+    L.pU = L.U + nr;
+    L.total = L.pU + round256(qln::lora_down_partial_bytes(n, cols, r, kSplitTargetSms));
     return L;
 }
 
@@ -72,9 +77,12 @@ BwdWs bwd_layout(int64_t rows, int64_t cols, int64_t n, int r) {
     L.G = L.Bt + round256((size_t)rows * r * 2);
     L.sG = L.G + nr;
     L.U = L.sG + nr;
+    L.pGU = L.U + nr;
+    const size_t pg = qln::lora_down_partial_bytes(n, rows, r, kSplitTargetSms);
+    const size_t pu = qln::lora_down_partial_bytes(n, cols, r, kSplitTargetSms);
     L.splitA = qln::tn_reduce_splits(n, r, cols, kSplitTargetSms);
     L.splitB = qln::tn_reduce_splits(n, rows, r, kSplitTargetSms);
-    L.pA = L.U + nr;
+    L.pA = L.pGU + round256(pg > pu ? pg : pu);
     L.pB = L.pA + round256(qln::tn_reduce_partials_bytes(r, cols, L.splitA));
     L.total = L.pB + round256(qln::tn_reduce_partials_bytes(rows, r, L.splitB));
     return L;
@@ -186,7 +194,7 @@ qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     if (st != QLN_OK) return st;
     if (!Y || !ws) return QLN_ERR_NULL;
     if (!aligned(Y, 16) || (U_out && !aligned(U_out, 16)) || !aligned(ws, 256)) return QLN_ERR_ALIGN;
-    const FwdWs L = fwd_layout(n, r);
+    const FwdWs L = fwd_layout(w->rows, w->cols, n, r);
     if (ws_bytes < L.total) return QLN_ERR_WORKSPACE;
     int sms = 0;
     st = check_device(&sms);
@@ -196,10 +204,11 @@ qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     int *status = reinterpret_cast<int *>(wsb);
     uint16_t *sU = reinterpret_cast<uint16_t *>(wsb + L.sU);
     uint16_t *U = U_out ? U_out : reinterpret_cast<uint16_t *>(wsb + L.U);
+    float *pU = reinterpret_cast<float *>(wsb + L.pU);
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     // U = X A^T (and s*U for the adapter MMA), then the fused weight GEMM.
-    e = qln::launch_lora_down(X, n, w->cols, A, w->cols, 1, r, s, U, sU, cs, sms);
+    e = qln::launch_lora_down(X, n, w->cols, A, r, s, U, sU, pU, cs, kSplitTargetSms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     e = fused_gemm(w, false, X, n, sU, B, r, Y, status, cs, sms);
     return from_cuda(e);
@@ -225,13 +234,14 @@ qln_status qlora_linear_bwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     uint16_t *Bt = reinterpret_cast<uint16_t *>(wsb + L.Bt);
     uint16_t *G = reinterpret_cast<uint16_t *>(wsb + L.G);
     uint16_t *sG = reinterpret_cast<uint16_t *>(wsb + L.sG);
+    float *pGU = reinterpret_cast<float *>(wsb + L.pGU);
     float *pA = reinterpret_cast<float *>(wsb + L.pA);
     float *pB = reinterpret_cast<float *>(wsb + L.pB);
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     if (!U) {
         uint16_t *Uw = reinterpret_cast<uint16_t *>(wsb + L.U);
-        e = qln::launch_lora_down(X, n, w->cols, A, w->cols, 1, r, s, Uw, nullptr, cs, sms);
+        e = qln::launch_lora_down(X, n, w->cols, A, r, s, Uw, nullptr, pGU, cs, kSplitTargetSms);
         if (e != cudaSuccess) return QLN_ERR_CUDA;
         U = Uw;
     }
@@ -244,7 +254,7 @@ qln_status qlora_linear_bwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
         if (cudaGetLastError() != cudaSuccess) return QLN_ERR_CUDA;
     }
     // G = dY B (and s*G), dX = dY W' + (s G) A, dA = s G^T X, dB = s dY^T U.
-    e = qln::launch_lora_down(dY, n, w->rows, Bt, w->rows, 1, r, s, G, sG, cs, sms);
+    e = qln::launch_lora_down(dY, n, w->rows, Bt, r, s, G, sG, pGU, cs, kSplitTargetSms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     e = fused_gemm(w, true, dY, n, sG, A, r, dX, status, cs, sms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
@@ -259,7 +269,7 @@ size_t qln_workspace_bytes(int32_t op, int64_t rows, int64_t cols, int64_t n, in
         case QLN_OP_DOUBLE_QUANT:
             return rows > 0 ? qln::dq_workspace_bytes(rows) : 0;
         case QLN_OP_LINEAR_FWD:
-            return (n > 0 && r > 0) ? fwd_layout(n, r).total : 0;
+            return (rows > 0 && cols > 0 && n > 0 && r > 0) ? fwd_layout(rows, cols, n, r).total : 0;
         case QLN_OP_LINEAR_BWD:
             return (rows > 0 && cols > 0 && n > 0 && r > 0) ? bwd_layout(rows, cols, n, r).total : 0;
         default:

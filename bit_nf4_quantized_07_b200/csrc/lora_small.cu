@@ -14,143 +14,189 @@ namespace qln {
 
 // ===========================================================================
 // lora_down: out[t][j] = sum_k in[t][k] * wt[j][k], in [n][K], wt [r][K].
-// A CTA owns 16*MT tokens; its 8 warps split K (64-wide chunks round robin)
-// and fold their partial tiles pairwise through shared memory (a fixed order:
-// deterministic).  Fragments come straight from global memory: in mma step s
-// of a chunk, lane (g, c) feeds k = 16s + 4c .. 16s + 4c + 3 (one 8-byte load
-// per row), i.e. each 16-wide step uses k in the natural order.
+// Split-K tiles: a CTA owns 64 tokens x all r outputs over `cps` chunks of 64
+// k, streamed through a 4-stage cp.async ring (both operands K-contiguous, so
+// plain ldmatrix feeds the MMA); 4 warps x 16 tokens each.  Each split writes
+// an fp32 partial tile; lora_fold adds the splits in a fixed order
+// (deterministic) and writes out = bf16(sum) and out_scaled = bf16(scale*sum).
 // ===========================================================================
-constexpr int kDownWarps = 8;
+constexpr int kDnStages = 4;
+constexpr int kDnLd = 72;  // padded row (bf16) of the staged tiles
 
-template <int MT, int NT>
-__global__ void __launch_bounds__(kDownWarps * 32) lora_down_kernel(const uint16_t *__restrict__ in, int64_t n,
-                                                                     int64_t K, const uint16_t *__restrict__ wt,
-                                                                     int r, float scale, uint16_t *__restrict__ out,
-                                                                     uint16_t *__restrict__ out_scaled) {
-    extern __shared__ float red[];  // [kDownWarps/2][16*MT][8*NT]
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+template <int NT>
+__global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t *__restrict__ in, int64_t n, int64_t K,
+                                                        const uint16_t *__restrict__ wt, int r, int cps,
+                                                        float *__restrict__ partial) {
+    extern __shared__ __align__(16) uint16_t dsm[];
+    constexpr int WR = NT * 8;                              // adapter rows staged (r rounded up to 8)
+    constexpr int STAGE = (64 + WR) * kDnLd;                // elements per stage
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
-    const int64_t t0 = (int64_t)blockIdx.x * 16 * MT;
-    float acc[MT][NT][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+    const int64_t t0 = (int64_t)blockIdx.x * 64;
+    const int split = blockIdx.y;
+    const int64_t nch = K / 64;
+    const int64_t ch0 = (int64_t)split * cps;
+    const int64_t ch1 = ch0 + cps < nch ? ch0 + cps : nch;
 
-    const int64_t nchunks = K / 64;
-    for (int64_t ch = warp; ch < nchunks; ch += kDownWarps) {
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+
+    auto load = [&](int stage, int64_t ch) {
+        uint16_t *Xs = dsm + stage * STAGE;
+        uint16_t *Ws = Xs + 64 * kDnLd;
         const int64_t k0 = ch * 64;
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const int64_t kk = k0 + 16 * s + 4 * c;
-            uint32_t a[MT][4];
+        for (int i = 0; i < 4; ++i) {  // 64 rows x 8 chunks
+            const int idx = tid + 128 * i, row = idx >> 3, ck = idx & 7;
+            const int64_t t = t0 + row;
+            const bool ok = t < n;
+            cp_async16_zfill(Xs + row * kDnLd + 8 * ck, ok ? in + t * K + k0 + 8 * ck : in, ok ? 16 : 0);
+        }
+        for (int idx = tid; idx < WR * 8; idx += 128) {
+            const int row = idx >> 3, ck = idx & 7;
+            const bool ok = row < r;
+            cp_async16_zfill(Ws + row * kDnLd + 8 * ck, ok ? wt + (int64_t)row * K + k0 + 8 * ck : wt, ok ? 16 : 0);
+        }
+    };
+
+    // prologue: fill kDnStages-1 stages (empty commit groups keep the count uniform)
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                const int64_t ta = t0 + 16 * mt + g, tb = ta + 8;
-                uint2 va = make_uint2(0u, 0u), vb = va;
-                if (ta < n) va = __ldg(reinterpret_cast<const uint2 *>(in + ta * K + kk));
-                if (tb < n) vb = __ldg(reinterpret_cast<const uint2 *>(in + tb * K + kk));
-                a[mt][0] = va.x;  // (row g,   k 4c, 4c+1)
-                a[mt][1] = vb.x;  // (row g+8, k 4c, 4c+1)
-                a[mt][2] = va.y;  // (row g,   k 4c+2, 4c+3)
-                a[mt][3] = vb.y;  // (row g+8, k 4c+2, 4c+3)
+    for (int i = 0; i < kDnStages - 1; ++i) {
+        if (ch0 + i < ch1) load(i, ch0 + i);
+        cp_async_commit();
+    }
+    for (int64_t ch = ch0; ch < ch1; ++ch) {
+        const int it = (int)(ch - ch0);
+        {
+            const int64_t nx = ch + kDnStages - 1;
+            if (nx < ch1) load((it + kDnStages - 1) % kDnStages, nx);
+            cp_async_commit();
+        }
+        cp_async_wait<kDnStages - 1>();
+        __syncthreads();
+        const uint16_t *Xs = dsm + (it % kDnStages) * STAGE;
+        const uint16_t *Ws = Xs + 64 * kDnLd;
+#pragma unroll
+        for (int kk = 0; kk < 64; kk += 16) {
+            uint32_t a[4];
+            {
+                const int row = 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int col = kk + (lane >> 4) * 8;
+                ldmatrix_x4(a[0], a[1], a[2], a[3], Xs + row * kDnLd + col);
             }
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int j = 8 * nt + g;
-                uint2 vw = make_uint2(0u, 0u);
-                if (j < r) vw = __ldg(reinterpret_cast<const uint2 *>(wt + (int64_t)j * K + kk));
-                const uint32_t b[2] = {vw.x, vw.y};
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) mma_bf16_16816(acc[mt][nt], a[mt], b);
+            for (int np = 0; np < NT / 2; ++np) {
+                const int row = np * 16 + (lane & 7) + (lane >> 4) * 8;
+                const int col = kk + ((lane >> 3) & 1) * 8;
+                uint32_t r0, r1, r2, r3;
+                ldmatrix_x4(r0, r1, r2, r3, Ws + row * kDnLd + col);
+                const uint32_t b0[2] = {r0, r1}, b1[2] = {r2, r3};
+                mma_bf16_16816(acc[2 * np], a, b0);
+                mma_bf16_16816(acc[2 * np + 1], a, b1);
+            }
+            if (NT & 1) {
+                const int row = (NT - 1) * 8 + (lane & 7);
+                const int col = kk + ((lane >> 3) & 1) * 8;
+                uint32_t r0, r1;
+                ldmatrix_x2(r0, r1, Ws + row * kDnLd + col);
+                const uint32_t b0[2] = {r0, r1};
+                mma_bf16_16816(acc[NT - 1], a, b0);
             }
         }
-    }
-    // Pairwise fold of the 8 warp tiles: 8 -> 4 -> 2 -> 1.
-    constexpr int TILE = 16 * MT * 8 * NT;
-#pragma unroll
-    for (int half = kDownWarps / 2; half >= 1; half >>= 1) {
-        if (warp >= half && warp < 2 * half) {
-            float *dst = red + (warp - half) * TILE;
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int row = 16 * mt + g + 8 * (e >> 1), col = 8 * nt + 2 * c + (e & 1);
-                        dst[row * 8 * NT + col] = acc[mt][nt][e];
-                    }
-        }
-        __syncthreads();
-        if (warp < half) {
-            const float *src = red + warp * TILE;
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int row = 16 * mt + g + 8 * (e >> 1), col = 8 * nt + 2 * c + (e & 1);
-                        acc[mt][nt][e] = __fadd_rn(acc[mt][nt][e], src[row * 8 * NT + col]);
-                    }
-        }
         __syncthreads();
     }
-    if (warp == 0) {
+    cp_async_wait<0>();
+
+    float *dst = partial + (int64_t)split * n * r;
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int64_t t = t0 + 16 * mt + g + 8 * (e >> 1);
-                    const int j = 8 * nt + 2 * c + (e & 1);
-                    if (t < n && j < r) {
-                        const float v = acc[mt][nt][e];
-                        out[t * r + j] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-                        if (out_scaled)
-                            out_scaled[t * r + j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, v)));
-                    }
-                }
+        for (int e = 0; e < 4; ++e) {
+            const int64_t t = t0 + 16 * warp + g + 8 * (e >> 1);
+            const int j = 8 * nt + 2 * c + (e & 1);
+            if (t < n && j < r) dst[t * r + j] = acc[nt][e];
+        }
+}
+
+__global__ void lora_fold_kernel(const float *__restrict__ partial, int splits, int64_t total, float scale,
+                                 uint16_t *__restrict__ out, uint16_t *__restrict__ out_scaled) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+        float v = 0.f;
+        for (int z = 0; z < splits; ++z) v = __fadd_rn(v, partial[(int64_t)z * total + i]);
+        out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        if (out_scaled) out_scaled[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, v)));
     }
 }
 
-template <int MT, int NT>
-static cudaError_t launch_down_t(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, float scale,
-                                 uint16_t *out, uint16_t *out_scaled, cudaStream_t st) {
-    const size_t smem = (size_t)(kDownWarps / 2) * 16 * MT * 8 * NT * sizeof(float);
-    auto kern = lora_down_kernel<MT, NT>;
+// Splits of the K range: about 6 CTAs per SM, at least 4 chunks of 64 per CTA.
+void lora_down_plan(int64_t n, int64_t K, int num_sms, int *splits, int *cps) {
+    const int64_t nch = K / 64;
+    const int64_t ttiles = (n + 63) / 64;
+    int64_t sp = (6 * (int64_t)num_sms + ttiles - 1) / ttiles;
+    const int64_t maxsp = nch / 4 > 0 ? nch / 4 : 1;
+    if (sp > maxsp) sp = maxsp;
+    if (sp < 1) sp = 1;
+    const int64_t c = (nch + sp - 1) / sp;
+    *cps = (int)c;
+    *splits = (int)((nch + c - 1) / c);
+}
+
+size_t lora_down_partial_bytes(int64_t n, int64_t K, int r, int num_sms) {
+    int sp, cps;
+    lora_down_plan(n, K, num_sms, &sp, &cps);
+    return (size_t)sp * (size_t)n * (size_t)r * sizeof(float);
+}
+
+template <int NT>
+static cudaError_t launch_down_t(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, int splits,
+                                 int cps, float *partial, cudaStream_t st) {
+    const size_t smem = (size_t)kDnStages * (64 + NT * 8) * kDnLd * sizeof(uint16_t);
+    auto kern = lora_down_kernel<NT>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    const int64_t grid = (n + 16 * MT - 1) / (16 * MT);
-    kern<<<(unsigned)grid, kDownWarps * 32, smem, st>>>(in, n, K, wt, r, scale, out, out_scaled);
+    dim3 grid((unsigned)((n + 63) / 64), (unsigned)splits);
+    kern<<<grid, 128, smem, st>>>(in, n, K, wt, r, cps, partial);
     note_launch();
     return cudaGetLastError();
 }
 
-template <int MT>
-static cudaError_t launch_down_mt(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, float scale,
-                                  uint16_t *out, uint16_t *out_scaled, cudaStream_t st) {
+cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, float scale,
+                             uint16_t *out, uint16_t *out_scaled, float *partial, cudaStream_t st, int num_sms) {
+    int splits, cps;
+    lora_down_plan(n, K, num_sms, &splits, &cps);
     const int nt = (r + 7) / 8;
-    if (nt <= 1) return launch_down_t<MT, 1>(in, n, K, wt, r, scale, out, out_scaled, st);
-    if (nt <= 2) return launch_down_t<MT, 2>(in, n, K, wt, r, scale, out, out_scaled, st);
-    if (nt <= 4) return launch_down_t<MT, 4>(in, n, K, wt, r, scale, out, out_scaled, st);
-    if (nt <= 8) return launch_down_t<MT, 8>(in, n, K, wt, r, scale, out, out_scaled, st);
-    return launch_down_t<MT, 16>(in, n, K, wt, r, scale, out, out_scaled, st);
-}
-
-cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int64_t wt_sj,
-                             int64_t wt_sk, int r, float scale, uint16_t *out, uint16_t *out_scaled,
-                             cudaStream_t st, int num_sms) {
-    (void)wt_sj;
-    (void)wt_sk;  // wt is always [r][K] row-major here (the caller transposes B once)
-    if (n / 32 >= num_sms) return launch_down_mt<2>(in, n, K, wt, r, scale, out, out_scaled, st);
-    return launch_down_mt<1>(in, n, K, wt, r, scale, out, out_scaled, st);
+    cudaError_t e;
+    switch (nt) {
+        case 1: e = launch_down_t<1>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 2: e = launch_down_t<2>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 3: e = launch_down_t<3>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 4: e = launch_down_t<4>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 5: e = launch_down_t<5>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 6: e = launch_down_t<6>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 7: e = launch_down_t<7>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 8: e = launch_down_t<8>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 9: e = launch_down_t<9>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 10: e = launch_down_t<10>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 11: e = launch_down_t<11>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 12: e = launch_down_t<12>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 13: e = launch_down_t<13>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 14: e = launch_down_t<14>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 15: e = launch_down_t<15>(in, n, K, wt, r, splits, cps, partial, st); break;
+        default: e = launch_down_t<16>(in, n, K, wt, r, splits, cps, partial, st); break;
+    }
+    if (e != cudaSuccess) return e;
+    const int64_t total = n * r;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    lora_fold_kernel<<<(unsigned)blocks, 256, 0, st>>>(partial, splits, total, scale, out, out_scaled);
+    note_launch();
+    return cudaGetLastError();
 }
 
 // ===========================================================================
@@ -161,13 +207,13 @@ cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uin
 // of the grid covers an interleaved share of the token steps and writes an
 // fp32 partial tile; tn_fold adds the slices in a fixed order.
 // ===========================================================================
-constexpr int kTnBM = 64, kTnBN = 64, kTnBK = 32, kTnPad = 72;
+constexpr int kTnBM = 64, kTnBN = 64, kTnBK = 32, kTnPad = 72, kTnStages = 4;
 
 __global__ void __launch_bounds__(128) tn_reduce_kernel(const uint16_t *__restrict__ P, const uint16_t *__restrict__ Q,
                                                         int64_t n, int64_t M, int64_t N, float scale,
                                                         float *__restrict__ C, float *__restrict__ partials) {
-    __shared__ __align__(16) uint16_t Ps[2][kTnBK][kTnPad];
-    __shared__ __align__(16) uint16_t Qs[2][kTnBK][kTnPad];
+    __shared__ __align__(16) uint16_t Ps[kTnStages][kTnBK][kTnPad];
+    __shared__ __align__(16) uint16_t Qs[kTnStages][kTnBK][kTnPad];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int wm = warp & 1, wn = warp >> 1;  // 2x2 warps, 32x32 each
@@ -199,21 +245,24 @@ __global__ void __launch_bounds__(128) tn_reduce_kernel(const uint16_t *__restri
             uint16_t *dst = op ? &Qs[buf][row][8 * ck] : &Ps[buf][row][8 * ck];
             cp_async16_zfill(dst, src, ok ? 16 : 0);
         }
-        cp_async_commit();
     };
 
-    int64_t step = split;
-    if (step < nsteps) load(0, step);
-    int buf = 0;
-    for (; step < nsteps; step += nsplit) {
-        const int64_t next = step + nsplit;
-        if (next < nsteps) {
-            load(buf ^ 1, next);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+    // this split's token steps: split, split + nsplit, ...
+    const int64_t mysteps = split < nsteps ? (nsteps - split + nsplit - 1) / nsplit : 0;
+#pragma unroll
+    for (int i = 0; i < kTnStages - 1; ++i) {
+        if (i < mysteps) load(i, split + (int64_t)i * nsplit);
+        cp_async_commit();
+    }
+    for (int64_t it = 0; it < mysteps; ++it) {
+        {
+            const int64_t nx = it + kTnStages - 1;
+            if (nx < mysteps) load((int)(nx % kTnStages), split + nx * nsplit);
+            cp_async_commit();
         }
+        cp_async_wait<kTnStages - 1>();
         __syncthreads();
+        const int buf = (int)(it % kTnStages);
 #pragma unroll
         for (int kk = 0; kk < kTnBK; kk += 16) {
             uint32_t a[2][4], b[4][2];
@@ -242,8 +291,8 @@ __global__ void __launch_bounds__(128) tn_reduce_kernel(const uint16_t *__restri
                 for (int nt = 0; nt < 4; ++nt) mma_bf16_16816(acc[mt][nt], a[mt], b[nt]);
         }
         __syncthreads();
-        buf ^= 1;
     }
+    cp_async_wait<0>();
 
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
@@ -270,11 +319,15 @@ __global__ void tn_fold_kernel(const float *__restrict__ partials, int splits, i
     }
 }
 
+// About 6 CTAs per SM, each with at least 8 token steps (256 tokens).
 int tn_reduce_splits(int64_t n, int64_t M, int64_t N, int num_sms) {
     const int64_t tiles = ((M + kTnBM - 1) / kTnBM) * ((N + kTnBN - 1) / kTnBN);
     const int64_t steps = (n + kTnBK - 1) / kTnBK;
-    int64_t splits = 1;
-    while (tiles * splits < 2 * num_sms && splits * 2 <= steps && splits < 16) splits *= 2;
+    int64_t splits = (6 * (int64_t)num_sms + tiles - 1) / tiles;
+    const int64_t maxsp = steps / 8 > 0 ? steps / 8 : 1;
+    if (splits > maxsp) splits = maxsp;
+    if (splits > 64) splits = 64;
+    if (splits < 1) splits = 1;
     return (int)splits;
 }
 

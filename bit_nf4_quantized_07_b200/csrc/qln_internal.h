@@ -26,11 +26,12 @@ int64_t dq_static_max_blocks();
 int64_t dq_max_blocks();
 
 // lora_small.cu: skinny products around the adapters.
-//   out[t][j] = bf16(sum_k in[t][k] * wt(j, k)) and, if out_scaled != NULL,
-//   out_scaled[t][j] = bf16(scale * that sum); wt(j, k) = wt[j*wt_sj + k*wt_sk].
-cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int64_t wt_sj,
-                             int64_t wt_sk, int r, float scale, uint16_t *out, uint16_t *out_scaled,
-                             cudaStream_t st, int num_sms);
+//   out[t][j] = bf16(sum_k in[t][k] * wt[j][k]) and, if out_scaled != NULL,
+//   out_scaled[t][j] = bf16(scale * that sum); wt is [r][K] row-major.
+//   `partial` is fp32 scratch of lora_down_partial_bytes(n, K, r, num_sms).
+cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, float scale,
+                             uint16_t *out, uint16_t *out_scaled, float *partial, cudaStream_t st, int num_sms);
+size_t lora_down_partial_bytes(int64_t n, int64_t K, int r, int num_sms);
 //   C[m][c] = scale * sum_t P[t][m] * Q[t][c]  (P [n][M], Q [n][N] row-major), fp32 out.
 cudaError_t launch_tn_reduce(const uint16_t *P, const uint16_t *Q, int64_t n, int64_t M, int64_t N, float scale,
                              float *C, float *partials, int splits, cudaStream_t st);
