@@ -17,27 +17,25 @@ namespace qln {
 // K1: quantize.  One warp streams 256 consecutive weights (4 blocks) per step:
 // lane l holds float4 #l and #(l+32), i.e. elements 4l..4l+3 of block l/16 and
 // of block 2 + l/16.  Each 16-lane half reduces its block's absmax with four
-// xor-shuffles and every element is divided by it (IEEE fp32 division, x in
-// [-1, 1]).
-// Snap without a 15-way compare: the top 12 bits of x (sign, exponent, three
-// mantissa bits) name an interval of fp32 values that contains at most one
-// snap threshold (the narrowest gap between thresholds, 0.08, is wider than
+// xor-shuffles; x = w / absmax is the IEEE fp32 quotient, in [-1, 1].
+// Snap without a 15-way compare and (almost always) without a division: the
+// top 12 bits of x (sign, exponent, three mantissa bits) name an interval of
+// fp32 values that contains at most one snap threshold (the narrowest gap between thresholds, 0.08, is wider than
 // any such interval below 1 in magnitude).  A per-CTA table gives, for each
 // key, the code of the interval's smallest value and that one threshold (or
 // +inf), so  q = base[key] + (x > thr[key])  -- exactly #{k : x > t_k}.
 // ===========================================================================
 constexpr int kSnapKeys = 4096;
 
-__device__ __forceinline__ uint32_t snap_lut(float x, const uint2 *lut) {
-    const uint2 e = lut[__float_as_uint(x) >> 20];
-    return e.y + ((x > __uint_as_float(e.x)) ? 1u : 0u);
-}
-
+// Only keys of |x| <= 1.125 are ever looked up (|x| <= 1 up to a few ulps of
+// the reciprocal product), i.e. keys 0x000..0x3F8 and 0x800..0xBF8.
 __device__ void build_snap_lut(uint2 *lut) {
     float t[15];
 #pragma unroll
     for (int k = 0; k < 15; ++k) t[k] = nf4_threshold(k);
-    for (int key = threadIdx.x; key < kSnapKeys; key += blockDim.x) {
+    for (int i = threadIdx.x; i < 2 * 1024; i += blockDim.x) {
+        const int key = (i & 1023) | ((i >> 10) << 11);
+        if ((key & 0x3FF) > 0x3F8) continue;
         const float a = __uint_as_float((uint32_t)key << 20);
         const float b = __uint_as_float(((uint32_t)key << 20) | 0xFFFFFu);
         const bool neg = (key & 0x800) != 0;
@@ -52,13 +50,37 @@ __device__ void build_snap_lut(uint2 *lut) {
     }
 }
 
-__device__ __forceinline__ uint32_t snap_pair(float w0, float w1, float a, const uint2 *lut) {
-    float x0 = 0.f, x1 = 0.f;
-    if (a > 0.f) {
-        x0 = __fdiv_rn(w0, a);
-        x1 = __fdiv_rn(w1, a);
+// Codes of the 4 weights of v (block absmax a > 0, inv = RN(1/a)), packed as
+// two bytes, first weight in the high nibble of the first byte.  The product
+// y = RN(w * inv) is within 2 ulp of w/a, and x = RN(w/a) within half an ulp,
+// so y and x fall on the same side of a threshold t unless |y - t| < 3 ulp(t)
+// <= 2^-21 (|t| < 1).  Only then is the exact quotient formed (IEEE
+// division) and used instead: the code is always that of x.  The test looks
+// only at the threshold of y's own key interval; that is enough because every
+// threshold lies more than 15,000 ulps inside its key interval, so no
+// threshold of a neighbouring interval is within 3 ulps of y.
+__device__ __forceinline__ uint32_t snap4(float4 v, float a, float inv, const uint2 *lut) {
+    const float w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t q[4];
+    bool near = false;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float y = __fmul_rn(w[i], inv);
+        const uint2 e = lut[__float_as_uint(y) >> 20];
+        const float d = __fsub_rn(y, __uint_as_float(e.x));
+        q[i] = e.y + (d > 0.f ? 1u : 0u);
+        near |= fabsf(d) < 4.76837158203125e-07f;  // 2^-21
     }
-    return (snap_lut(x0, lut) << 4) | snap_lut(x1, lut);  // first element in the high nibble
+    if (near) {  // rare: redo the whole group exactly
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float x = __fdiv_rn(w[i], a);
+            const uint2 e = lut[__float_as_uint(x) >> 20];
+            q[i] = e.y + ((x > __uint_as_float(e.x)) ? 1u : 0u);
+        }
+    }
+    if (!(a > 0.f)) return 0x7777u;  // all-zero block: the exact zero
+    return (q[0] << 4) | q[1] | (q[2] << 12) | (q[3] << 8);
 }
 
 __device__ __forceinline__ float absmax4(float4 v) {
@@ -77,27 +99,44 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float4 *__restr
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
     const int64_t nchunks = (nb + 3) / 4;  // 4 blocks (256 weights) per chunk
 
-    for (int64_t c = warp; c < nchunks; c += nwarps) {
-        const int64_t b0 = 4 * c + (lane >> 4);  // block of v0
-        const int64_t b1 = b0 + 2;               // block of v1
-        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-        if (b0 < nb) v0 = __ldcs(W + 64 * c + lane);
-        if (b1 < nb) v1 = __ldcs(W + 64 * c + 32 + lane);
-        float m0 = absmax4(v0), m1 = absmax4(v1);
+    // Two 256-weight chunks per iteration: four 16-byte loads in flight per lane.
+    for (int64_t c0 = warp; c0 < nchunks; c0 += 2 * nwarps) {
+        float4 v[2][2];
 #pragma unroll
-        for (int off = 8; off >= 1; off >>= 1) {
-            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
-            m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
+        for (int u = 0; u < 2; ++u) {
+            const int64_t c = c0 + u * nwarps;
+            const int64_t b0 = 4 * c + (lane >> 4);
+            const float4 *src = W + 64 * c + lane;
+            v[u][0] = (c < nchunks && b0 < nb) ? __ldcs(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[u][1] = (c < nchunks && b0 + 2 < nb) ? __ldcs(src + 32) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        if (b0 < nb) {
-            uint32_t p = snap_pair(v0.x, v0.y, m0, lut) | (snap_pair(v0.z, v0.w, m0, lut) << 8);
-            __stcs(codes16 + 64 * c + lane, (uint16_t)p);
-            if ((lane & 15) == 0) absmax[b0] = m0;
+        float m[2][2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            m[u][0] = absmax4(v[u][0]);
+            m[u][1] = absmax4(v[u][1]);
         }
-        if (b1 < nb) {
-            uint32_t p = snap_pair(v1.x, v1.y, m1, lut) | (snap_pair(v1.z, v1.w, m1, lut) << 8);
-            __stcs(codes16 + 64 * c + 32 + lane, (uint16_t)p);
-            if ((lane & 15) == 0) absmax[b1] = m1;
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                m[u][0] = fmaxf(m[u][0], __shfl_xor_sync(0xffffffffu, m[u][0], off));
+                m[u][1] = fmaxf(m[u][1], __shfl_xor_sync(0xffffffffu, m[u][1], off));
+            }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int64_t c = c0 + u * nwarps;
+            if (c >= nchunks) break;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int64_t b = 4 * c + (lane >> 4) + 2 * h;  // block of v[u][h]
+                if (b < nb) {
+                    const float a = m[u][h];
+                    const float inv = a > 0.f ? __frcp_rn(a) : 0.f;
+                    __stcs(codes16 + 64 * c + 32 * h + lane, (uint16_t)snap4(v[u][h], a, inv, lut));
+                    if ((lane & 15) == 0) absmax[b] = a;
+                }
+            }
         }
     }
 }
@@ -108,7 +147,7 @@ cudaError_t launch_nf4_quantize(const float *W, int64_t numel, uint8_t *codes, f
     const int64_t nchunks = (nb + 3) / 4;
     const int threads = 256;
     int64_t grid = (nchunks + 7) / 8;
-    const int64_t cap = (int64_t)num_sms * 4;  // persistent-ish: the table is built once per CTA
+    const int64_t cap = (int64_t)num_sms * 4;  // the table is built once per CTA
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
     nf4_quantize_kernel<<<(unsigned)grid, threads, 0, st>>>(reinterpret_cast<const float4 *>(W), nb,
@@ -356,40 +395,50 @@ cudaError_t launch_nf4_double_quant_static(const float *absmax, int64_t nb, int8
 }
 
 // ===========================================================================
-// K4: doubleDequant to BF16.  A warp streams 64 code words (512 weights,
-// 8 blocks) per step: lane l decodes words 2l and 2l+1 (16 weights of block
-// l/4) with the register-only table decode and stores 32 contiguous bytes.
+// K4: doubleDequant to BF16.  A warp streams 32 code words (256 weights, 4
+// blocks): lane l decodes word l (8 weights) and stores 16 bytes, so every
+// load and store instruction is fully coalesced.  A 256-entry shared table
+// maps a code byte to the book values of its two codes (c[hi], c[lo]); the
+// products with the restored constant are fp32 multiplies rounded once to
+// BF16, spreading the work over the load/store, FMA and integer pipes.
 // w' = bf16_RN(fp32(ahat * c[q])).
 // ===========================================================================
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint2 *__restrict__ codes64,
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t *__restrict__ codes32,
                                                           const float *__restrict__ absmax,
                                                           const int8_t *__restrict__ qabs,
                                                           const float *__restrict__ scale,
-                                                          const float *__restrict__ mu_p, int64_t npairs,
+                                                          const float *__restrict__ mu_p, int64_t nwords,
                                                           uint4 *__restrict__ out) {
+    __shared__ float2 pair_tab[256];
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) pair_tab[i] = make_float2(nf4_value(i >> 4), nf4_value(i & 15));
+    __syncthreads();
     const float mu = qabs ? __ldg(mu_p) : 0.f;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < npairs; i += stride) {
-        const int64_t j = i >> 2;  // 4 pairs of words (64 codes) per block
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nwords; i += stride) {
+        const int64_t j = i >> 3;  // 8 words (64 codes) per block
         float ah;
         if (qabs) ah = dq_restore(__ldg(qabs + j), __ldg(scale + (j >> 8)), mu);
         else ah = __ldg(absmax + j);
-        const uint2 cw = __ldcs(codes64 + i);
-        const NF4Table t = nf4_table(ah);
-        __stcs(out + 2 * i, nf4_decode8(cw.x, t));
-        __stcs(out + 2 * i + 1, nf4_decode8(cw.y, t));
+        const uint32_t cw = __ldcs(codes32 + i);
+        uint32_t o[4];
+#pragma unroll
+        for (int bi = 0; bi < 4; ++bi) {
+            const float2 cc = pair_tab[(cw >> (8 * bi)) & 0xffu];
+            o[bi] = pack_bf16x2(__fmul_rn(ah, cc.x), __fmul_rn(ah, cc.y));
+        }
+        __stcs(out + i, make_uint4(o[0], o[1], o[2], o[3]));
     }
 }
 
 cudaError_t launch_nf4_dequant(const qln_nf4_weight *w, uint16_t *out, cudaStream_t st, int num_sms) {
     const int64_t numel = w->rows * w->cols;
-    const int64_t npairs = numel / 16;
-    int64_t grid = (npairs + 255) / 256;
+    const int64_t nwords = numel / 8;
+    int64_t grid = (nwords + 255) / 256;
     const int64_t cap = (int64_t)num_sms * 8;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
-    nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint2 *>(w->codes), w->absmax,
-                                                      w->qabs, w->dq_scale, w->dq_mean, npairs,
+    nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint32_t *>(w->codes), w->absmax,
+                                                      w->qabs, w->dq_scale, w->dq_mean, nwords,
                                                       reinterpret_cast<uint4 *>(out));
     note_launch();
     return cudaGetLastError();
