@@ -46,6 +46,33 @@ def _load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def _kernel_sources_sha1():
+    """SHA-1 over the library's CUDA sources: identifies the kernels a
+    committed ncu record was taken from."""
+    import hashlib
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "bit_nf4_quantized_07_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def _recorded_traffic(workload):
+    """DRAM bytes per qlora_linear_fwd call from profiles/roofline_traffic.json,
+    or None when the record is missing, for another workload, or taken from
+    kernel sources other than the current ones."""
+    p = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    if rec.get("workload") != workload or rec.get("kernel_sources_sha1") != _kernel_sources_sha1():
+        return None
+    return rec.get("dram_bytes_per_call")
+
+
 def _workload(name):
     from bit_nf4_quantized_07_b200 import synthetic
     return {"prefill": synthetic.PREFILL, "large": synthetic.LARGE, "pr1": synthetic.PR1}[name]
@@ -310,7 +337,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from bit_nf4_quantized_07_b200 import api, synthetic
+    from bit_nf4_quantized_07_b200 import api, dp, synthetic
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -379,8 +406,7 @@ def run_ours(args):
         if marks is not None:
             marks[4].record(stream)
         if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+            dp.allreduce_adapter_grads(dA, dB)
 
     for i in range(args.warmup):
         step(i)
@@ -411,9 +437,7 @@ def run_ours(args):
         sec["bwd"] += m[3].elapsed_time(m[4])
     sec = {k: v / args.steps for k, v in sec.items()}
     if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+        elapsed_ms = dp.max_over_ranks(elapsed_ms, device=dev)
 
     # End to end through the C ABI with host buffers: copies inside the timed region.
     W, X, A, B, dYs = sets[0]
@@ -430,8 +454,7 @@ def run_ours(args):
         api.qlora_linear_fwd(wq, dXi, dAi, dBi, cfg.s, Y=Y, U_out=U, ws=ws_f)
         api.qlora_linear_bwd(wq, dXi, dAi, dBi, cfg.s, ddY, U=U, dX=dX, dA=dA, dB=dB, ws=ws_b)
         if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+            dp.allreduce_adapter_grads(dA, dB)
         for h, d in ((oY, Y), (odX, dX), (odA, dA), (odB, dB)):
             h.copy_(d, non_blocking=True)
 
@@ -451,9 +474,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+        e2e_ms = dp.max_over_ranks(e2e_ms, device=dev)
 
     flops = cfg.fwd_flops() + cfg.bwd_flops()
     ms_per_step = elapsed_ms / args.steps
@@ -464,7 +485,7 @@ def run_ours(args):
     fwd_tflops = cfg.fwd_flops() / (sec["fwd"] * 1e-3) / 1e12
     roof = {"kernel": "qlora_linear_fwd (fused NF4 GEMM + U)", "bound": "tensor", "achieved": fwd_tflops,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": fwd_tflops / peaks["bf16_tflops"],
-            "traffic": None, "peak_source": peaks["source"] + " bf16 burst"}
+            "traffic": _recorded_traffic(cfg.name), "peak_source": peaks["source"] + " bf16 burst"}
     parts = {
         "quantize_dq_GBs": numel * qb / (sec["quantize_dq"] * 1e-3) / 1e9,
         "dequant_GBs": numel * db / (sec["dequant"] * 1e-3) / 1e9,
@@ -514,9 +535,16 @@ def main():
     ap.add_argument("--workload", choices=["prefill", "large", "pr1"], default="prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode-shape and codec-sweep measurements")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode-shape measurement and print it (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.decode_only:
+        import torch
+        from bit_nf4_quantized_07_b200 import api
+        print(json.dumps(measure_decode(api, torch.device("cuda", 0), copies=16, reps=2)))
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -210,7 +210,8 @@ qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     // U = X A^T (and s*U for the adapter MMA), then the fused weight GEMM.
     e = qln::launch_lora_down(X, n, w->cols, A, r, s, U, sU, pU, cs, kSplitTargetSms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
-    e = fused_gemm(w, false, X, n, sU, B, r, Y, status, cs, sms);
+    if (qln::nf4_gemv_supported(w, n, r)) e = qln::launch_nf4_gemv(w, X, n, sU, B, r, Y, cs);
+    else e = fused_gemm(w, false, X, n, sU, B, r, Y, status, cs, sms);
     return from_cuda(e);
 }
 
