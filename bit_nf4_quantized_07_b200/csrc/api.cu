@@ -66,7 +66,9 @@ FwdWs fwd_layout(int64_t rows, int64_t cols, int64_t n, int r) {
     L.sU = 256;
     L.U = L.sU + nr;
     L.pU = L.U + nr;
-    L.total = L.pU + round256(qln::lora_down_partial_bytes(n, cols, r, kSplitTargetSms));
+    const size_t pl = qln::lora_down_partial_bytes(n, cols, r, kSplitTargetSms);
+    const size_t pg = qln::nf4_gemv_upart_bytes(n, r);
+    L.total = L.pU + round256(pl > pg ? pl : pg);
     return L;
 }
 
@@ -205,13 +207,17 @@ qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     uint16_t *sU = reinterpret_cast<uint16_t *>(wsb + L.sU);
     uint16_t *U = U_out ? U_out : reinterpret_cast<uint16_t *>(wsb + L.U);
     float *pU = reinterpret_cast<float *>(wsb + L.pU);
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
+    cudaError_t e = cudaMemsetAsync(status, 0, 2 * sizeof(int), cs);  // status word + decode counter
     if (e != cudaSuccess) return QLN_ERR_CUDA;
+    if (qln::nf4_gemv_supported(w, n, r)) {
+        // decode-sized n: one cooperative launch forms U and the whole forward
+        e = qln::launch_nf4_gemv(w, X, n, A, B, r, s, Y, U_out, pU, status + 1, status, cs, sms);
+        return from_cuda(e);
+    }
     // U = X A^T (and s*U for the adapter MMA), then the fused weight GEMM.
     e = qln::launch_lora_down(X, n, w->cols, A, r, s, U, sU, pU, cs, kSplitTargetSms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
-    if (qln::nf4_gemv_supported(w, n, r)) e = qln::launch_nf4_gemv(w, X, n, sU, B, r, Y, cs);
-    else e = fused_gemm(w, false, X, n, sU, B, r, Y, status, cs, sms);
+    e = fused_gemm(w, false, X, n, sU, B, r, Y, status, cs, sms);
     return from_cuda(e);
 }
 

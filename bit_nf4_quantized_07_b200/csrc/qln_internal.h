@@ -45,11 +45,15 @@ cudaError_t launch_nf4_mma_gemm(const qln_nf4_weight *w, bool trans, const uint1
                                 const uint16_t *lact, const uint16_t *lw, int r, uint16_t *out,
                                 int *status, cudaStream_t st, int num_sms);
 
-// nf4_gemv.cu: fused NF4 decode + forward for decode-sized n (<= 32).
-//   Y[t][o] = bf16(sum_k X[t][k] W'[o][k] + sum_j sU[t][j] B[o][j])
+// nf4_gemv.cu: the whole forward for decode-sized n (<= 32) in one cooperative
+// launch: U = X A^T, Y = bf16(X W'^T + bf16(s U) B^T), U_out = bf16(U).
+//   upart: fp32 scratch of nf4_gemv_upart_bytes(n, r); counter: int zeroed
+//   before the launch; status: the status word.
 bool nf4_gemv_supported(const qln_nf4_weight *w, int64_t n, int r);
-cudaError_t launch_nf4_gemv(const qln_nf4_weight *w, const uint16_t *X, int64_t n, const uint16_t *sU,
-                            const uint16_t *B, int r, uint16_t *Y, cudaStream_t st);
+size_t nf4_gemv_upart_bytes(int64_t n, int r);
+cudaError_t launch_nf4_gemv(const qln_nf4_weight *w, const uint16_t *X, int64_t n, const uint16_t *A,
+                            const uint16_t *B, int r, float s, uint16_t *Y, uint16_t *U_out, float *upart,
+                            int *counter, int *status, cudaStream_t st, int num_sms);
 
 // nf4_gemm_sm100.cu: fused NF4 decode + tcgen05 GEMM (TMA, TMEM accumulators).
 cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16_t *act, int64_t n,

@@ -76,6 +76,25 @@ def test_decode_forward(batch):
     _compare("Y", got["Y"], Y)
 
 
+DECODE_SHAPES = [
+    synthetic.custom("dec_8192x512_n24_r32", 8192, 512, 24, 32, s=1.5, index=21),    # >1 row group per CTA
+    synthetic.custom("dec_4096x1024_n32_r128", 4096, 1024, 32, 128, s=0.5, index=22),
+    synthetic.custom("dec_1024x4096_n5_r8", 1024, 4096, 5, 8, s=2.0, index=23),
+    synthetic.custom("dec_256x2048_n9_r16", 256, 2048, 9, 16, s=2.0, index=24),      # 8 row groups exactly
+]
+
+
+@pytest.mark.parametrize("cfg", DECODE_SHAPES, ids=lambda c: c.name)
+@pytest.mark.parametrize("dq", [True, False], ids=["dq", "plain"])
+def test_decode_shaped_forward(cfg, dq):
+    w, X, A, B, dY = workload(cfg)
+    ow = OracleWeight(w, double_quant=dq)
+    got = _run(cfg, w, X, A, B, dY, double_quant=dq, backward=False)
+    Y, U = forward_ref(ow, X, A, B, cfg.s)
+    _compare("U", got["U"], U)
+    _compare("Y", got["Y"], Y)
+
+
 def test_adapter_off_matches_cublas_on_materialised_weight():
     """B = 0 (or s = 0): the fused forward reduces to X W'^T; cross-check it
     against torch.matmul (cuBLAS) on nf4_dequant's materialised W'."""
