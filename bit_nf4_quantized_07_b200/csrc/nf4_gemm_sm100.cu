@@ -11,10 +11,12 @@
 //   forward (TRANS = false): out[t][m] = sum_k X[t][k] W'[m][k]  + sum_j sU[t][j] B[m][j]
 //   dX      (TRANS = true) : out[t][m] = sum_k dY[t][k] W'[k][m] + sum_j sG[t][j] A[j][m]
 //
-// One CTA computes a (128*MT) (m) x BN (tokens, <= 256) tile as MT
+// One CTA computes a (128*MT) (m) x (NT*BN) (tokens) tile as MT*NT <= 2
 // accumulators of 128 TMEM lanes x BN columns, K in steps of 64.  MT = 2 lets
-// two 128-row weight tiles share every activation tile, halving the
-// activation bytes each FLOP pulls from L2.
+// two 128-row weight tiles share every activation tile (half the activation
+// bytes per FLOP); NT = 2 lets every decoded weight tile serve two token
+// tiles (half the decode work per FLOP, the integer-pipe bound of the
+// decoders).  The shape is chosen per call.
 //   A_op (weights): decoded by 128*MT threads (one 64-wide row block each)
 //     into the canonical 128-byte-swizzled layout, K-major for the forward
 //     (W' rows along K) and MN-major for dX (W' rows are the K index, their
@@ -37,18 +39,19 @@ namespace tc {
 
 constexpr int kBM = 128;   // rows per accumulator (TMEM lanes)
 constexpr int kBK = 64;
-constexpr int kMaxBN = 256;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
 
-template <int MT>
+template <int MT, int NT>
 struct Cfg {
-    static constexpr int kStages = MT == 1 ? 4 : 3;
+    static_assert(MT * NT <= 2, "two TMEM accumulators of up to 256 columns at most");
+    static constexpr int kStages = MT * NT == 1 ? 4 : 3;
+    static constexpr int kMaxBN = NT == 1 ? 256 : 208;     // tokens per accumulator
     static constexpr int kDecThreads = 128 * MT;
     static constexpr int kThreads = 64 + kDecThreads;
-    static constexpr uint32_t kABytes = 16384u * MT;       // MT x (128 rows x 64 K) bf16
-    static constexpr uint32_t kBBytes = kMaxBN * kBK * 2;  // 32 KB
-    static constexpr uint32_t kCBytes = 4096u * MT;        // codes of the A tile
-    static constexpr uint32_t kTmemCols = 256u * MT;
+    static constexpr uint32_t kABytes = 16384u * MT;        // MT x (128 rows x 64 K) bf16
+    static constexpr uint32_t kBBytes = NT * kMaxBN * kBK * 2;
+    static constexpr uint32_t kCBytes = 4096u * MT;         // codes of the A tile
+    static constexpr uint32_t kTmemCols = 256u * MT * NT;
     static constexpr uint32_t kOffA = 0;
     static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
     static constexpr uint32_t kOffC = kOffB + kStages * kBBytes;
@@ -71,15 +74,15 @@ struct Params {
     int *status;
     int KT;            // weight k-steps
     int RT;            // adapter k-steps
-    int BN;            // tokens per tile (multiple of 16, <= 256)
+    int BN;            // tokens per accumulator (multiple of 16)
 };
 
-template <bool TRANS, int MT>
-__global__ void __launch_bounds__(Cfg<MT>::kThreads, 1)
+template <bool TRANS, int MT, int NT>
+__global__ void __launch_bounds__(Cfg<MT, NT>::kThreads, 1)
 nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_act,
                    const __grid_constant__ CUtensorMap tm_lw, const __grid_constant__ CUtensorMap tm_lact,
                    const Params p) {
-    using C = Cfg<MT>;
+    using C = Cfg<MT, NT>;
     constexpr int S = C::kStages;
     constexpr int TM = kBM * MT;  // rows of the CTA tile
     extern __shared__ uint8_t smem_raw[];
@@ -96,7 +99,7 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     volatile int *epi_go = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t0 = (int64_t)blockIdx.x * p.BN;
+    const int64_t t0 = (int64_t)blockIdx.x * NT * p.BN;  // NT accumulators of BN tokens each
     const int64_t m0 = (int64_t)blockIdx.y * TM;
     const int nsteps = p.KT + p.RT;
 
@@ -132,7 +135,8 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            const uint32_t bbytes = (uint32_t)p.BN * kBK * 2;
+            const uint32_t bsub = (uint32_t)p.BN * kBK * 2;  // one token sub-tile
+            const uint32_t bbytes = NT * bsub;
             int issued = 0;
             for (int kt = 0; kt < nsteps; ++kt) {
                 const int s = kt % S;
@@ -154,7 +158,9 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                             tma_load_2d(sC + 2048 * d, &tm_codes, (int32_t)(m0 / 2) + 32 * d, kt * kBK, code_full(s));
                     }
                     mbar_arrive_expect_tx(tma_full(s), bbytes);
-                    tma_load_2d(sB, &tm_act, kt * kBK, (int32_t)t0, tma_full(s));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        tma_load_2d(sB + nt * bsub, &tm_act, kt * kBK, (int32_t)(t0 + nt * p.BN), tma_full(s));
                 } else {
                     const int a = kt - p.KT;
                     mbar_arrive_expect_tx(tma_full(s), C::kABytes + bbytes);
@@ -165,7 +171,9 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                         for (int d = 0; d < 2 * MT; ++d)
                             tma_load_2d(sA + 8192 * d, &tm_lw, (int32_t)m0 + 64 * d, a * kBK, tma_full(s));
                     }
-                    tma_load_2d(sB, &tm_lact, a * kBK, (int32_t)t0, tma_full(s));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        tma_load_2d(sB + nt * bsub, &tm_lact, a * kBK, (int32_t)(t0 + nt * p.BN), tma_full(s));
                 }
                 issued = kt + 1;
             }
@@ -195,14 +203,17 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 #pragma unroll
                 for (int sub = 0; sub < MT; ++sub) {
 #pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k) {
-                        // K-major: next 16 K elements are 32 bytes further inside the
-                        // swizzled 128-byte rows.  MN-major: next two 8-row K groups.
-                        const uint32_t aS = sA + sub * 16384;
-                        const uint64_t adesc = TRANS ? smem_desc_sw128(aS + k * 2048, 8192, 1024)
-                                                     : smem_desc_sw128(aS + k * 32, 16, 1024);
-                        const uint64_t bdesc = smem_desc_sw128(sB + k * 32, 16, 1024);
-                        tc_mma_ss(tmem_d + sub * 256, adesc, bdesc, idesc, (kt | k) != 0 ? 1u : 0u);
+                    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                        for (int k = 0; k < kBK / 16; ++k) {
+                            // K-major: next 16 K elements are 32 bytes further inside the
+                            // swizzled 128-byte rows.  MN-major: next two 8-row K groups.
+                            const uint32_t aS = sA + sub * 16384;
+                            const uint64_t adesc = TRANS ? smem_desc_sw128(aS + k * 2048, 8192, 1024)
+                                                         : smem_desc_sw128(aS + k * 32, 16, 1024);
+                            const uint64_t bdesc = smem_desc_sw128(sB + nt * p.BN * 128 + k * 32, 16, 1024);
+                            tc_mma_ss(tmem_d + (sub * NT + nt) * 256, adesc, bdesc, idesc, (kt | k) != 0 ? 1u : 0u);
+                        }
                     }
                 }
                 tc_commit(empty(s));
@@ -300,21 +311,25 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         if (*epi_go) {
             tc_fence_after();
             const int q = warp & 3;              // TMEM lane quadrant of this warp
-            const int sub = (warp - 2) >> 2;     // accumulator of this warp
-            uint16_t *Os = reinterpret_cast<uint16_t *>(smem);  // [BN][TM] bf16; all MMAs are done
+            const int sub = (warp - 2) >> 2;     // weight sub-tile of this warp
+            uint16_t *Os = reinterpret_cast<uint16_t *>(smem);  // [NT*BN][TM] bf16; all MMAs are done
             const int m = sub * kBM + q * 32 + lane;
-            for (int c0 = 0; c0 < p.BN; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)(sub * 256 + c0), v);
-                tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (c0 + j < p.BN)
-                        Os[(c0 + j) * TM + m] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+            for (int nt = 0; nt < NT; ++nt) {
+                for (int c0 = 0; c0 < p.BN; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)((sub * NT + nt) * 256 + c0), v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (c0 + j < p.BN)
+                            Os[(nt * p.BN + c0 + j) * TM + m] =
+                                __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+                }
             }
             asm volatile("bar.sync 1, %0;" ::"n"(C::kDecThreads) : "memory");
             constexpr int kChunksPerRow = TM / 8;
-            const int chunks = p.BN * kChunksPerRow;
+            const int chunks = NT * p.BN * kChunksPerRow;
             for (int idx = dt; idx < chunks; idx += C::kDecThreads) {
                 const int row = idx / kChunksPerRow, ch = idx % kChunksPerRow;
                 const int64_t t = t0 + row;
@@ -369,37 +384,53 @@ static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const vo
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tokens per tile: a multiple of 16 in [128, 256] (or all of n when n <= 256)
-// chosen to waste the least on the last partial wave of CTAs (one CTA per SM)
-// and on padding the last token tile, preferring wide tiles.
-static int choose_bn(int64_t n, int64_t mtiles, int num_sms) {
-    const int64_t n16 = (n + 15) / 16 * 16;
-    if (n16 <= kMaxBN) return (int)n16;
-    int best = kMaxBN;
-    double best_eff = -1.0;
-    for (int bn = kMaxBN; bn >= 128; bn -= 16) {
-        const int64_t ttiles = (n + bn - 1) / bn;
-        const int64_t tiles = ttiles * mtiles;
-        const int64_t rounds = (tiles + num_sms - 1) / num_sms;
-        // narrower tiles decode each weight for fewer tokens: a mild penalty
-        const double eff = ((double)tiles / (double)(rounds * num_sms)) * ((double)n / (double)(ttiles * bn)) -
-                           0.1 * (double)(kMaxBN - bn) / 128.0;
-        if (eff > best_eff + 1e-3) {
-            best_eff = eff;
-            best = bn;
+// Tile shape per call.  Candidates: MT weight sub-tiles of 128 rows and NT
+// token sub-tiles of BN tokens (MT * NT <= 2, BN a multiple of 16).  A simple
+// cost model picks the fastest: one CTA per SM; a k-step costs the larger of
+// its tensor time (at the measured dense rate, about 5700 FLOP per cycle per
+// SM) and its decode time (about 0.12 cycle per decoded weight, integer-pipe
+// bound), plus a fixed cost per tile; waves are counted whole.
+struct TileShape {
+    int MT, NT, BN;
+};
+
+static TileShape choose_shape(int64_t M, int64_t K, int64_t n, int num_sms) {
+    const int64_t ksteps = K / kBK + 1;
+    TileShape best{1, 1, 128};
+    double best_cost = 1e300;
+    const int shapes[3][2] = {{2, 1}, {1, 2}, {1, 1}};
+    for (const auto &sh : shapes) {
+        const int MT = sh[0], NT = sh[1];
+        if ((M % (kBM * MT)) != 0) continue;
+        const int maxbn = NT == 1 ? 256 : 208;
+        for (int bn = maxbn; bn >= 16; bn -= 16) {
+            if (bn < 128 && (int64_t)NT * bn < n) break;  // narrow tiles only for small n
+            const int64_t tile_tok = (int64_t)NT * bn;
+            const int64_t ttiles = (n + tile_tok - 1) / tile_tok;
+            const int64_t tiles = ttiles * (M / (kBM * MT));
+            const int64_t rounds = (tiles + num_sms - 1) / num_sms;
+            const double mma = 2.0 * kBM * MT * tile_tok * kBK / 5700.0;
+            const double dec = 0.12 * 8192.0 * MT;
+            const double tile = ksteps * (mma > dec ? mma : dec) + 4000.0;
+            // ties go to the fewest padded tokens
+            const double cost = rounds * tile * (1.0 + 1e-4 * (double)(ttiles * tile_tok - n) / (double)n);
+            if (cost < best_cost * 0.999) {
+                best_cost = cost;
+                best = TileShape{MT, NT, bn};
+            }
         }
     }
     return best;
 }
 
-template <bool TRANS, int MT>
+template <bool TRANS, int MT, int NT>
 static cudaError_t launch_t(const CUtensorMap &m_codes, const CUtensorMap &m_act, const CUtensorMap &m_lw,
                             const CUtensorMap &m_lact, const Params &p, dim3 grid, cudaStream_t st) {
-    using C = Cfg<MT>;
-    cudaError_t e = cudaFuncSetAttribute(nf4_tc_gemm_kernel<TRANS, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
+    using C = Cfg<MT, NT>;
+    cudaError_t e = cudaFuncSetAttribute(nf4_tc_gemm_kernel<TRANS, MT, NT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    nf4_tc_gemm_kernel<TRANS, MT><<<grid, C::kThreads, C::kSmemBytes, st>>>(m_codes, m_act, m_lw, m_lact, p);
+    nf4_tc_gemm_kernel<TRANS, MT, NT><<<grid, C::kThreads, C::kSmemBytes, st>>>(m_codes, m_act, m_lw, m_lact, p);
     note_launch();
     return cudaGetLastError();
 }
@@ -420,9 +451,9 @@ cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16
     const int64_t rows = w->rows, cols = w->cols;
     const int64_t M = trans ? cols : rows;
     const int64_t K = trans ? rows : cols;
-    const int MT = (M % 256) == 0 ? 2 : 1;
+    const TileShape shape = choose_shape(M, K, n, num_sms > 0 ? num_sms : 148);
+    const int MT = shape.MT, NT = shape.NT, BN = shape.BN;
     const int TM = kBM * MT;
-    const int BN = choose_bn(n, M / TM, num_sms > 0 ? num_sms : 148);
     CUtensorMap m_codes, m_act, m_lw, m_lact;
     bool ok = true;
     // codes as bytes [rows][cols/2]
@@ -451,11 +482,15 @@ cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16
     p.KT = (int)(K / kBK);
     p.RT = (r + kBK - 1) / kBK;
     p.BN = BN;
-    dim3 grid((unsigned)((n + BN - 1) / BN), (unsigned)(M / TM));
-    if (trans) return MT == 2 ? launch_t<true, 2>(m_codes, m_act, m_lw, m_lact, p, grid, st)
-                              : launch_t<true, 1>(m_codes, m_act, m_lw, m_lact, p, grid, st);
-    return MT == 2 ? launch_t<false, 2>(m_codes, m_act, m_lw, m_lact, p, grid, st)
-                   : launch_t<false, 1>(m_codes, m_act, m_lw, m_lact, p, grid, st);
+    dim3 grid((unsigned)((n + (int64_t)NT * BN - 1) / ((int64_t)NT * BN)), (unsigned)(M / TM));
+    if (trans) {
+        if (MT == 2) return launch_t<true, 2, 1>(m_codes, m_act, m_lw, m_lact, p, grid, st);
+        if (NT == 2) return launch_t<true, 1, 2>(m_codes, m_act, m_lw, m_lact, p, grid, st);
+        return launch_t<true, 1, 1>(m_codes, m_act, m_lw, m_lact, p, grid, st);
+    }
+    if (MT == 2) return launch_t<false, 2, 1>(m_codes, m_act, m_lw, m_lact, p, grid, st);
+    if (NT == 2) return launch_t<false, 1, 2>(m_codes, m_act, m_lw, m_lact, p, grid, st);
+    return launch_t<false, 1, 1>(m_codes, m_act, m_lw, m_lact, p, grid, st);
 }
 
 }  // namespace qln
