@@ -46,16 +46,21 @@ def _load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# Sources of the kernels a prefill-shaped qlora_linear_fwd launches (adapter
+# product + fold, fused tcgen05 GEMM) and of the dispatch that picks them.
+FWD_PATH_SOURCES = ("api.cu", "lora_small.cu", "nf4_gemm_sm100.cu", "qln_common.cuh", "qln_internal.h",
+                    "tc_ptx.cuh")
+
+
 def _kernel_sources_sha1():
-    """SHA-1 over the library's CUDA sources: identifies the kernels a
-    committed ncu record was taken from."""
+    """SHA-1 over the CUDA sources of the forward path: identifies the kernels
+    a committed ncu traffic record was taken from."""
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "bit_nf4_quantized_07_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode() + b"\0" + f.read())
+    for fn in FWD_PATH_SOURCES:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + b"\0" + f.read())
     return h.hexdigest()
 
 
