@@ -234,11 +234,12 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # Secondary measurements (reported under "parts", not part of the step)
 # ---------------------------------------------------------------------------
-def measure_decode(api, dev, copies=64, reps=3):
+def measure_decode(api, dev, copies=64, reps=5):
     """Decode-shaped forward (4096 x 4096, r = 16, n in {1, 4, 16}) over
-    `copies` distinct NF4 + DQ weights (~553 MB, far above L2), one call per
-    weight, CUDA events around each sweep.  GB/s counts the algorithmic bytes
-    of a call: codes, DQ constants, X, A, B, U and Y."""
+    `copies` distinct NF4 + DQ weights (~553 MB, far above L2): one call per
+    weight, captured once as a CUDA graph and replayed `reps` times between
+    CUDA events, reported per call.  GB/s counts the algorithmic bytes of a
+    call: codes, DQ constants, X, A, B, U and Y."""
     import torch
     from bit_nf4_quantized_07_b200 import synthetic
     cfg = synthetic.DECODE[1]
@@ -253,28 +254,40 @@ def measure_decode(api, dev, copies=64, reps=3):
     A = (torch.randn(r, cols, generator=gen, device=dev) * cfg.ab_sigma).to(torch.bfloat16)
     B = (torch.randn(rows, r, generator=gen, device=dev) * cfg.ab_sigma).to(torch.bfloat16)
     out = {}
-    stream = torch.cuda.current_stream()
     for n in (1, 4, 16):
         X = torch.randn(n, cols, generator=gen, device=dev).to(torch.bfloat16)
         Y = torch.empty(n, rows, dtype=torch.bfloat16, device=dev)
         U = torch.empty(n, r, dtype=torch.bfloat16, device=dev)
         ws = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_FWD, rows, cols, n, r), dev)
-        for w in weights[:4]:
-            api.qlora_linear_fwd(w, X, A, B, 2.0, Y=Y, U_out=U, ws=ws)
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for w in weights[:4]:
+                api.qlora_linear_fwd(w, X, A, B, 2.0, Y=Y, U_out=U, ws=ws)
+        torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for w in weights:
+                api.qlora_linear_fwd(w, X, A, B, 2.0, Y=Y, U_out=U, ws=ws)
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(reps):
-            for w in weights:
-                api.qlora_linear_fwd(w, X, A, B, 2.0, Y=Y, U_out=U, ws=ws)
+            graph.replay()
         e1.record(stream)
         torch.cuda.synchronize()
         per_call = e0.elapsed_time(e1) / (reps * copies) * 1e-3
+        del graph
         nb = rows * cols // 64
         wbytes = rows * cols // 2 + nb + 4 * ((nb + 255) // 256) + 4
         bytes_call = wbytes + 2 * n * cols + 2 * r * cols + 2 * rows * r + 2 * n * r + 2 * n * rows
         out[f"n{n}"] = {"us_per_call": per_call * 1e6, "GBs": bytes_call / per_call / 1e9,
-                        "TFLOPs": 2 * n * (rows * cols + r * cols + rows * r) / per_call / 1e12}
+                        "TFLOPs": 2 * n * (rows * cols + r * cols + rows * r) / per_call / 1e12,
+                        "timing": f"CUDA graph of {copies} calls on {copies} weight copies, {reps} replays"}
     del weights
     torch.cuda.empty_cache()
     return out

@@ -44,9 +44,11 @@ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int kSplitTargetSms = 148;
 
 // Workspace layout of the linear calls (all offsets 256-byte aligned):
-//   [0, 256)        int32 device status word (0 = QLN_OK) + reserved
+//   [0, 256)        header: int32 device status word (0 = QLN_OK) at 0, the
+//                   decode-sized forward's counters at 64 and 128
 //   fwd: sU [n][r] bf16, U [n][r] bf16 (used when U_out is NULL),
-//        split-K partials of U (fp32)
+//        split-K partials of U (fp32) -- or, for decode-sized n, the parts of
+//        U and bf16(s U) of the one-launch forward
 //   bwd: Bt [r][dout] bf16, G [n][r] bf16, sG [n][r] bf16, U [n][r] bf16,
 //        split-K partials of G / U (fp32, reused), dA partials, dB partials
 // Split counts are planned for a fixed SM count so that the workspace size
@@ -60,22 +62,22 @@ struct BwdWs {
 };
 
 FwdWs fwd_layout(int64_t rows, int64_t cols, int64_t n, int r) {
-    (void)rows;
     FwdWs L;
     const size_t nr = round256((size_t)n * r * 2);
-    L.sU = 256;
+    (void)rows;
+    L.sU = qln::kWsHeaderBytes;
     L.U = L.sU + nr;
     L.pU = L.U + nr;
-    const size_t pl = qln::lora_down_partial_bytes(n, cols, r, kSplitTargetSms);
-    const size_t pg = qln::nf4_gemv_upart_bytes(n, r);
-    L.total = L.pU + round256(pl > pg ? pl : pg);
+    const size_t generic = L.pU + round256(qln::lora_down_partial_bytes(n, cols, r, kSplitTargetSms));
+    const size_t decode = qln::kWsHeaderBytes + round256(qln::nf4_gemv_ws_bytes(n, r));
+    L.total = generic > decode ? generic : decode;
     return L;
 }
 
 BwdWs bwd_layout(int64_t rows, int64_t cols, int64_t n, int r) {
     BwdWs L;
     const size_t nr = round256((size_t)n * r * 2);
-    L.Bt = 256;
+    L.Bt = qln::kWsHeaderBytes;
     L.G = L.Bt + round256((size_t)rows * r * 2);
     L.sG = L.G + nr;
     L.U = L.sG + nr;
@@ -207,13 +209,13 @@ qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     uint16_t *sU = reinterpret_cast<uint16_t *>(wsb + L.sU);
     uint16_t *U = U_out ? U_out : reinterpret_cast<uint16_t *>(wsb + L.U);
     float *pU = reinterpret_cast<float *>(wsb + L.pU);
-    cudaError_t e = cudaMemsetAsync(status, 0, 2 * sizeof(int), cs);  // status word + decode counter
-    if (e != cudaSuccess) return QLN_ERR_CUDA;
     if (qln::nf4_gemv_supported(w, n, r)) {
-        // decode-sized n: one cooperative launch forms U and the whole forward
-        e = qln::launch_nf4_gemv(w, X, n, A, B, r, s, Y, U_out, pU, status + 1, status, cs, sms);
-        return from_cuda(e);
+        // decode-sized n: one launch forms U and the whole forward; it clears
+        // the status word itself, so no memset precedes it
+        return from_cuda(qln::launch_nf4_gemv(w, X, n, A, B, r, s, Y, U_out, ws, cs));
     }
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
+    if (e != cudaSuccess) return QLN_ERR_CUDA;
     // U = X A^T (and s*U for the adapter MMA), then the fused weight GEMM.
     e = qln::launch_lora_down(X, n, w->cols, A, r, s, U, sU, pU, cs, kSplitTargetSms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;

@@ -384,6 +384,15 @@ static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const vo
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+}  // namespace tc
+
+bool make_tensor_map_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t inner,
+                        uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    return tc::make_map(m, dt, esize, base, inner, outer, box_inner, box_outer, sw);
+}
+
+namespace tc {
+
 // Tile shape per call.  Candidates: MT weight sub-tiles of 128 rows and NT
 // token sub-tiles of BN tokens (MT * NT <= 2, BN a multiple of 16).  A simple
 // cost model picks the fastest: one CTA per SM; a k-step costs the larger of

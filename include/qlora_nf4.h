@@ -44,7 +44,7 @@
  *   QLN_ERR_CUDA (cudaGetLastError).  Kernels that wait on on-chip barriers
  *   give up after a bounded number of polls and write QLN_ERR_TIMEOUT into the
  *   int32 status word at byte offset 0 of the workspace; read it after the
- *   stream has synchronised (0 = QLN_OK).
+ *   stream has synchronised (0 = QLN_OK).  Each workspace call clears it.
  */
 #ifndef QLORA_NF4_H
 #define QLORA_NF4_H
@@ -180,7 +180,11 @@ QLN_API qln_status nf4_dequant(const qln_nf4_weight *w, uint16_t *out, void *str
  *   Y [n][dout] bf16 out = bf16_RN(X W'^T + s U B^T) with fp32 accumulation,
  *   U_out [n][r] bf16 out (nullable): U = bf16_RN(X A^T), unscaled, for reuse
  *   by qlora_linear_bwd.
- * W' is decoded tile by tile on chip and never written to HBM.
+ * W' is decoded tile by tile on chip and never written to HBM.  For n <= 32
+ * the whole call is one launch of thread-block clusters (U, the weight
+ * stream and the adapter term); its split-K sums are folded in an order fixed
+ * by the shape, so results do not depend on timing or on the device's SM
+ * count.
  *   ws: at least qln_workspace_bytes(QLN_OP_LINEAR_FWD, dout, din, n, r)
  *   bytes, 256-byte aligned; byte 0 holds the device status word afterwards.
  * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE (n < 1; r not a multiple of 8 in

@@ -80,7 +80,11 @@ DECODE_SHAPES = [
     synthetic.custom("dec_8192x512_n24_r32", 8192, 512, 24, 32, s=1.5, index=21),    # >1 row group per CTA
     synthetic.custom("dec_4096x1024_n32_r128", 4096, 1024, 32, 128, s=0.5, index=22),
     synthetic.custom("dec_1024x4096_n5_r8", 1024, 4096, 5, 8, s=2.0, index=23),
-    synthetic.custom("dec_256x2048_n9_r16", 256, 2048, 9, 16, s=2.0, index=24),      # 8 row groups exactly
+    synthetic.custom("dec_256x2048_n9_r16", 256, 2048, 9, 16, s=2.0, index=24),
+    synthetic.custom("dec_128x11008_n3_r24", 128, 11008, 3, 24, s=1.0, index=25),   # ragged K ranges, 3 U warp columns
+    synthetic.custom("dec_64x64_n32_r8", 64, 64, 32, 8, s=2.0, index=26),           # one block: empty U sub-ranges
+    synthetic.custom("dec_512x768_n17_r40", 512, 768, 17, 40, s=0.5, index=27),     # 3 token tiles, r % 16 == 8
+    synthetic.custom("dec_1024x1536_n25_r64", 1024, 1536, 25, 64, s=1.5, index=28), # 4 token tiles
 ]
 
 
@@ -91,6 +95,49 @@ def test_decode_shaped_forward(cfg, dq):
     ow = OracleWeight(w, double_quant=dq)
     got = _run(cfg, w, X, A, B, dY, double_quant=dq, backward=False)
     Y, U = forward_ref(ow, X, A, B, cfg.s)
+    _compare("U", got["U"], U)
+    _compare("Y", got["Y"], Y)
+
+
+def test_decode_forward_repeats_and_replays_bit_identically():
+    """The one-launch decode forward folds its split-K partials in an order
+    fixed by the shape: back-to-back calls on one workspace, a call after a
+    backward on the same workspace, and CUDA graph replays must all give the
+    same bits."""
+    cfg = synthetic.custom("rep_1024x2048_n12_r16", 1024, 2048, 12, 16, s=2.0, index=29)
+    w, X, A, B, dY = workload(cfg)
+    wq = _gpu_weight(w)
+    Xd, Ad, Bd, dYd = bf16_to_dev(X), bf16_to_dev(A), bf16_to_dev(B), bf16_to_dev(dY)
+    nbytes = max(api.workspace_bytes(api.OP_LINEAR_FWD, cfg.dout, cfg.din, cfg.n, cfg.r),
+                 api.workspace_bytes(api.OP_LINEAR_BWD, cfg.dout, cfg.din, cfg.n, cfg.r))
+    ws = api.alloc_workspace(nbytes)
+    Y0, U0 = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s, ws=ws)
+    for _ in range(3):
+        Y1, U1 = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s, ws=ws)
+        assert torch.equal(Y0, Y1) and torch.equal(U0, U1)
+    api.qlora_linear_bwd(wq, Xd, Ad, Bd, cfg.s, dYd, U=U0, ws=ws)
+    Y2, U2 = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s, ws=ws)
+    assert torch.equal(Y0, Y2) and torch.equal(U0, U2)
+    assert api.device_status(ws) == 0
+    Yg = torch.empty_like(Y0)
+    Ug = torch.empty_like(U0)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s, Y=Yg, U_out=Ug, ws=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(4):
+            api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s, Y=Yg, U_out=Ug, ws=ws)
+    Yg.zero_()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(Y0, Yg) and torch.equal(U0, Ug)
+    got = {"Y": f64(dev_bf16_bits(Yg)), "U": f64(dev_bf16_bits(Ug))}
+    Y, U = forward_ref(OracleWeight(w), X, A, B, cfg.s)
     _compare("U", got["U"], U)
     _compare("Y", got["Y"], Y)
 
