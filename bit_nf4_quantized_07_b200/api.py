@@ -118,8 +118,10 @@ def workspace_bytes(op: int, rows: int, cols: int = 0, n: int = 0, r: int = 0) -
 
 
 def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
-    """Device scratch (torch-allocated, 256-byte aligned by the caching allocator)."""
-    t = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+    """Device scratch (torch-allocated, 256-byte aligned by the caching
+    allocator), zero-filled: the counters in the workspace header must start
+    at zero, and every call leaves them there."""
+    t = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
     assert t.data_ptr() % 256 == 0
     return t
 

@@ -25,10 +25,11 @@
 //   1. At launch every warp requests the code bytes of its first two units
 //      (one 2-D TMA copy each, 16 rows x 128 bytes, into its two-stage ring);
 //      the CTA stages its K range of X and builds the decode table.
-//   2. U = X A^T is formed once for the grid: CTAs 0..UG-1 each take one of UG
-//      K ranges, store the fp32 part in the workspace and count themselves in;
-//      the last of them folds the parts in order into bf16(s U) (and U_out) and
-//      raises the ready flag.
+//   2. U = X A^T is formed once for the grid by UG = 8 extra CTAs that follow
+//      the decode clusters and do nothing else: each takes one of 8 K ranges,
+//      stores the fp32 part in the workspace and counts itself in; the last of
+//      them folds the parts in order into bf16(s U) (and U_out) and raises the
+//      ready flag.  The decode CTAs never wait for U before their fold.
 //   3. Each round a warp decodes its unit into the register layout of the
 //      m16n8k16 A operand (a byte of two codes -> a BF16 pair from the table),
 //      multiplies with X per block, scales by ahat, stores the fp32 partial
@@ -37,7 +38,9 @@
 //      rounds and one cluster barrier every CTA folds its tiles from its own
 //      shared memory in a fixed order (CTA rank, then sub-range), adds
 //      bf16(s U) B^T (after a bounded wait on the ready flag) as one more MMA
-//      pass and writes Y.
+//      pass and writes Y.  Each decode CTA counts itself out once it has read
+//      bf16(s U); the last one resets the workspace counters for the next call,
+//      so no memset precedes a launch.
 // Decoding: in each 64-wide block, lane (g, c) owns code bytes 8c..8c+7 of rows
 // g and g+8; MMA step st uses bytes 2st (k pair "2c") and 2st+1 (k pair
 // "2c+8"), and X is read with the same permutation of k, so every product still
@@ -48,6 +51,8 @@
 // host picks S per shape and device), so results do not depend on timing.
 // Remote shared-memory accesses are stores only and all land before the
 // epoch's cluster barrier.
+#include <type_traits>
+
 #include "qln_common.cuh"
 #include "qln_internal.h"
 #include "tc_ptx.cuh"
@@ -87,7 +92,7 @@ struct DvParams {
     uint16_t *sUg;       // [8 NT][r], rows t >= n zero
     int S, Q, nsub, nkb_max, UG;
     int epoch;                                       // rounds per epoch
-    int off_slots, off_red, off_su, off_bar;         // shared-memory layout (bytes)
+    int off_slots, off_su, off_bar;                  // shared-memory layout (bytes)
 };
 
 // ---- cluster and memory-model primitives -------------------------------------
@@ -139,7 +144,6 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
     uint8_t *tab = dsm;                                         // table rows; X lines in their second halves
     uint8_t *ring = dsm + kDvTabBytes;                          // [2][16 warps][16 rows][128 B], swizzled
     float *slots = reinterpret_cast<float *>(dsm + p.off_slots);  // pushed partials of one epoch
-    float *red = reinterpret_cast<float *>(dsm + p.off_red);    // U parts of the warps (U CTAs)
     uint16_t *sU = reinterpret_cast<uint16_t *>(dsm + p.off_su);  // [8 NT][r]
     const uint32_t bars = smem_u32(dsm + p.off_bar);            // [16 warps][2] mbarriers
     volatile int *flag = reinterpret_cast<volatile int *>(dsm + p.off_bar + 2 * kDvWarps * 8);
@@ -159,87 +163,16 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
     const bool dq = p.qabs != nullptr;
     int *ucount = reinterpret_cast<int *>(reinterpret_cast<char *>(p.status) + kWsUCountOffset);
     int *uflag = reinterpret_cast<int *>(reinterpret_cast<char *>(p.status) + kWsUFlagOffset);
+    int *udone = reinterpret_cast<int *>(reinterpret_cast<char *>(p.status) + kWsDoneOffset);
 
-    cluster_arrive_relaxed();  // "started": no peer writes here before every CTA of the cluster runs
-
-    // ---- 1. requests: two units of codes per warp, X chunk, constants, table ---
-    const uint32_t wbar = bars + (uint32_t)warp * 16u;  // stage st's barrier at + 8 st
-    if (lane == 0) {
-        tc::mbar_init(wbar, 1);
-        tc::mbar_init(wbar + 8, 1);
-        tc::mbar_fence_init();
-        tc::tma_prefetch_map(&tm_codes);
-    }
-    __syncwarp();
-    const uint32_t ring_s = smem_u32(ring) + (uint32_t)(warp * kDvStageBytes);  // stage st at + st * 16 stages
-    auto issue_codes = [&](int k, int st) {  // round k's unit of this warp -> stage st
-        const int64_t tl = t0 + (int64_t)(kDvWarps * k + warp) / nsub;
-        if (k < rounds && tl < t1 && lane == 0) {
-            tc::fence_proxy_async_smem();  // the stage's earlier reads come before the copy
-            tc::mbar_arrive_expect_tx(wbar + 8u * st, (uint32_t)kDvStageBytes);
-            tc::tma_load_2d(ring_s + (uint32_t)(st * kDvWarps * kDvStageBytes), &tm_codes,
-                            (int32_t)((kb0 + sb0) * 32), (int32_t)(tl * 16), wbar + 8u * st);
-        }
-    };
-    auto load_consts = [&](int k, DvConsts &o) {
-        const int64_t tl = t0 + (int64_t)(kDvWarps * k + warp) / nsub;
-        if (k < rounds && tl < t1) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int64_t jb0 = (tl * 16 + g + 8 * h) * KB + kb0 + sb0;
-                if (dq) {
-#pragma unroll
-                    for (int b = 0; b < kDvUnitKb; ++b)
-                        if (b < snb) o.raw[b][h] = (uint32_t)(int)__ldg(p.qabs + jb0 + b);
-                    o.sc[h][0] = __ldg(p.dq_scale + (jb0 >> 8));
-                    o.sc[h][1] = __ldg(p.dq_scale + ((jb0 + snb - 1) >> 8));
-                    o.lo[h] = (int)(jb0 & 255);
-                } else {
-#pragma unroll
-                    for (int b = 0; b < kDvUnitKb; ++b)
-                        if (b < snb) o.raw[b][h] = __float_as_uint(__ldg(p.absmax + jb0 + b));
-                }
-            }
-        }
-    };
-    issue_codes(0, 0);
-    issue_codes(1, 1);
-    // X chunk: line (token t, block bl) at row t * nkbx + bl, second half; 16-B chunks swizzled by t & 1
-    for (int i = tid; i < 8 * NT * nkbx * 8; i += kDvThreads) {
-        const int t = i / (nkbx * 8), j = i % (nkbx * 8);
-        uint8_t *dst = tab + (t * nkbx + (j >> 3)) * 256 + 128 + (((j & 7) ^ (t & 1)) << 4);
-        if (t < n && j < nkb * 8)
-            cp_async16(dst, p.X + (int64_t)t * cols + kb0 * 64 + j * 8);
-        else
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    cp_async_commit();
-    DvConsts kc;
-    load_consts(0, kc);
-    const float mu = dq ? __ldg(p.dq_mean) : 0.f;
-    {   // the adapter rows this cluster folds with, into L2 (split over the ranks)
-        const char *bb = reinterpret_cast<const char *>(p.B + t0 * 16 * r);
-        const int64_t lines = ((t1 - t0) * 16 * r * 2 + 127) / 128;
-        for (int64_t l = rank * kDvThreads + tid; l < lines; l += (int64_t)S * kDvThreads)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(bb + l * 128));
-    }
-    {   // table: warp w writes the rows e = 16 k + w, so c[e >> 4] = c[k] is a constant
-        float clo = 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-            if (q == warp) clo = nf4_value(q);
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-            *reinterpret_cast<uint32_t *>(tab + (16 * k + warp) * 256 + lane * 4) = pack_bf16x2(nf4_value(k), clo);
-    }
-
-    // ---- 2. U = X A^T, once for the grid -------------------------------------------
-    if ((int)blockIdx.x < p.UG) {
-        const int u = blockIdx.x;
+    // ---- U CTAs: U = X A^T, once for the grid ------------------------------------
+    if ((int)blockIdx.x >= p.Q * S) {
+        const int u = (int)blockIdx.x - p.Q * S;  // 0 .. UG-1; U clusters hold U CTAs only
         const int64_t ub0 = KB * u / p.UG, ub1 = KB * (u + 1) / p.UG;  // this CTA's K range of U
         const int njt = r / 8, nsubu = kDvWarps / njt;
         const int jt = warp % njt, subu = warp / njt;
         const int mtu = (n + 15) / 16;
+        float *red = reinterpret_cast<float *>(dsm);  // [nsubu][n][r]
         if (subu < nsubu) {
             const int64_t b0 = ub0 + (ub1 - ub0) * subu / nsubu, b1 = ub0 + (ub1 - ub0) * (subu + 1) / nsubu;
             float acc_u[2][4];
@@ -285,9 +218,10 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
         }
         __threadfence();
         __syncthreads();
-        if (tid == 0) *flag = atomicAdd(ucount, 1) == p.UG - 1;
+        volatile int *last = reinterpret_cast<volatile int *>(dsm + kDvRedBytes);
+        if (tid == 0) *last = atomicAdd(ucount, 1) == p.UG - 1;
         __syncthreads();
-        if (*flag) {  // every part is published: fold them in order
+        if (*last) {  // every part is published: fold them in order
             __threadfence();
             for (int i = tid; i < 8 * NT * r; i += kDvThreads) {
                 const int t = i / r;
@@ -301,7 +235,83 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
             __syncthreads();
             if (tid == 0) st_release_gpu(uflag, 1);
         }
+        return;
     }
+
+    if (blockIdx.x == 0 && tid == 0) *p.status = QLN_OK;
+    cluster_arrive_relaxed();  // "started": no peer writes here before every CTA of the cluster runs
+
+    // ---- 1. requests: two units of codes per warp, X chunk, constants, table ---
+    const uint32_t wbar = bars + (uint32_t)warp * 16u;  // stage st's barrier at + 8 st
+    if (lane == 0) {
+        tc::mbar_init(wbar, 1);
+        tc::mbar_init(wbar + 8, 1);
+        tc::mbar_fence_init();
+        tc::tma_prefetch_map(&tm_codes);
+    }
+    __syncwarp();
+    const uint32_t ring_s = smem_u32(ring) + (uint32_t)(warp * kDvStageBytes);  // stage st at + st * 16 stages
+    auto issue_codes = [&](int k, int st) {  // round k's unit of this warp -> stage st
+        const int64_t tl = t0 + (int64_t)(kDvWarps * k + warp) / nsub;
+        if (k < rounds && tl < t1 && lane == 0) {
+            tc::fence_proxy_async_smem();  // the stage's earlier reads come before the copy
+            tc::mbar_arrive_expect_tx(wbar + 8u * st, (uint32_t)kDvStageBytes);
+            tc::tma_load_2d(ring_s + (uint32_t)(st * kDvWarps * kDvStageBytes), &tm_codes,
+                            (int32_t)((kb0 + sb0) * 32), (int32_t)(tl * 16), wbar + 8u * st);
+        }
+    };
+    auto load_consts = [&](int k, DvConsts &o) {
+        const int64_t tl = t0 + (int64_t)(kDvWarps * k + warp) / nsub;
+        if (k < rounds && tl < t1) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int64_t jb0 = (tl * 16 + g + 8 * h) * KB + kb0 + sb0;
+                if (dq) {
+#pragma unroll
+                    for (int b = 0; b < kDvUnitKb; ++b)
+                        if (b < snb) o.raw[b][h] = (uint32_t)(int)__ldg(p.qabs + jb0 + b);
+                    o.sc[h][0] = __ldg(p.dq_scale + (jb0 >> 8));
+                    o.sc[h][1] = __ldg(p.dq_scale + ((jb0 + snb - 1) >> 8));
+                    o.lo[h] = (int)(jb0 & 255);
+                } else {
+#pragma unroll
+                    for (int b = 0; b < kDvUnitKb; ++b)
+                        if (b < snb) o.raw[b][h] = __float_as_uint(__ldg(p.absmax + jb0 + b));
+                }
+            }
+        }
+    };
+    issue_codes(0, 0);
+    issue_codes(1, 1);
+    // X chunk: line (token t, block bl) at row t * nkbx + bl, second half; 16-B chunks swizzled by t & 1
+    for (int t = warp; t < 8 * NT; t += kDvWarps)
+        for (int j = lane; j < nkbx * 8; j += 32) {
+            uint8_t *dst = tab + (t * nkbx + (j >> 3)) * 256 + 128 + (((j & 7) ^ (t & 1)) << 4);
+            if (t < n && j < nkb * 8)
+                cp_async16(dst, p.X + (int64_t)t * cols + kb0 * 64 + j * 8);
+            else
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
+    cp_async_commit();
+    DvConsts kc;
+    load_consts(0, kc);
+    const float mu = dq ? __ldg(p.dq_mean) : 0.f;
+    {   // the adapter rows this cluster folds with, into L2 (split over the ranks)
+        const char *bb = reinterpret_cast<const char *>(p.B + t0 * 16 * r);
+        const int64_t lines = ((t1 - t0) * 16 * r * 2 + 127) / 128;
+        for (int64_t l = rank * kDvThreads + tid; l < lines; l += (int64_t)S * kDvThreads)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(bb + l * 128));
+    }
+    {   // table: warp w writes the rows e = 16 k + w, so c[e >> 4] = c[k] is a constant
+        float clo = 0.f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            if (q == warp) clo = nf4_value(q);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            *reinterpret_cast<uint32_t *>(tab + (16 * k + warp) * 256 + lane * 4) = pack_bf16x2(nf4_value(k), clo);
+    }
+
     cp_async_wait<0>();  // X
     __syncthreads();
     cluster_wait();      // every CTA of the cluster has started
@@ -314,6 +324,16 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
     for (int nt = 0; nt < NT; ++nt) {
         const int t = 8 * nt + g;
         xoff[nt] = (uint32_t)((t * nkbx + sb0) * 256 + 128 + (((2 * c) ^ (t & 1)) << 4));
+    }
+    // n <= 8: the warp's X fragments for its whole K sub-range stay in registers
+    // (the sub-range is the same in every round)
+    uint4 xr[kDvUnitKb][2];
+    if constexpr (NT == 1) {
+#pragma unroll
+        for (int b = 0; b < kDvUnitKb; ++b)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                xr[b][hh] = b < snb ? lds128(tab + ((xoff[0] + b * 256) ^ (uint32_t)(hh << 4))) : make_uint4(0u, 0u, 0u, 0u);
     }
     int e0 = 0;  // first round of the current epoch
     for (int k = 0; k < rounds; ++k) {
@@ -329,55 +349,68 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
             if (!tc::mbar_wait_bounded(wbar + 8u * (k & 1), (uint32_t)((k >> 1) & 1), nullptr, kDvWaitNs))
                 atomicExch(p.status, (int)QLN_ERR_TIMEOUT);
             const uint8_t *cs = ring + (k & 1) * (kDvWarps * kDvStageBytes) + warp * kDvStageBytes + g * 128 + (c & 1) * 8;
+            auto unit = [&](auto full_tag) {
+                constexpr bool kFull = decltype(full_tag)::value;
 #pragma unroll
-            for (int b = 0; b < kDvUnitKb; ++b) {
-                if (b < snb) {
-                    const int ch = ((2 * b + (c >> 1)) ^ g) << 4;  // 16-B chunk of block b, swizzled by row & 7
-                    uint2 cw[2];
-                    cw[0] = *reinterpret_cast<const uint2 *>(cs + ch);
-                    cw[1] = *reinterpret_cast<const uint2 *>(cs + 8 * 128 + ch);
-                    float ah[2];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        ah[h] = dq ? dq_restore((int8_t)kc.raw[b][h], (kc.lo[h] + b >= 256) ? kc.sc[h][1] : kc.sc[h][0], mu)
-                                   : __uint_as_float(kc.raw[b][h]);
-                    float tmp[NT][4];
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint4 xv[NT];
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) xv[nt] = lds128(tab + ((xoff[nt] + b * 256) ^ (uint32_t)(hh << 4)));
-#pragma unroll
-                        for (int sp = 0; sp < 2; ++sp) {
-                            const int st = 2 * hh + sp;
-                            uint32_t a[4];
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {  // (row g, 2c) (row g+8, 2c) (row g, 2c+8) (row g+8, 2c+8)
-                                const int h = q & 1, bi = 2 * st + (q >> 1);  // byte of the lane's share
-                                const uint32_t word = (bi < 4) ? cw[h].x : cw[h].y;
-                                // table row of the code byte, this lane's column: byte * 256 + lane * 4
-                                const uint32_t off = prmt(word, lane4, 0x5504u | ((uint32_t)(bi & 3) << 4));
-                                a[q] = *reinterpret_cast<const uint32_t *>(tab + off);
-                            }
-#pragma unroll
+                for (int b = 0; b < kDvUnitKb; ++b) {
+                    if (kFull || b < snb) {
+                        const int ch = ((2 * b + (c >> 1)) ^ g) << 4;  // 16-B chunk of block b, swizzled by row & 7
+                        uint2 cw[2];
+                        cw[0] = *reinterpret_cast<const uint2 *>(cs + ch);
+                        cw[1] = *reinterpret_cast<const uint2 *>(cs + 8 * 128 + ch);
+                        float ah[2];
+    #pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            ah[h] = dq ? dq_restore((int8_t)kc.raw[b][h], (kc.lo[h] + b >= 256) ? kc.sc[h][1] : kc.sc[h][0], mu)
+                                       : __uint_as_float(kc.raw[b][h]);
+                        float tmp[NT][4];
+    #pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            uint4 xv[NT];
+    #pragma unroll
                             for (int nt = 0; nt < NT; ++nt) {
-                                const uint32_t bb[2] = {sp ? xv[nt].z : xv[nt].x, sp ? xv[nt].w : xv[nt].y};
-                                if (st == 0)
-                                    mma_bf16_16816_zero(tmp[nt], a, bb);
+                                if constexpr (NT == 1)
+                                    xv[nt] = xr[b][hh];
                                 else
-                                    mma_bf16_16816(tmp[nt], a, bb);
+                                    xv[nt] = lds128(tab + ((xoff[nt] + b * 256) ^ (uint32_t)(hh << 4)));
+                            }
+    #pragma unroll
+                            for (int sp = 0; sp < 2; ++sp) {
+                                const int st = 2 * hh + sp;
+                                uint32_t a[4];
+    #pragma unroll
+                                for (int q = 0; q < 4; ++q) {  // (row g, 2c) (row g+8, 2c) (row g, 2c+8) (row g+8, 2c+8)
+                                    const int h = q & 1, bi = 2 * st + (q >> 1);  // byte of the lane's share
+                                    const uint32_t word = (bi < 4) ? cw[h].x : cw[h].y;
+                                    // table row of the code byte, this lane's column: byte * 256 + lane * 4
+                                    const uint32_t off = prmt(word, lane4, 0x5504u | ((uint32_t)(bi & 3) << 4));
+                                    a[q] = *reinterpret_cast<const uint32_t *>(tab + off);
+                                }
+    #pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    const uint32_t bb[2] = {sp ? xv[nt].z : xv[nt].x, sp ? xv[nt].w : xv[nt].y};
+                                    if (st == 0)
+                                        mma_bf16_16816_zero(tmp[nt], a, bb);
+                                    else
+                                        mma_bf16_16816(tmp[nt], a, bb);
+                                }
                             }
                         }
-                    }
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        acc[nt][0] = __fmaf_rn(ah[0], tmp[nt][0], acc[nt][0]);
-                        acc[nt][1] = __fmaf_rn(ah[0], tmp[nt][1], acc[nt][1]);
-                        acc[nt][2] = __fmaf_rn(ah[1], tmp[nt][2], acc[nt][2]);
-                        acc[nt][3] = __fmaf_rn(ah[1], tmp[nt][3], acc[nt][3]);
+    #pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            acc[nt][0] = __fmaf_rn(ah[0], tmp[nt][0], acc[nt][0]);
+                            acc[nt][1] = __fmaf_rn(ah[0], tmp[nt][1], acc[nt][1]);
+                            acc[nt][2] = __fmaf_rn(ah[1], tmp[nt][2], acc[nt][2]);
+                            acc[nt][3] = __fmaf_rn(ah[1], tmp[nt][3], acc[nt][3]);
+                        }
                     }
                 }
-            }
+    
+            };
+            if (snb == kDvUnitKb)
+                unit(std::true_type{});
+            else
+                unit(std::false_type{});
         }
         __syncwarp();  // every lane is done with this stage
         issue_codes(k + 2, k & 1);
@@ -400,9 +433,7 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
         const int64_t et0 = t0 + (int64_t)kDvWarps * e0 / nsub;
         const int64_t et1e = t0 + (int64_t)kDvWarps * (k + 1) / nsub;
         const int m = (int)((et1e < t1 ? et1e : t1) - et0);
-        cluster_arrive();
-        cluster_wait();  // every partial of the epoch has landed here
-        if (e0 == 0) {   // bf16(s U), once the U CTAs have folded it
+        if (e0 == 0) {   // bf16(s U), once the U CTAs have folded it (long done by now, as a rule)
             if (tid == 0) {
                 bool ok = ld_acquire_gpu(uflag) != 0;
                 if (!ok) {
@@ -419,20 +450,29 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
             const bool ok = *flag != 0;
             for (int i = tid; i < 8 * NT * r / 2; i += kDvThreads)
                 reinterpret_cast<uint32_t *>(sU)[i] = ok ? __ldcg(reinterpret_cast<const unsigned int *>(p.sUg) + i) : 0u;
-            __syncthreads();
+            if (tid == 0 && atomicAdd(udone, 1) == p.Q * S - 1) {
+                // every decode CTA has read bf16(s U): leave the counters at zero for the next call
+                *ucount = 0;
+                *uflag = 0;
+                *udone = 0;
+            }
         }
+        // B fragments of this warp's first tile of the epoch, requested before the barrier
+        const int i0 = warp * S + rank;
+        uint32_t ba[2][4];
+#pragma unroll
+        for (int js = 0; js < 2; ++js)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int64_t row = (et0 + (i0 < m ? i0 : 0)) * 16 + g + 8 * (q & 1);
+                const int j = 16 * js + 2 * c + 8 * (q >> 1);
+                ba[js][q] = (i0 < m && j < r) ? __ldg(reinterpret_cast<const uint32_t *>(p.B + row * r + j)) : 0u;
+            }
+        cluster_arrive();
+        cluster_wait();  // every partial of the epoch has landed here (and sU is in place)
         for (int i = warp * S + rank; i < m; i += kDvWarps * S) {
             const int64_t row0 = (et0 + i) * 16;
             const int li = i / S;
-            uint32_t ba[2][4];  // B fragments of the first two 16-column steps, requested up front
-#pragma unroll
-            for (int js = 0; js < 2; ++js)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int64_t row = row0 + g + 8 * (q & 1);
-                    const int j = 16 * js + 2 * c + 8 * (q >> 1);
-                    ba[js][q] = (j < r) ? __ldg(reinterpret_cast<const uint32_t *>(p.B + row * r + j)) : 0u;
-                }
             float f[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -452,7 +492,7 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
             }
             for (int j0 = 0; j0 < r; j0 += 16) {
                 uint32_t a[4];
-                if (j0 < 32) {
+                if (i == i0 && j0 < 32) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) a[q] = j0 == 0 ? ba[0][q] : ba[1][q];
                 } else {
@@ -492,7 +532,7 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
 // Shared-memory layout and split of one launch.
 struct DvLayout {
     int S, nsub, NT, nkb_max, epoch;
-    int off_slots, off_red, off_su, off_bar;
+    int off_slots, off_su, off_bar;
     size_t smem;
     bool ok;
 };
@@ -509,7 +549,7 @@ static DvLayout dv_layout(int64_t KB, int64_t n, int r, int S) {
     const int64_t xbytes = (int64_t)8 * L.NT * L.nkb_max * 128;
     L.ok = false;
     L.epoch = 0;
-    L.off_slots = L.off_red = L.off_su = L.off_bar = 0;
+    L.off_slots = L.off_su = L.off_bar = 0;
     L.smem = 0;
     if (S > KB || xbytes > kDvXMax || L.nsub > kDvWarps) return L;  // (a round must hold whole tiles)
     // an owner parks, per tile it folds, S x nsub partials; with tile i of an epoch
@@ -517,14 +557,13 @@ static DvLayout dv_layout(int64_t KB, int64_t n, int r, int S) {
     // hold (epoch * tiles per round + S - 1) tiles' worth of partials
     const int64_t per_tile = (int64_t)L.nsub * L.NT * 512;
     const int64_t tpr = kDvWarps / L.nsub;
-    const int64_t fixed = (int64_t)kDvTabBytes + kDvRingBytes + kDvRedBytes + kDvSUBytes + kDvBarBytes;
+    const int64_t fixed = (int64_t)kDvTabBytes + kDvRingBytes + kDvSUBytes + kDvBarBytes;
     const int64_t room = (int64_t)kDvSmemMax - fixed - (S - 1) * per_tile;
     int64_t ep = room > 0 ? room / (tpr * per_tile) : 0;
     if (ep > 16) ep = 16;
     L.epoch = (int)ep;
     L.off_slots = kDvTabBytes + kDvRingBytes;
-    L.off_red = L.off_slots + dv_a128((ep * tpr + S - 1) * per_tile);
-    L.off_su = L.off_red + kDvRedBytes;
+    L.off_su = L.off_slots + dv_a128((ep * tpr + S - 1) * per_tile);
     L.off_bar = L.off_su + kDvSUBytes;
     L.smem = (size_t)L.off_bar + kDvBarBytes;
     L.ok = S <= KB && xbytes <= kDvXMax && L.nsub <= kDvWarps && ep >= 1 && L.smem <= kDvSmemMax &&
@@ -589,8 +628,11 @@ static cudaError_t launch_dv(DvParams p, const qln_nf4_weight *w, cudaStream_t s
         int nclus = 0;
         cudaError_t e = dv_max_clusters<NT>(S, &nclus);
         if (e != cudaSuccess) return e;
-        int64_t Q = nclus < T ? nclus : T;
-        if (Q * S > kDvPlanSms) Q = kDvPlanSms / S;
+        // the decode clusters leave room for the 8 / S clusters of U CTAs
+        int64_t Q = nclus - kDvUParts / S;
+        if (Q > T) Q = T;
+        if ((Q + kDvUParts / S) * S > kDvPlanSms) Q = kDvPlanSms / S - kDvUParts / S;
+        if (Q < 1) continue;
         if (Q * S > best) {
             best = Q * S;
             best_L = L;
@@ -610,10 +652,8 @@ static cudaError_t launch_dv(DvParams p, const qln_nf4_weight *w, cudaStream_t s
     p.nsub = L.nsub;
     p.nkb_max = L.nkb_max;
     p.epoch = L.epoch;
-    p.UG = (int)(KB < kDvUParts ? KB : kDvUParts);
-    if (p.UG > bestQ * L.S) p.UG = (int)(bestQ * L.S);
+    p.UG = kDvUParts;
     p.off_slots = L.off_slots;
-    p.off_red = L.off_red;
     p.off_su = L.off_su;
     p.off_bar = L.off_bar;
     cudaLaunchConfig_t cfg = {};
@@ -622,7 +662,7 @@ static cudaError_t launch_dv(DvParams p, const qln_nf4_weight *w, cudaStream_t s
     attr[0].val.clusterDim.x = (unsigned)L.S;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3((unsigned)(bestQ * L.S));
+    cfg.gridDim = dim3((unsigned)((bestQ + kDvUParts / L.S) * L.S));
     cfg.blockDim = dim3(kDvThreads);
     cfg.dynamicSmemBytes = L.smem;
     cfg.stream = st;
@@ -656,9 +696,6 @@ cudaError_t launch_nf4_gemv(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     p.status = reinterpret_cast<int *>(wsb);
     p.upart = reinterpret_cast<float *>(wsb + kWsHeaderBytes);
     p.sUg = reinterpret_cast<uint16_t *>(wsb + kWsHeaderBytes + dv_a128((int64_t)kDvUParts * n * r * 4));
-    // status word, U counter and ready flag start at zero
-    cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeaderBytes, st);
-    if (e != cudaSuccess) return e;
     switch ((n + 7) / 8) {
         case 1: return launch_dv<1>(p, w, st);
         case 2: return launch_dv<2>(p, w, st);

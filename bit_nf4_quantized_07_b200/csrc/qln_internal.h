@@ -50,12 +50,13 @@ cudaError_t launch_nf4_mma_gemm(const qln_nf4_weight *w, bool trans, const uint1
 bool make_tensor_map_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t inner,
                         uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
 
-// Workspace header of the linear calls: the int32 status word at byte 0 and,
-// for the decode-sized forward, an arrival counter and a ready flag; each call
-// zeroes the header before its kernels run.
+// Workspace header of the linear calls: the int32 status word at byte 0 and
+// three counters of the decode-sized forward.  The counters must be zero when a
+// workspace is first used; every launch that uses them leaves them at zero.
 constexpr int kWsHeaderBytes = 256;
 constexpr int kWsUCountOffset = 64;   // int32: CTAs that have published their part of U
 constexpr int kWsUFlagOffset = 128;   // int32: 1 once bf16(s U) of the call is in the workspace
+constexpr int kWsDoneOffset = 192;    // int32: CTAs that have read bf16(s U)
 // SM count the decode-sized forward sizes its workspace for (B200); its grid
 // never exceeds it.
 constexpr int kDvPlanSms = 148;

@@ -45,6 +45,10 @@
  *   give up after a bounded number of polls and write QLN_ERR_TIMEOUT into the
  *   int32 status word at byte offset 0 of the workspace; read it after the
  *   stream has synchronised (0 = QLN_OK).  Each workspace call clears it.
+ * - Bytes 4..255 of a workspace hold counters of the decode-sized forward
+ *   (n <= 32).  Zero-fill a workspace once before its first use; every call
+ *   leaves the counters at zero again (also across CUDA graph replays).  After
+ *   a call that reported QLN_ERR_TIMEOUT, zero the first 256 bytes again.
  */
 #ifndef QLORA_NF4_H
 #define QLORA_NF4_H
