@@ -50,15 +50,18 @@ __device__ void build_snap_lut(uint2 *lut) {
     }
 }
 
-// Codes of the 4 weights of v (block absmax a > 0, inv = RN(1/a)), packed as
-// two bytes, first weight in the high nibble of the first byte.  The product
-// y = RN(w * inv) is within 2 ulp of w/a, and x = RN(w/a) within half an ulp,
-// so y and x fall on the same side of a threshold t unless |y - t| < 3 ulp(t)
-// <= 2^-21 (|t| < 1).  Only then is the exact quotient formed (IEEE
-// division) and used instead: the code is always that of x.  The test looks
-// only at the threshold of y's own key interval; that is enough because every
-// threshold lies more than 15,000 ulps inside its key interval, so no
-// threshold of a neighbouring interval is within 3 ulps of y.
+// Codes of the 4 weights of v (block absmax a > 0, inv = the hardware
+// reciprocal of a, relative error <= 2^-23), packed as two bytes, first weight
+// in the high nibble of the first byte.  The product y = RN(w * inv) differs
+// from the real quotient w/a by at most |w/a| (2^-23 + 2^-24) < 1.8e-7, and
+// x = RN(w/a) is within 2^-25 of it, so y and x fall on the same side of a
+// threshold t unless |y - t| < 2.2e-7 < 2^-21.  Only then is the exact quotient
+// formed (IEEE division) and used instead: the code is always that of x.  The
+// test looks only at the threshold of y's own key interval; that is enough
+// because every threshold lies more than 15,000 ulps inside its key interval,
+// so no threshold of a neighbouring interval is that close to y.  When a or
+// 1/a is subnormal (a < 2^-126 or a >= 2^126) the bound does not hold and the
+// group takes the exact path outright.
 __device__ __forceinline__ uint32_t snap4(float4 v, float a, float inv, const uint2 *lut) {
     const float w[4] = {v.x, v.y, v.z, v.w};
     uint32_t q[4];
@@ -71,7 +74,7 @@ __device__ __forceinline__ uint32_t snap4(float4 v, float a, float inv, const ui
         q[i] = e.y + (d > 0.f ? 1u : 0u);
         near |= fabsf(d) < 4.76837158203125e-07f;  // 2^-21
     }
-    if (near) {  // rare: redo the whole group exactly
+    if (near || !(a >= 0x1p-126f && a < 0x1p126f)) {  // rare: redo the group exactly (also for a or 1/a subnormal)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const float x = __fdiv_rn(w[i], a);
@@ -110,19 +113,15 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float4 *__restr
             v[u][0] = (c < nchunks && b0 < nb) ? __ldcs(src) : make_float4(0.f, 0.f, 0.f, 0.f);
             v[u][1] = (c < nchunks && b0 + 2 < nb) ? __ldcs(src + 32) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        // block absmax: |w| >= 0, so the bit patterns order like the values and a
+        // 16-lane integer max reduction (one per half-warp, each with its own mask) is exact
+        const unsigned half_mask = (lane < 16) ? 0x0000ffffu : 0xffff0000u;
         float m[2][2];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            m[u][0] = absmax4(v[u][0]);
-            m[u][1] = absmax4(v[u][1]);
-        }
+        for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int off = 8; off >= 1; off >>= 1)
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                m[u][0] = fmaxf(m[u][0], __shfl_xor_sync(0xffffffffu, m[u][0], off));
-                m[u][1] = fmaxf(m[u][1], __shfl_xor_sync(0xffffffffu, m[u][1], off));
-            }
+            for (int h = 0; h < 2; ++h)
+                m[u][h] = __uint_as_float(__reduce_max_sync(half_mask, __float_as_uint(absmax4(v[u][h]))));
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int64_t c = c0 + u * nwarps;
@@ -132,7 +131,8 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float4 *__restr
                 const int64_t b = 4 * c + (lane >> 4) + 2 * h;  // block of v[u][h]
                 if (b < nb) {
                     const float a = m[u][h];
-                    const float inv = a > 0.f ? __frcp_rn(a) : 0.f;
+                    float inv = 0.f;
+                    if (a > 0.f) asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(a));
                     __stcs(codes16 + 64 * c + 32 * h + lane, (uint16_t)snap4(v[u][h], a, inv, lut));
                     if ((lane & 15) == 0) absmax[b] = a;
                 }
@@ -395,50 +395,67 @@ cudaError_t launch_nf4_double_quant_static(const float *absmax, int64_t nb, int8
 }
 
 // ===========================================================================
-// K4: doubleDequant to BF16.  A warp streams 32 code words (256 weights, 4
-// blocks): lane l decodes word l (8 weights) and stores 16 bytes, so every
-// load and store instruction is fully coalesced.  A 256-entry shared table
-// maps a code byte to the book values of its two codes (c[hi], c[lo]); the
-// products with the restored constant are fp32 multiplies rounded once to
-// BF16, spreading the work over the load/store, FMA and integer pipes.
-// w' = bf16_RN(fp32(ahat * c[q])).
+// K4: doubleDequant to BF16.  A thread takes 32 consecutive weights at a time
+// (16 bytes of codes, half of one 64-weight block) and writes 64 bytes of
+// BF16; the next group's code bytes and constants are requested before the
+// current group is decoded, so about 32 bytes per thread are in flight.  The
+// decode is register-only: the 16 products bf16_RN(fp32(ahat * c[q])) of the
+// block are built once and split into byte tables, and a byte permute looks up
+// four codes at a time -- exactly w' = bf16_RN(fp32(ahat * c[q])), with no
+// shared-memory traffic.
 // ===========================================================================
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t *__restrict__ codes32,
+struct DeqIn {
+    uint4 cw;   // 32 codes
+    int8_t q;   // DQ code of the block (or unused)
+    float v;    // DQ scale of the block's group, or the plain absmax
+};
+
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4 *__restrict__ codes128,
                                                           const float *__restrict__ absmax,
                                                           const int8_t *__restrict__ qabs,
                                                           const float *__restrict__ scale,
-                                                          const float *__restrict__ mu_p, int64_t nwords,
+                                                          const float *__restrict__ mu_p, int64_t ngroups,
                                                           uint4 *__restrict__ out) {
-    __shared__ float2 pair_tab[256];
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) pair_tab[i] = make_float2(nf4_value(i >> 4), nf4_value(i & 15));
-    __syncthreads();
     const float mu = qabs ? __ldg(mu_p) : 0.f;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nwords; i += stride) {
-        const int64_t j = i >> 3;  // 8 words (64 codes) per block
-        float ah;
-        if (qabs) ah = dq_restore(__ldg(qabs + j), __ldg(scale + (j >> 8)), mu);
-        else ah = __ldg(absmax + j);
-        const uint32_t cw = __ldcs(codes32 + i);
-        uint32_t o[4];
-#pragma unroll
-        for (int bi = 0; bi < 4; ++bi) {
-            const float2 cc = pair_tab[(cw >> (8 * bi)) & 0xffu];
-            o[bi] = pack_bf16x2(__fmul_rn(ah, cc.x), __fmul_rn(ah, cc.y));
+    auto fetch = [&](int64_t i, DeqIn &d) {
+        if (i < ngroups) {
+            const int64_t j = i >> 1;  // two 32-weight groups per block
+            d.cw = __ldcs(codes128 + i);
+            if (qabs) {
+                d.q = __ldg(qabs + j);
+                d.v = __ldg(scale + (j >> 8));
+            } else {
+                d.q = 0;
+                d.v = __ldg(absmax + j);
+            }
         }
-        __stcs(out + i, make_uint4(o[0], o[1], o[2], o[3]));
+    };
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    DeqIn cur, nxt;
+    fetch(i, cur);
+    for (; i < ngroups; i += stride) {
+        fetch(i + stride, nxt);
+        const float ah = qabs ? dq_restore(cur.q, cur.v, mu) : cur.v;
+        const NF4Table t = nf4_table(ah);
+        uint4 *o = out + 4 * i;
+        __stcs(o + 0, nf4_decode8(cur.cw.x, t));
+        __stcs(o + 1, nf4_decode8(cur.cw.y, t));
+        __stcs(o + 2, nf4_decode8(cur.cw.z, t));
+        __stcs(o + 3, nf4_decode8(cur.cw.w, t));
+        cur = nxt;
     }
 }
 
 cudaError_t launch_nf4_dequant(const qln_nf4_weight *w, uint16_t *out, cudaStream_t st, int num_sms) {
     const int64_t numel = w->rows * w->cols;
-    const int64_t nwords = numel / 8;
-    int64_t grid = (nwords + 255) / 256;
+    const int64_t ngroups = numel / 32;
+    int64_t grid = (ngroups + 255) / 256;
     const int64_t cap = (int64_t)num_sms * 8;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
-    nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint32_t *>(w->codes), w->absmax,
-                                                      w->qabs, w->dq_scale, w->dq_mean, nwords,
+    nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(w->codes), w->absmax, w->qabs,
+                                                      w->dq_scale, w->dq_mean, ngroups,
                                                       reinterpret_cast<uint4 *>(out));
     note_launch();
     return cudaGetLastError();
