@@ -49,15 +49,15 @@ constexpr int kSplitTargetSms = 148;
 //   fwd: sU [n][r] bf16, U [n][r] bf16 (used when U_out is NULL),
 //        split-K partials of U (fp32) -- or, for decode-sized n, the parts of
 //        U and bf16(s U) of the one-launch forward
-//   bwd: Bt [r][dout] bf16, G [n][r] bf16, sG [n][r] bf16, U [n][r] bf16,
-//        split-K partials of G / U (fp32, reused), dA partials, dB partials
+//   bwd: G [n][r] bf16, sG [n][r] bf16, U [n][r] bf16, split-K partials of
+//        G / U (fp32, reused), dA partials, dB partials
 // Split counts are planned for a fixed SM count so that the workspace size
 // does not depend on the device queried.
 struct FwdWs {
     size_t sU, U, pU, total;
 };
 struct BwdWs {
-    size_t Bt, G, sG, U, pGU, pA, pB, total;
+    size_t G, sG, U, pGU, pA, pB, total;
     int splitA, splitB;
 };
 
@@ -77,18 +77,17 @@ FwdWs fwd_layout(int64_t rows, int64_t cols, int64_t n, int r) {
 BwdWs bwd_layout(int64_t rows, int64_t cols, int64_t n, int r) {
     BwdWs L;
     const size_t nr = round256((size_t)n * r * 2);
-    L.Bt = qln::kWsHeaderBytes;
-    L.G = L.Bt + round256((size_t)rows * r * 2);
+    L.G = qln::kWsHeaderBytes;
     L.sG = L.G + nr;
     L.U = L.sG + nr;
     L.pGU = L.U + nr;
     const size_t pg = qln::lora_down_partial_bytes(n, rows, r, kSplitTargetSms);
     const size_t pu = qln::lora_down_partial_bytes(n, cols, r, kSplitTargetSms);
-    L.splitA = qln::tn_reduce_splits(n, r, cols, kSplitTargetSms);
-    L.splitB = qln::tn_reduce_splits(n, rows, r, kSplitTargetSms);
+    L.splitA = qln::tn_skinny_splits(n, cols, kSplitTargetSms);
+    L.splitB = qln::tn_skinny_splits(n, rows, kSplitTargetSms);
     L.pA = L.pGU + round256(pg > pu ? pg : pu);
-    L.pB = L.pA + round256(qln::tn_reduce_partials_bytes(r, cols, L.splitA));
-    L.total = L.pB + round256(qln::tn_reduce_partials_bytes(rows, r, L.splitB));
+    L.pB = L.pA + round256(qln::tn_skinny_partials_bytes(cols, r, L.splitA));
+    L.total = L.pB + round256(qln::tn_skinny_partials_bytes(rows, r, L.splitB));
     return L;
 }
 
@@ -119,17 +118,6 @@ qln_status check_linear(const qln_nf4_weight *w, const uint16_t *X, int64_t n, c
 }
 
 qln_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QLN_OK : QLN_ERR_CUDA; }
-
-// B [rows][r] -> Bt [r][rows]
-__global__ void transpose_bf16_kernel(const uint16_t *__restrict__ B, int64_t rows, int r, uint16_t *__restrict__ Bt) {
-    const int64_t total = rows * r;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
-        const int64_t o = i / r;
-        const int j = (int)(i % r);
-        Bt[(int64_t)j * rows + o] = B[i];
-    }
-}
 
 // The fused weight GEMM: tcgen05 where the shape fills its tiles, otherwise
 // the register-level path.
@@ -217,7 +205,7 @@ qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     // U = X A^T (and s*U for the adapter MMA), then the fused weight GEMM.
-    e = qln::launch_lora_down(X, n, w->cols, A, r, s, U, sU, pU, cs, kSplitTargetSms);
+    e = qln::launch_lora_down(X, n, w->cols, A, false, r, s, U, sU, pU, cs, kSplitTargetSms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     e = fused_gemm(w, false, X, n, sU, B, r, Y, status, cs, sms);
     return from_cuda(e);
@@ -240,7 +228,6 @@ qln_status qlora_linear_bwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     cudaStream_t cs = (cudaStream_t)stream;
     char *wsb = reinterpret_cast<char *>(ws);
     int *status = reinterpret_cast<int *>(wsb);
-    uint16_t *Bt = reinterpret_cast<uint16_t *>(wsb + L.Bt);
     uint16_t *G = reinterpret_cast<uint16_t *>(wsb + L.G);
     uint16_t *sG = reinterpret_cast<uint16_t *>(wsb + L.sG);
     float *pGU = reinterpret_cast<float *>(wsb + L.pGU);
@@ -250,26 +237,19 @@ qln_status qlora_linear_bwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     if (!U) {
         uint16_t *Uw = reinterpret_cast<uint16_t *>(wsb + L.U);
-        e = qln::launch_lora_down(X, n, w->cols, A, r, s, Uw, nullptr, pGU, cs, kSplitTargetSms);
+        e = qln::launch_lora_down(X, n, w->cols, A, false, r, s, Uw, nullptr, pGU, cs, kSplitTargetSms);
         if (e != cudaSuccess) return QLN_ERR_CUDA;
         U = Uw;
     }
-    {
-        const int64_t total = w->rows * r;
-        int64_t blocks = (total + 255) / 256;
-        if (blocks > 4096) blocks = 4096;
-        transpose_bf16_kernel<<<(unsigned)blocks, 256, 0, cs>>>(B, w->rows, r, Bt);
-        note_launch();
-        if (cudaGetLastError() != cudaSuccess) return QLN_ERR_CUDA;
-    }
-    // G = dY B (and s*G), dX = dY W' + (s G) A, dA = s G^T X, dB = s dY^T U.
-    e = qln::launch_lora_down(dY, n, w->rows, Bt, r, s, G, sG, pGU, cs, kSplitTargetSms);
+    // G = dY B (and s*G; B read as stored, [dout][r]), dX = dY W' + (s G) A,
+    // dA = s G^T X (the transpose of s X^T G), dB = s dY^T U.
+    e = qln::launch_lora_down(dY, n, w->rows, B, true, r, s, G, sG, pGU, cs, kSplitTargetSms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     e = fused_gemm(w, true, dY, n, sG, A, r, dX, status, cs, sms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
-    e = qln::launch_tn_reduce(G, X, n, r, w->cols, s, dA, pA, L.splitA, cs);
+    e = qln::launch_tn_skinny(X, G, n, w->cols, r, s, true, dA, pA, L.splitA, cs);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
-    e = qln::launch_tn_reduce(dY, U, n, w->rows, r, s, dB, pB, L.splitB, cs);
+    e = qln::launch_tn_skinny(dY, U, n, w->rows, r, s, false, dB, pB, L.splitB, cs);
     return from_cuda(e);
 }
 

@@ -395,14 +395,16 @@ cudaError_t launch_nf4_double_quant_static(const float *absmax, int64_t nb, int8
 }
 
 // ===========================================================================
-// K4: doubleDequant to BF16.  A thread takes 32 consecutive weights at a time
-// (16 bytes of codes, half of one 64-weight block) and writes 64 bytes of
-// BF16; the next group's code bytes and constants are requested before the
-// current group is decoded, so about 32 bytes per thread are in flight.  The
-// decode is register-only: the 16 products bf16_RN(fp32(ahat * c[q])) of the
-// block are built once and split into byte tables, and a byte permute looks up
-// four codes at a time -- exactly w' = bf16_RN(fp32(ahat * c[q])), with no
-// shared-memory traffic.
+// K4: doubleDequant to BF16.  A warp takes 1024 consecutive weights at a time
+// (512 bytes of codes, 16 blocks): lane l loads 16 bytes, 32 weights of block
+// l/2.  The code bytes and constants of the warp's next two chunks are
+// requested before the current one is decoded.  The decode is register-only:
+// the 16 products bf16_RN(fp32(ahat * c[q])) of the block are built once and
+// split into byte tables, and a byte permute looks up four codes at a time --
+// exactly w' = bf16_RN(fp32(ahat * c[q])).  The 2 KB of BF16 go through a
+// per-warp shared buffer (16-byte pieces rotated so that neither side has
+// bank conflicts) and leave as four 512-byte rows, one contiguous store
+// instruction each.
 // ===========================================================================
 struct DeqIn {
     uint4 cw;   // 32 codes
@@ -414,13 +416,17 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4 *__restric
                                                           const float *__restrict__ absmax,
                                                           const int8_t *__restrict__ qabs,
                                                           const float *__restrict__ scale,
-                                                          const float *__restrict__ mu_p, int64_t ngroups,
+                                                          const float *__restrict__ mu_p, int64_t nchunks,
                                                           uint4 *__restrict__ out) {
+    __shared__ __align__(16) uint4 stage[8][128];  // per warp 2 KB
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    uint4 *buf = stage[wib];
     const float mu = qabs ? __ldg(mu_p) : 0.f;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    auto fetch = [&](int64_t i, DeqIn &d) {
-        if (i < ngroups) {
-            const int64_t j = i >> 1;  // two 32-weight groups per block
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    auto fetch = [&](int64_t ch, DeqIn &d) {
+        if (ch < nchunks) {
+            const int64_t i = ch * 32 + lane;  // 32-weight group
+            const int64_t j = i >> 1;          // two groups per block
             d.cw = __ldcs(codes128 + i);
             if (qabs) {
                 d.q = __ldg(qabs + j);
@@ -431,34 +437,75 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4 *__restric
             }
         }
     };
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    DeqIn cur, nxt;
-    fetch(i, cur);
-    for (; i < ngroups; i += stride) {
-        fetch(i + stride, nxt);
-        const float ah = qabs ? dq_restore(cur.q, cur.v, mu) : cur.v;
+    int64_t ch = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib;
+    DeqIn d0, d1, d2;
+    fetch(ch, d0);
+    fetch(ch + nwarps, d1);
+    for (; ch < nchunks; ch += nwarps) {
+        fetch(ch + 2 * nwarps, d2);
+        const float ah = qabs ? dq_restore(d0.q, d0.v, mu) : d0.v;
         const NF4Table t = nf4_table(ah);
-        uint4 *o = out + 4 * i;
-        __stcs(o + 0, nf4_decode8(cur.cw.x, t));
-        __stcs(o + 1, nf4_decode8(cur.cw.y, t));
-        __stcs(o + 2, nf4_decode8(cur.cw.z, t));
-        __stcs(o + 3, nf4_decode8(cur.cw.w, t));
-        cur = nxt;
+        // piece w of lane l (bytes 64 l + 16 w of the chunk) sits at slot 4 l + ((w + l/2) & 3)
+        const int rot = lane >> 1;
+        buf[4 * lane + ((0 + rot) & 3)] = nf4_decode8(d0.cw.x, t);
+        buf[4 * lane + ((1 + rot) & 3)] = nf4_decode8(d0.cw.y, t);
+        buf[4 * lane + ((2 + rot) & 3)] = nf4_decode8(d0.cw.z, t);
+        buf[4 * lane + ((3 + rot) & 3)] = nf4_decode8(d0.cw.w, t);
+        __syncwarp();
+        uint4 *o = out + ch * 128;
+#pragma unroll
+        for (int row = 0; row < 4; ++row) {
+            const int piece = 32 * row + lane;            // 16-byte piece of the chunk
+            const int src = piece >> 2, w = piece & 3;    // written by lane src as its piece w
+            __stcs(o + piece, buf[4 * src + ((w + (src >> 1)) & 3)]);
+        }
+        __syncwarp();
+        d0 = d1;
+        d1 = d2;
     }
+}
+
+// The last (numel mod 1024) weights: one thread per 32-weight group.
+__global__ void nf4_dequant_tail_kernel(const uint4 *__restrict__ codes128, const float *__restrict__ absmax,
+                                        const int8_t *__restrict__ qabs, const float *__restrict__ scale,
+                                        const float *__restrict__ mu_p, int64_t g0, int64_t ng,
+                                        uint4 *__restrict__ out) {
+    const int64_t k = threadIdx.x;
+    if (k >= ng) return;
+    const int64_t i = g0 + k, j = i >> 1;
+    const float ah = qabs ? dq_restore(__ldg(qabs + j), __ldg(scale + (j >> 8)), __ldg(mu_p)) : __ldg(absmax + j);
+    const NF4Table t = nf4_table(ah);
+    const uint4 cw = __ldg(codes128 + i);
+    out[4 * i + 0] = nf4_decode8(cw.x, t);
+    out[4 * i + 1] = nf4_decode8(cw.y, t);
+    out[4 * i + 2] = nf4_decode8(cw.z, t);
+    out[4 * i + 3] = nf4_decode8(cw.w, t);
 }
 
 cudaError_t launch_nf4_dequant(const qln_nf4_weight *w, uint16_t *out, cudaStream_t st, int num_sms) {
     const int64_t numel = w->rows * w->cols;
-    const int64_t ngroups = numel / 32;
-    int64_t grid = (ngroups + 255) / 256;
-    const int64_t cap = (int64_t)num_sms * 8;
+    const int64_t nchunks = numel / 1024;  // weights come in whole 64-blocks; chunks of 1024 + a tail below
+    const int64_t tail = numel - nchunks * 1024;
+    int64_t grid = (nchunks + 7) / 8;
+    const int64_t cap = (int64_t)num_sms * 6;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
-    nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(w->codes), w->absmax, w->qabs,
-                                                      w->dq_scale, w->dq_mean, ngroups,
-                                                      reinterpret_cast<uint4 *>(out));
-    note_launch();
-    return cudaGetLastError();
+    if (nchunks > 0) {
+        nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(w->codes), w->absmax,
+                                                          w->qabs, w->dq_scale, w->dq_mean, nchunks,
+                                                          reinterpret_cast<uint4 *>(out));
+        note_launch();
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (tail > 0) {  // fewer than 1024 weights left: whole blocks, one 32-weight group per thread
+        const int64_t g0 = nchunks * 32, ng = tail / 32;
+        nf4_dequant_tail_kernel<<<1, 64, 0, st>>>(reinterpret_cast<const uint4 *>(w->codes), w->absmax, w->qabs,
+                                                   w->dq_scale, w->dq_mean, g0, ng, reinterpret_cast<uint4 *>(out));
+        note_launch();
+        return cudaGetLastError();
+    }
+    return cudaSuccess;
 }
 
 }  // namespace qln

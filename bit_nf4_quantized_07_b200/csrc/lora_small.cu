@@ -6,14 +6,16 @@
 // first (r x dseq) and BA never is; only A and B are trained.  Deck
 // "3 QLoRA Finetuning" card 1: gradients flow through the dequantized weight.
 //   lora_down : U = X A^T  (forward)  and  G = dY B  (backward)
-//   tn_reduce : dA = s G^T X  and  dB = s dY^T U    (reductions over tokens)
+//   tn_skinny : dA = s G^T X  and  dB = s dY^T U    (reductions over tokens)
 #include "qln_common.cuh"
 #include "qln_internal.h"
 
 namespace qln {
 
 // ===========================================================================
-// lora_down: out[t][j] = sum_k in[t][k] * wt[j][k], in [n][K], wt [r][K].
+// lora_down: out[t][j] = sum_k in[t][k] * wt[j][k], in [n][K], wt [r][K]
+// (WKM = false) or wt stored K-major as [K][r] (WKM = true, i.e. wt^T row-major:
+// G = dY B reads B [dout][r] as it is stored, no transpose).
 // Split-K tiles: a CTA owns 64 tokens x all r outputs over `cps` chunks of 64
 // k, streamed through a 4-stage cp.async ring (both operands K-contiguous, so
 // plain ldmatrix feeds the MMA); 4 warps x 16 tokens each.  Each split writes
@@ -23,13 +25,14 @@ namespace qln {
 constexpr int kDnStages = 4;
 constexpr int kDnLd = 72;  // padded row (bf16) of the staged tiles
 
-template <int NT>
+template <int NT, bool WKM>
 __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t *__restrict__ in, int64_t n, int64_t K,
                                                         const uint16_t *__restrict__ wt, int r, int cps,
                                                         float *__restrict__ partial) {
     extern __shared__ __align__(16) uint16_t dsm[];
     constexpr int WR = NT * 8;                              // adapter rows staged (r rounded up to 8)
-    constexpr int STAGE = (64 + WR) * kDnLd;                // elements per stage
+    constexpr int WKLD = WR + 8;                            // padded row of a K-major wt stage
+    constexpr int STAGE = 64 * kDnLd + (WKM ? 64 * WKLD : WR * kDnLd);  // elements per stage
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int64_t t0 = (int64_t)blockIdx.x * 64;
@@ -55,10 +58,18 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t *__restri
             const bool ok = t < n;
             cp_async16_zfill(Xs + row * kDnLd + 8 * ck, ok ? in + t * K + k0 + 8 * ck : in, ok ? 16 : 0);
         }
-        for (int idx = tid; idx < WR * 8; idx += 128) {
-            const int row = idx >> 3, ck = idx & 7;
-            const bool ok = row < r;
-            cp_async16_zfill(Ws + row * kDnLd + 8 * ck, ok ? wt + (int64_t)row * K + k0 + 8 * ck : wt, ok ? 16 : 0);
+        if (WKM) {  // 64 k rows x WR/8 chunks of the [K][r] layout
+            for (int idx = tid; idx < 64 * (WR / 8); idx += 128) {
+                const int row = idx / (WR / 8), ck = idx % (WR / 8);
+                const bool ok = 8 * ck < r;
+                cp_async16_zfill(Ws + row * WKLD + 8 * ck, ok ? wt + (k0 + row) * (int64_t)r + 8 * ck : wt, ok ? 16 : 0);
+            }
+        } else {
+            for (int idx = tid; idx < WR * 8; idx += 128) {
+                const int row = idx >> 3, ck = idx & 7;
+                const bool ok = row < r;
+                cp_async16_zfill(Ws + row * kDnLd + 8 * ck, ok ? wt + (int64_t)row * K + k0 + 8 * ck : wt, ok ? 16 : 0);
+            }
         }
     };
 
@@ -87,23 +98,43 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t *__restri
                 const int col = kk + (lane >> 4) * 8;
                 ldmatrix_x4(a[0], a[1], a[2], a[3], Xs + row * kDnLd + col);
             }
+            if (WKM) {  // Ws [k][j]: the transposing load gives the k x n fragment
 #pragma unroll
-            for (int np = 0; np < NT / 2; ++np) {
-                const int row = np * 16 + (lane & 7) + (lane >> 4) * 8;
-                const int col = kk + ((lane >> 3) & 1) * 8;
-                uint32_t r0, r1, r2, r3;
-                ldmatrix_x4(r0, r1, r2, r3, Ws + row * kDnLd + col);
-                const uint32_t b0[2] = {r0, r1}, b1[2] = {r2, r3};
-                mma_bf16_16816(acc[2 * np], a, b0);
-                mma_bf16_16816(acc[2 * np + 1], a, b1);
-            }
-            if (NT & 1) {
-                const int row = (NT - 1) * 8 + (lane & 7);
-                const int col = kk + ((lane >> 3) & 1) * 8;
-                uint32_t r0, r1;
-                ldmatrix_x2(r0, r1, Ws + row * kDnLd + col);
-                const uint32_t b0[2] = {r0, r1};
-                mma_bf16_16816(acc[NT - 1], a, b0);
+                for (int np = 0; np < NT / 2; ++np) {
+                    const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const int ncol = np * 16 + (lane >> 4) * 8;
+                    uint32_t r0, r1, r2, r3;
+                    ldmatrix_x4_trans(r0, r1, r2, r3, Ws + krow * WKLD + ncol);
+                    const uint32_t b0[2] = {r0, r1}, b1[2] = {r2, r3};
+                    mma_bf16_16816(acc[2 * np], a, b0);
+                    mma_bf16_16816(acc[2 * np + 1], a, b1);
+                }
+                if (NT & 1) {
+                    const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    uint32_t r0, r1;
+                    ldmatrix_x2_trans(r0, r1, Ws + krow * WKLD + (NT - 1) * 8);
+                    const uint32_t b0[2] = {r0, r1};
+                    mma_bf16_16816(acc[NT - 1], a, b0);
+                }
+            } else {
+#pragma unroll
+                for (int np = 0; np < NT / 2; ++np) {
+                    const int row = np * 16 + (lane & 7) + (lane >> 4) * 8;
+                    const int col = kk + ((lane >> 3) & 1) * 8;
+                    uint32_t r0, r1, r2, r3;
+                    ldmatrix_x4(r0, r1, r2, r3, Ws + row * kDnLd + col);
+                    const uint32_t b0[2] = {r0, r1}, b1[2] = {r2, r3};
+                    mma_bf16_16816(acc[2 * np], a, b0);
+                    mma_bf16_16816(acc[2 * np + 1], a, b1);
+                }
+                if (NT & 1) {
+                    const int row = (NT - 1) * 8 + (lane & 7);
+                    const int col = kk + ((lane >> 3) & 1) * 8;
+                    uint32_t r0, r1;
+                    ldmatrix_x2(r0, r1, Ws + row * kDnLd + col);
+                    const uint32_t b0[2] = {r0, r1};
+                    mma_bf16_16816(acc[NT - 1], a, b0);
+                }
             }
         }
         __syncthreads();
@@ -151,11 +182,12 @@ size_t lora_down_partial_bytes(int64_t n, int64_t K, int r, int num_sms) {
     return (size_t)sp * (size_t)n * (size_t)r * sizeof(float);
 }
 
-template <int NT>
+template <int NT, bool WKM>
 static cudaError_t launch_down_t(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, int splits,
                                  int cps, float *partial, cudaStream_t st) {
-    const size_t smem = (size_t)kDnStages * (64 + NT * 8) * kDnLd * sizeof(uint16_t);
-    auto kern = lora_down_kernel<NT>;
+    const size_t smem =
+        (size_t)kDnStages * (64 * kDnLd + (WKM ? 64 * (NT * 8 + 8) : NT * 8 * kDnLd)) * sizeof(uint16_t);
+    auto kern = lora_down_kernel<NT, WKM>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
@@ -166,30 +198,39 @@ static cudaError_t launch_down_t(const uint16_t *in, int64_t n, int64_t K, const
     return cudaGetLastError();
 }
 
-cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, float scale,
-                             uint16_t *out, uint16_t *out_scaled, float *partial, cudaStream_t st, int num_sms) {
-    int splits, cps;
-    lora_down_plan(n, K, num_sms, &splits, &cps);
+template <bool WKM>
+static cudaError_t launch_down_nt(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, int splits,
+                                  int cps, float *partial, cudaStream_t st) {
     const int nt = (r + 7) / 8;
     cudaError_t e;
     switch (nt) {
-        case 1: e = launch_down_t<1>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 2: e = launch_down_t<2>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 3: e = launch_down_t<3>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 4: e = launch_down_t<4>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 5: e = launch_down_t<5>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 6: e = launch_down_t<6>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 7: e = launch_down_t<7>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 8: e = launch_down_t<8>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 9: e = launch_down_t<9>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 10: e = launch_down_t<10>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 11: e = launch_down_t<11>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 12: e = launch_down_t<12>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 13: e = launch_down_t<13>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 14: e = launch_down_t<14>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 15: e = launch_down_t<15>(in, n, K, wt, r, splits, cps, partial, st); break;
-        default: e = launch_down_t<16>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 1: e = launch_down_t<1, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 2: e = launch_down_t<2, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 3: e = launch_down_t<3, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 4: e = launch_down_t<4, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 5: e = launch_down_t<5, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 6: e = launch_down_t<6, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 7: e = launch_down_t<7, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 8: e = launch_down_t<8, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 9: e = launch_down_t<9, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 10: e = launch_down_t<10, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 11: e = launch_down_t<11, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 12: e = launch_down_t<12, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 13: e = launch_down_t<13, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 14: e = launch_down_t<14, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 15: e = launch_down_t<15, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        default: e = launch_down_t<16, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
     }
+    return e;
+}
+
+cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, bool wt_kmajor, int r,
+                             float scale, uint16_t *out, uint16_t *out_scaled, float *partial, cudaStream_t st,
+                             int num_sms) {
+    int splits, cps;
+    lora_down_plan(n, K, num_sms, &splits, &cps);
+    cudaError_t e = wt_kmajor ? launch_down_nt<true>(in, n, K, wt, r, splits, cps, partial, st)
+                              : launch_down_nt<false>(in, n, K, wt, r, splits, cps, partial, st);
     if (e != cudaSuccess) return e;
     const int64_t total = n * r;
     int64_t blocks = (total + 255) / 256;
@@ -200,95 +241,101 @@ cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uin
 }
 
 // ===========================================================================
-// tn_reduce: C[m][c] = scale * sum_t P[t][m] Q[t][c], P [n][M], Q [n][N]
-// (both row-major bf16), fp32 C.  64x64 output tiles, 32 tokens per step,
-// both operands staged with cp.async and read with ldmatrix.trans (the
-// reduction index t is the row index of both).  With splits > 1 each z-slice
-// of the grid covers an interleaved share of the token steps and writes an
-// fp32 partial tile; tn_fold adds the slices in a fixed order.
+// tn_skinny: C[m][j] = scale * sum_t P[t][m] Q[t][j] for a narrow side j < R
+// (R = the adapter rank, <= 128): P [n][M], Q [n][R] row-major bf16, fp32 out,
+// stored as C[m][j] or, with `transpose`, as C[j][m].  dB = s dY^T U is
+// (P = dY, Q = U); dA = s G^T X is the transpose of (P = X, Q = G).  A CTA owns
+// 128 m x all R over an interleaved share of the 32-token steps: 4 warps x 32
+// m, both operands staged by cp.async and read with ldmatrix.trans (t is the row
+// index of both).  Partials per token split are folded in a fixed order.
 // ===========================================================================
-constexpr int kTnBM = 64, kTnBN = 64, kTnBK = 32, kTnPad = 72, kTnStages = 4;
+constexpr int kSkBM = 128, kSkBK = 32, kSkPad = 136, kSkStages = 4;
 
-__global__ void __launch_bounds__(128) tn_reduce_kernel(const uint16_t *__restrict__ P, const uint16_t *__restrict__ Q,
-                                                        int64_t n, int64_t M, int64_t N, float scale,
+template <int NTJ>  // R <= 8 NTJ
+__global__ void __launch_bounds__(128) tn_skinny_kernel(const uint16_t *__restrict__ P, const uint16_t *__restrict__ Q,
+                                                        int64_t n, int64_t M, int R, float scale, bool transpose,
                                                         float *__restrict__ C, float *__restrict__ partials) {
-    __shared__ __align__(16) uint16_t Ps[kTnStages][kTnBK][kTnPad];
-    __shared__ __align__(16) uint16_t Qs[kTnStages][kTnBK][kTnPad];
+    constexpr int QW = NTJ * 8, QLD = QW + 8;
+    extern __shared__ __align__(16) uint16_t sk[];
+    uint16_t *Ps = sk;                                   // [stages][32][kSkPad]
+    uint16_t *Qs = sk + kSkStages * kSkBK * kSkPad;      // [stages][32][QLD]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
-    const int wm = warp & 1, wn = warp >> 1;  // 2x2 warps, 32x32 each
-    const int64_t m0 = (int64_t)blockIdx.y * kTnBM, n0 = (int64_t)blockIdx.x * kTnBN;
-    const int split = blockIdx.z, nsplit = gridDim.z;
-    const int64_t nsteps = (n + kTnBK - 1) / kTnBK;
+    const int64_t m0 = (int64_t)blockIdx.x * kSkBM;
+    const int split = blockIdx.y, nsplit = gridDim.y;
+    const int64_t nsteps = (n + kSkBK - 1) / kSkBK;
 
-    float acc[2][4][4];
+    float acc[2][NTJ][4];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < NTJ; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
 
     auto load = [&](int buf, int64_t step) {
-        const int64_t tb = step * kTnBK;
-        // 32 rows x 64 cols x 2 operands = 512 16-byte chunks; 4 per thread
+        const int64_t tb = step * kSkBK;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int idx = tid + 128 * i;  // 0..511
-            const int op = idx >> 8, rem = idx & 255, row = rem >> 3, ck = rem & 7;
+        for (int i = 0; i < 4; ++i) {  // P: 32 rows x 16 chunks
+            const int idx = tid + 128 * i, row = idx >> 4, ck = idx & 15;
+            const int64_t t = tb + row, col = m0 + 8 * ck;
+            const bool ok = t < n && col < M;
+            cp_async16_zfill(Ps + (buf * kSkBK + row) * kSkPad + 8 * ck, ok ? P + t * M + col : P, ok ? 16 : 0);
+        }
+        for (int idx = tid; idx < kSkBK * NTJ; idx += 128) {  // Q: 32 rows x NTJ chunks
+            const int row = idx / NTJ, ck = idx % NTJ;
             const int64_t t = tb + row;
-            const uint16_t *base = op ? Q : P;
-            const int64_t width = op ? N : M;
-            const int64_t col = (op ? n0 : m0) + 8 * ck;
-            const bool ok = (t < n) && (col < width);
-            const uint16_t *src = ok ? base + t * width + col : base;
-            uint16_t *dst = op ? &Qs[buf][row][8 * ck] : &Ps[buf][row][8 * ck];
-            cp_async16_zfill(dst, src, ok ? 16 : 0);
+            const bool ok = t < n && 8 * ck < R;
+            cp_async16_zfill(Qs + (buf * kSkBK + row) * QLD + 8 * ck, ok ? Q + t * R + 8 * ck : Q, ok ? 16 : 0);
         }
     };
 
-    // this split's token steps: split, split + nsplit, ...
     const int64_t mysteps = split < nsteps ? (nsteps - split + nsplit - 1) / nsplit : 0;
 #pragma unroll
-    for (int i = 0; i < kTnStages - 1; ++i) {
+    for (int i = 0; i < kSkStages - 1; ++i) {
         if (i < mysteps) load(i, split + (int64_t)i * nsplit);
         cp_async_commit();
     }
     for (int64_t it = 0; it < mysteps; ++it) {
         {
-            const int64_t nx = it + kTnStages - 1;
-            if (nx < mysteps) load((int)(nx % kTnStages), split + nx * nsplit);
+            const int64_t nx = it + kSkStages - 1;
+            if (nx < mysteps) load((int)(nx % kSkStages), split + nx * nsplit);
             cp_async_commit();
         }
-        cp_async_wait<kTnStages - 1>();
+        cp_async_wait<kSkStages - 1>();
         __syncthreads();
-        const int buf = (int)(it % kTnStages);
+        const int buf = (int)(it % kSkStages);
+        const uint16_t *Pb = Ps + buf * kSkBK * kSkPad;
+        const uint16_t *Qb = Qs + buf * kSkBK * QLD;
 #pragma unroll
-        for (int kk = 0; kk < kTnBK; kk += 16) {
-            uint32_t a[2][4], b[4][2];
+        for (int kk = 0; kk < kSkBK; kk += 16) {
+            uint32_t a[2][4];
+            const int mat = lane >> 3;
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
-                const int mat = lane >> 3;
                 const int krow = kk + (mat >> 1) * 8 + (lane & 7);
-                const int mcol = wm * 32 + mt * 16 + (mat & 1) * 8;
-                ldmatrix_x4_trans(a[mt][0], a[mt][1], a[mt][2], a[mt][3], &Ps[buf][krow][mcol]);
+                const int mcol = warp * 32 + mt * 16 + (mat & 1) * 8;
+                ldmatrix_x4_trans(a[mt][0], a[mt][1], a[mt][2], a[mt][3], Pb + krow * kSkPad + mcol);
             }
+            const int krow = kk + (mat & 1) * 8 + (lane & 7);
 #pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                const int mat = lane >> 3;
-                const int krow = kk + (mat & 1) * 8 + (lane & 7);
-                const int ncol = wn * 32 + np * 16 + (mat >> 1) * 8;
+            for (int np = 0; np < NTJ / 2; ++np) {
                 uint32_t r0, r1, r2, r3;
-                ldmatrix_x4_trans(r0, r1, r2, r3, &Qs[buf][krow][ncol]);
-                b[2 * np][0] = r0;
-                b[2 * np][1] = r1;
-                b[2 * np + 1][0] = r2;
-                b[2 * np + 1][1] = r3;
+                ldmatrix_x4_trans(r0, r1, r2, r3, Qb + krow * QLD + np * 16 + (mat >> 1) * 8);
+                const uint32_t b0[2] = {r0, r1}, b1[2] = {r2, r3};
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    mma_bf16_16816(acc[mt][2 * np], a[mt], b0);
+                    mma_bf16_16816(acc[mt][2 * np + 1], a[mt], b1);
+                }
             }
+            if (NTJ & 1) {
+                uint32_t r0, r1;
+                ldmatrix_x2_trans(r0, r1, Qb + krow * QLD + (NTJ - 1) * 8);
+                const uint32_t b0[2] = {r0, r1};
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) mma_bf16_16816(acc[mt][nt], a[mt], b[nt]);
+                for (int mt = 0; mt < 2; ++mt) mma_bf16_16816(acc[mt][NTJ - 1], a[mt], b0);
+            }
         }
         __syncthreads();
     }
@@ -297,55 +344,90 @@ __global__ void __launch_bounds__(128) tn_reduce_kernel(const uint16_t *__restri
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int nt = 0; nt < NTJ; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int64_t m = m0 + wm * 32 + mt * 16 + g + 8 * (e >> 1);
-                const int64_t cc = n0 + wn * 32 + nt * 8 + 2 * c + (e & 1);
-                if (m < M && cc < N) {
-                    if (partials) partials[((int64_t)split * M + m) * N + cc] = acc[mt][nt][e];
-                    else C[m * N + cc] = __fmul_rn(scale, acc[mt][nt][e]);
+                const int64_t m = m0 + warp * 32 + mt * 16 + g + 8 * (e >> 1);
+                const int j = nt * 8 + 2 * c + (e & 1);
+                if (m < M && j < R) {
+                    if (partials)
+                        partials[((int64_t)split * M + m) * R + j] = acc[mt][nt][e];
+                    else
+                        C[transpose ? (int64_t)j * M + m : m * R + j] = __fmul_rn(scale, acc[mt][nt][e]);
                 }
             }
 }
 
-__global__ void tn_fold_kernel(const float *__restrict__ partials, int splits, int64_t MN, float scale,
-                               float *__restrict__ C) {
+__global__ void tn_skinny_fold_kernel(const float *__restrict__ partials, int splits, int64_t M, int R, float scale,
+                                      bool transpose, float *__restrict__ C) {
+    const int64_t MR = M * R;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < MN; i += stride) {
-        float s = 0.f;
-        for (int z = 0; z < splits; ++z) s = __fadd_rn(s, partials[(int64_t)z * MN + i]);
-        C[i] = __fmul_rn(scale, s);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < MR; i += stride) {
+        float v = 0.f;
+        for (int z = 0; z < splits; ++z) v = __fadd_rn(v, partials[(int64_t)z * MR + i]);
+        const int64_t m = i / R;
+        const int j = (int)(i % R);
+        C[transpose ? (int64_t)j * M + m : i] = __fmul_rn(scale, v);
     }
 }
 
-// About 6 CTAs per SM, each with at least 8 token steps (256 tokens).
-int tn_reduce_splits(int64_t n, int64_t M, int64_t N, int num_sms) {
-    const int64_t tiles = ((M + kTnBM - 1) / kTnBM) * ((N + kTnBN - 1) / kTnBN);
-    const int64_t steps = (n + kTnBK - 1) / kTnBK;
+// About 6 CTAs per SM, each with at least 4 token steps (128 tokens).
+int tn_skinny_splits(int64_t n, int64_t M, int num_sms) {
+    const int64_t tiles = (M + kSkBM - 1) / kSkBM;
+    const int64_t steps = (n + kSkBK - 1) / kSkBK;
     int64_t splits = (6 * (int64_t)num_sms + tiles - 1) / tiles;
-    const int64_t maxsp = steps / 8 > 0 ? steps / 8 : 1;
+    const int64_t maxsp = steps / 4 > 0 ? steps / 4 : 1;
     if (splits > maxsp) splits = maxsp;
     if (splits > 64) splits = 64;
     if (splits < 1) splits = 1;
     return (int)splits;
 }
 
-size_t tn_reduce_partials_bytes(int64_t M, int64_t N, int splits) {
-    return splits > 1 ? (size_t)splits * (size_t)M * (size_t)N * sizeof(float) : 0;
+size_t tn_skinny_partials_bytes(int64_t M, int R, int splits) {
+    return splits > 1 ? (size_t)splits * (size_t)M * (size_t)R * sizeof(float) : 0;
 }
 
-cudaError_t launch_tn_reduce(const uint16_t *P, const uint16_t *Q, int64_t n, int64_t M, int64_t N, float scale,
-                             float *C, float *partials, int splits, cudaStream_t st) {
-    dim3 grid((unsigned)((N + kTnBN - 1) / kTnBN), (unsigned)((M + kTnBM - 1) / kTnBM), (unsigned)splits);
-    tn_reduce_kernel<<<grid, 128, 0, st>>>(P, Q, n, M, N, scale, C, splits > 1 ? partials : nullptr);
+template <int NTJ>
+static cudaError_t launch_skinny_t(const uint16_t *P, const uint16_t *Q, int64_t n, int64_t M, int R, float scale,
+                                   bool transpose, float *C, float *partials, int splits, cudaStream_t st) {
+    const size_t smem = (size_t)kSkStages * kSkBK * (kSkPad + NTJ * 8 + 8) * sizeof(uint16_t);
+    auto kern = tn_skinny_kernel<NTJ>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    dim3 grid((unsigned)((M + kSkBM - 1) / kSkBM), (unsigned)splits);
+    kern<<<grid, 128, smem, st>>>(P, Q, n, M, R, scale, transpose, C, splits > 1 ? partials : nullptr);
     note_launch();
-    cudaError_t e = cudaGetLastError();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tn_skinny(const uint16_t *P, const uint16_t *Q, int64_t n, int64_t M, int R, float scale,
+                             bool transpose, float *C, float *partials, int splits, cudaStream_t st) {
+    cudaError_t e;
+    switch ((R + 7) / 8) {
+        case 1: e = launch_skinny_t<1>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 2: e = launch_skinny_t<2>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 3: e = launch_skinny_t<3>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 4: e = launch_skinny_t<4>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 5: e = launch_skinny_t<5>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 6: e = launch_skinny_t<6>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 7: e = launch_skinny_t<7>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 8: e = launch_skinny_t<8>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 9: e = launch_skinny_t<9>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 10: e = launch_skinny_t<10>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 11: e = launch_skinny_t<11>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 12: e = launch_skinny_t<12>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 13: e = launch_skinny_t<13>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 14: e = launch_skinny_t<14>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        case 15: e = launch_skinny_t<15>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+        default: e = launch_skinny_t<16>(P, Q, n, M, R, scale, transpose, C, partials, splits, st); break;
+    }
     if (e != cudaSuccess || splits <= 1) return e;
-    const int64_t MN = M * N;
-    int64_t blocks = (MN + 255) / 256;
+    const int64_t MR = M * R;
+    int64_t blocks = (MR + 255) / 256;
     if (blocks > 4096) blocks = 4096;
-    tn_fold_kernel<<<(unsigned)blocks, 256, 0, st>>>(partials, splits, MN, scale, C);
+    tn_skinny_fold_kernel<<<(unsigned)blocks, 256, 0, st>>>(partials, splits, M, R, scale, transpose, C);
     note_launch();
     return cudaGetLastError();
 }

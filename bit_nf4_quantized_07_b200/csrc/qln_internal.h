@@ -30,14 +30,17 @@ int64_t dq_max_blocks();
 //   out[t][j] = bf16(sum_k in[t][k] * wt[j][k]) and, if out_scaled != NULL,
 //   out_scaled[t][j] = bf16(scale * that sum); wt is [r][K] row-major.
 //   `partial` is fp32 scratch of lora_down_partial_bytes(n, K, r, num_sms).
-cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, float scale,
-                             uint16_t *out, uint16_t *out_scaled, float *partial, cudaStream_t st, int num_sms);
+//   wt_kmajor: wt is stored [K][r] instead (out[t][j] = sum_k in[t][k] * wt[k][j]).
+cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, bool wt_kmajor, int r,
+                             float scale, uint16_t *out, uint16_t *out_scaled, float *partial, cudaStream_t st,
+                             int num_sms);
 size_t lora_down_partial_bytes(int64_t n, int64_t K, int r, int num_sms);
-//   C[m][c] = scale * sum_t P[t][m] * Q[t][c]  (P [n][M], Q [n][N] row-major), fp32 out.
-cudaError_t launch_tn_reduce(const uint16_t *P, const uint16_t *Q, int64_t n, int64_t M, int64_t N, float scale,
-                             float *C, float *partials, int splits, cudaStream_t st);
-size_t tn_reduce_partials_bytes(int64_t M, int64_t N, int splits);
-int tn_reduce_splits(int64_t n, int64_t M, int64_t N, int num_sms);
+//   C = scale * P^T Q with Q [n][R] narrow (R <= 128): C[m][j], or C[j][m] with
+//   `transpose`; fp32 partials of tn_skinny_partials_bytes(M, R, splits).
+cudaError_t launch_tn_skinny(const uint16_t *P, const uint16_t *Q, int64_t n, int64_t M, int R, float scale,
+                             bool transpose, float *C, float *partials, int splits, cudaStream_t st);
+size_t tn_skinny_partials_bytes(int64_t M, int R, int splits);
+int tn_skinny_splits(int64_t n, int64_t M, int num_sms);
 
 // nf4_gemm_sm80.cu: fused NF4 decode + legacy mma.sync GEMM (small n).
 //   trans = false: out[t][m] = bf16(sum_k act[t][k] W'[m][k] + sum_j lact[t][j] lw[m][j])   (forward)
