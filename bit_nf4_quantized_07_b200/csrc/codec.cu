@@ -64,16 +64,25 @@ __device__ void build_snap_lut(uint2 *lut) {
 // group takes the exact path outright.
 __device__ __forceinline__ uint32_t snap4(float4 v, float a, float inv, const uint2 *lut) {
     const float w[4] = {v.x, v.y, v.z, v.w};
+    float y[4];
+    {   // both products of a pair from one paired multiply (each rounded to nearest)
+        uint64_t inv2, p01, p23;
+        asm("mov.b64 %0, {%1, %1};" : "=l"(inv2) : "f"(inv));
+        asm("{\n\t.reg .b64 a;\n\tmov.b64 a, {%1, %2};\n\tmul.rn.f32x2 %0, a, %3;\n\t}" : "=l"(p01) : "f"(w[0]), "f"(w[1]), "l"(inv2));
+        asm("{\n\t.reg .b64 a;\n\tmov.b64 a, {%1, %2};\n\tmul.rn.f32x2 %0, a, %3;\n\t}" : "=l"(p23) : "f"(w[2]), "f"(w[3]), "l"(inv2));
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(y[0]), "=f"(y[1]) : "l"(p01));
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(y[2]), "=f"(y[3]) : "l"(p23));
+    }
     uint32_t q[4];
-    bool near = false;
+    float dmin = 1.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float y = __fmul_rn(w[i], inv);
-        const uint2 e = lut[__float_as_uint(y) >> 20];
-        const float d = __fsub_rn(y, __uint_as_float(e.x));
+        const uint2 e = lut[__float_as_uint(y[i]) >> 20];
+        const float d = __fsub_rn(y[i], __uint_as_float(e.x));
         q[i] = e.y + (d > 0.f ? 1u : 0u);
-        near |= fabsf(d) < 4.76837158203125e-07f;  // 2^-21
+        dmin = fminf(dmin, fabsf(d));
     }
+    const bool near = dmin < 4.76837158203125e-07f;  // some |y - t| < 2^-21
     if (near || !(a >= 0x1p-126f && a < 0x1p126f)) {  // rare: redo the group exactly (also for a or 1/a subnormal)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

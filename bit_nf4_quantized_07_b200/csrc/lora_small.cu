@@ -12,6 +12,21 @@
 
 namespace qln {
 
+// sum_{z < splits} p[z * pitch] in the order z = 0, 1, ...; the loads go out
+// eight at a time ahead of their adds.
+__device__ __forceinline__ float fold_splits(const float *__restrict__ p, int64_t pitch, int splits) {
+    float v = 0.f;
+    for (int z0 = 0; z0 < splits; z0 += 8) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = (z0 + u < splits) ? __ldcg(p + (int64_t)(z0 + u) * pitch) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (z0 + u < splits) v = __fadd_rn(v, x[u]);
+    }
+    return v;
+}
+
 // ===========================================================================
 // lora_down: out[t][j] = sum_k in[t][k] * wt[j][k], in [n][K], wt [r][K]
 // (WKM = false) or wt stored K-major as [K][r] (WKM = true, i.e. wt^T row-major:
@@ -156,8 +171,7 @@ __global__ void lora_fold_kernel(const float *__restrict__ partial, int splits, 
                                  uint16_t *__restrict__ out, uint16_t *__restrict__ out_scaled) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
-        float v = 0.f;
-        for (int z = 0; z < splits; ++z) v = __fadd_rn(v, partial[(int64_t)z * total + i]);
+        const float v = fold_splits(partial + i, total, splits);
         out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
         if (out_scaled) out_scaled[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, v)));
     }
@@ -363,8 +377,7 @@ __global__ void tn_skinny_fold_kernel(const float *__restrict__ partials, int sp
     const int64_t MR = M * R;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < MR; i += stride) {
-        float v = 0.f;
-        for (int z = 0; z < splits; ++z) v = __fadd_rn(v, partials[(int64_t)z * MR + i]);
+        const float v = fold_splits(partials + i, MR, splits);
         const int64_t m = i / R;
         const int j = (int)(i % R);
         C[transpose ? (int64_t)j * M + m : i] = __fmul_rn(scale, v);
