@@ -106,20 +106,67 @@ def nearest(x: float, cb=None) -> int:
 
 
 def quantize(w):
-    """fp32 weights (any shape, numel % 64 == 0, flattened row-major) ->
-    (codes uint8 [numel/2], absmax fp32 [numel/64]).
+    """fp32 weights (any shape and numel >= 1, flattened row-major) ->
+    (codes uint8 [ceil(numel/2)], absmax fp32 [ceil(numel/64)]).
 
     jjjymmm.cn "4-bit NormalFloat(NF4)": divide by the block ABSMAX, take the
-    nearest quant-book value; "LoRA 与 QLoRA" DQ: one constant per 64 weights."""
+    nearest quant-book value; "LoRA 与 QLoRA" DQ: one constant per 64 weights.
+    A last, partial block takes its absmax over the weights it has; an odd
+    numel leaves code 7 (a zero weight's code) in the last low nibble."""
     w = _c(w, np.float32).reshape(-1)
     n = w.size
-    if n % BLOCK:
-        raise ValueError("numel must be a multiple of 64")
-    codes = np.zeros(n // 2, np.uint8)
-    absmax = np.zeros(n // BLOCK, np.float32)
+    if n < 1:
+        raise ValueError("numel must be positive")
+    codes = np.zeros((n + 1) // 2, np.uint8)
+    absmax = np.zeros((n + BLOCK - 1) // BLOCK, np.float32)
     cb = cb32()
     lib().oracle_nf4_quantize(_ptr(w), n, _ptr(cb), _ptr(codes), _ptr(absmax))
     return codes, absmax
+
+
+def widen16(bits, kind: str):
+    """16-bit weights (bit patterns, uint16) -> their exact fp32 values.
+
+    The pages warn against loading a 16-bit checkpoint and then quantizing it
+    carelessly ("LoRA 与 QLoRA", QLoRA usage notes); the method itself is
+    defined on real weights, and every bf16 or fp16 value is exactly a binary32
+    value, so a 16-bit weight enters the quantizer as that value.
+      kind "bf16": the 16 bits are the top half of the binary32 pattern;
+      kind "f16":  IEEE binary16 -> binary32 (exact, subnormals included)."""
+    b = np.ascontiguousarray(bits, np.uint16).reshape(-1)
+    if kind == "bf16":
+        return (b.astype(np.uint32) << 16).view(np.float32)
+    if kind == "f16":
+        return _f16_to_f32(b)
+    raise ValueError(kind)
+
+
+def _f16_to_f32(b):
+    """binary16 bits -> binary32, written out from the two formats' fields."""
+    b = b.astype(np.uint32)
+    sign = (b >> 15) << 31
+    exp = (b >> 10) & 0x1F
+    man = b & 0x3FF
+    out = np.zeros(b.size, np.uint32)
+    normal = (exp > 0) & (exp < 31)
+    out[normal] = sign[normal] | ((exp[normal] + (127 - 15)) << 23) | (man[normal] << 13)
+    special = exp == 31  # inf / NaN keep their payload
+    out[special] = sign[special] | (0xFF << 23) | (man[special] << 13)
+    zero = (exp == 0) & (man == 0)
+    out[zero] = sign[zero]
+    sub = (exp == 0) & (man != 0)  # value man * 2^-24: normalise
+    for i in np.nonzero(sub)[0]:
+        m, e = int(man[i]), -14
+        while not (m & 0x400):
+            m <<= 1
+            e -= 1
+        out[i] = int(sign[i]) | ((e + 127) << 23) | ((m & 0x3FF) << 13)
+    return out.view(np.float32)
+
+
+def quantize16(bits, kind: str):
+    """quantize() of 16-bit weights: the exact fp32 values (widen16), quantized."""
+    return quantize(widen16(bits, kind))
 
 
 def pairwise_sum(a) -> float:
@@ -201,11 +248,11 @@ def bf16_bits_to_f64(bits):
 
 
 def unpack_codes(codes, numel):
-    """uint8 [numel/2] -> uint8 [numel] of 4-bit codes (element 2i = high nibble)."""
+    """uint8 [ceil(numel/2)] -> uint8 [numel] of 4-bit codes (element 2i = high nibble)."""
     c = np.ascontiguousarray(codes, np.uint8).reshape(-1)
     out = np.empty(numel, np.uint8)
-    out[0::2] = c >> 4
-    out[1::2] = c & 15
+    out[0::2] = (c >> 4)[:(numel + 1) // 2]
+    out[1::2] = (c & 15)[:numel // 2]
     return out
 
 

@@ -105,29 +105,34 @@ int oracle_nf4_nearest(float x, const float cb[16]) {
     return best;
 }
 
-/* W (numel fp32, numel % 64 == 0) -> codes (numel/2 bytes, element 2i in the
- * high nibble of byte i) and absmax (numel/64 fp32).
+/* W (numel fp32, any numel >= 1) -> codes (ceil(numel/2) bytes, element 2i
+ * in the high nibble of byte i) and absmax (ceil(numel/64) fp32).
  * a_j = max |w| over block j [P1 DQ: a_j = max|W_j|]; x = w / a_j rounded to
  * binary32; code = nearest entry.  An all-zero block (a_j == 0) gets code 7
- * (the exact zero) everywhere. */
+ * (the exact zero) everywhere.
+ * Tails (reading; the pages only use whole blocks): the last block holds the
+ * numel mod 64 remaining weights and its absmax is taken over them; when numel
+ * is odd the low nibble of the last byte is code 7, the code a zero weight
+ * gets -- the same bytes as quantizing W zero-padded to whole blocks. */
 void oracle_nf4_quantize(const float *w, int64_t numel, const float cb[16],
                          uint8_t *codes, float *absmax) {
-    int64_t nb = numel / 64;
+    int64_t nb = (numel + 63) / 64;
     for (int64_t j = 0; j < nb; ++j) {
         const float *blk = w + j * 64;
+        int len = numel - j * 64 < 64 ? (int)(numel - j * 64) : 64;
         float a = 0.0f;
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < len; ++i) {
             float m = fabsf(blk[i]);
             if (m > a) a = m;
         }
         absmax[j] = a;
         int q[64];
         for (int i = 0; i < 64; ++i) {
-            if (a == 0.0f) { q[i] = 7; continue; }
+            if (i >= len || a == 0.0f) { q[i] = 7; continue; }
             float x = blk[i] / a;
             q[i] = oracle_nf4_nearest(x, cb);
         }
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; 2 * i < len; ++i)
             codes[j * 32 + i] = (uint8_t)((q[2 * i] << 4) | q[2 * i + 1]);
     }
 }
@@ -219,15 +224,15 @@ uint16_t oracle_bf16_rn(float f) {
 /* [P4 QLoRA: doubleDequant restores the quantization constant first, then
  * dequantizes the weight with it; P4 NF4: dequantization takes the quant-book
  * value] [P2 card 1: weights are dequantized to BFloat16 for the matmul]
- *   w' = bf16_RN( fp32( ahat_j * cb[q] ) )
+ *   w' = bf16_RN( fp32( ahat_j * cb[q] ) ),  for the numel weights (any numel)
  * With qabs == NULL the block constants are the plain fp32 absmax (no DQ). */
 void oracle_nf4_dequant(const uint8_t *codes, int64_t numel, const float *absmax,
                         const int8_t *qabs, const float *scale, const float *mu,
                         const float cb[16], uint16_t *out) {
-    int64_t nb = numel / 64;
+    int64_t nb = (numel + 63) / 64;
     for (int64_t j = 0; j < nb; ++j) {
         float a = qabs ? oracle_dq_restore(qabs[j], scale[j / 256], *mu) : absmax[j];
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < 64 && j * 64 + i < numel; ++i) {
             int64_t e = j * 64 + i;
             uint8_t byte = codes[e / 2];
             int q = (e % 2 == 0) ? (byte >> 4) : (byte & 15);
@@ -241,10 +246,10 @@ void oracle_nf4_dequant(const uint8_t *codes, int64_t numel, const float *absmax
 void oracle_nf4_dequant_f32(const uint8_t *codes, int64_t numel, const float *absmax,
                             const int8_t *qabs, const float *scale, const float *mu,
                             const float cb[16], float *out) {
-    int64_t nb = numel / 64;
+    int64_t nb = (numel + 63) / 64;
     for (int64_t j = 0; j < nb; ++j) {
         float a = qabs ? oracle_dq_restore(qabs[j], scale[j / 256], *mu) : absmax[j];
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < 64 && j * 64 + i < numel; ++i) {
             int64_t e = j * 64 + i;
             uint8_t byte = codes[e / 2];
             int q = (e % 2 == 0) ? (byte >> 4) : (byte & 15);

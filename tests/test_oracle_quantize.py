@@ -136,6 +136,71 @@ def test_codebook_points_roundtrip():
     assert np.array_equal(cb[q] * np.float32(0.5), w)
 
 
-def test_rejects_ragged_numel():
+def test_rejects_empty_input():
     with pytest.raises(ValueError):
-        codec.quantize(np.zeros(65, np.float32))
+        codec.quantize(np.zeros(0, np.float32))
+
+
+@pytest.mark.parametrize("n", [1, 2, 5, 63, 65, 127, 130, 1000, 4097])
+def test_ragged_numel_equals_zero_padded_whole_blocks(n):
+    """A partial last block: its absmax covers only the weights it has, and the
+    bytes are those of W zero-padded to whole blocks (a zero weight gets code 7,
+    and |0| never raises an absmax), cut to ceil(n/2) bytes."""
+    w = synthetic.normal_f32((n,), 0.02, 100 + n)
+    codes, absmax = codec.quantize(w)
+    pad = np.zeros(-(-n // 64) * 64, np.float32)
+    pad[:n] = w
+    cp, ap = codec.quantize(pad)
+    assert codes.size == (n + 1) // 2 and absmax.size == -(-n // 64)
+    assert np.array_equal(codes, cp[:(n + 1) // 2])
+    assert np.array_equal(absmax, ap)
+    if n % 2:
+        assert codes[-1] & 15 == 7
+    # dequant of the ragged codes: the first n weights of the padded dequant
+    assert np.array_equal(codec.dequant(codes, n, absmax=absmax), codec.dequant(cp, pad.size, absmax=ap)[:n])
+
+
+def test_ragged_block_brute_force():
+    """Five weights, worked by hand in binary64: nearest book entry of
+    fp32(w / max|w|), lower code on ties, and the odd-numel padding nibble."""
+    w = np.array([0.3, -0.05, 0.012, -0.6, 0.2], np.float32)
+    codes, absmax = codec.quantize(w)
+    assert absmax[0] == np.float32(0.6)
+    cb = codec.cb32().astype(np.float64)
+    q = []
+    for v in w:
+        x = float(np.float32(v) / np.float32(0.6))
+        d = [abs(x - c) for c in cb]
+        q.append(min(range(16), key=lambda k: (d[k], k)))
+    assert q[3] == 0  # -absmax is the bottom of the book
+    expect = [(q[0] << 4) | q[1], (q[2] << 4) | q[3], (q[4] << 4) | 7]
+    assert list(codes) == expect
+
+
+def test_sixteen_bit_widening_is_exact():
+    """bf16 and fp16 weights enter the quantizer as their exact fp32 values:
+    checked against torch's bfloat16 and NumPy's float16 conversions on every
+    16-bit pattern, and on hand-picked values."""
+    import torch
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    f = codec.widen16(bits, "f16")
+    ref = bits.view(np.float16).astype(np.float32)
+    same = (f.view(np.uint32) == ref.view(np.uint32)) | (np.isnan(f) & np.isnan(ref))
+    assert same.all()
+    b = codec.widen16(bits, "bf16")
+    t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    same = (b.view(np.uint32) == t.view(np.uint32)) | (np.isnan(b) & np.isnan(t))
+    assert same.all()
+    assert codec.widen16(np.array([0x0001], np.uint16), "f16")[0] == np.float32(2.0 ** -24)
+    assert codec.widen16(np.array([0x3C00, 0xC000], np.uint16), "f16").tolist() == [1.0, -2.0]
+    assert codec.widen16(np.array([0x3F80, 0xBF00], np.uint16), "bf16").tolist() == [1.0, -0.5]
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f16"])
+def test_quantize16_is_quantize_of_the_widened_weights(kind):
+    g = np.random.Generator(np.random.PCG64(5))
+    w = (g.standard_normal(1000) * 0.02).astype(np.float32)
+    bits = (w.view(np.uint32) >> 16).astype(np.uint16) if kind == "bf16" else w.astype(np.float16).view(np.uint16)
+    codes, absmax = codec.quantize16(bits, kind)
+    c2, a2 = codec.quantize(codec.widen16(bits, kind))
+    assert np.array_equal(codes, c2) and np.array_equal(absmax, a2)
