@@ -293,10 +293,11 @@ def measure_decode(api, dev, copies=64, reps=5):
     return out
 
 
-def measure_sweep(api, dev):
+def measure_sweep(api, dev, use_graph=True):
     """Quantize + DQ and dequant of every linear of a 32-layer d=4096,
     ffn=11008 decoder (6.48 B parameters, generated on the device), one pass
-    each, CUDA events around each pass."""
+    each, CUDA events around each pass.  Each pass is a CUDA graph of all 224
+    matrices' calls (use_graph=False: enqueued from Python)."""
     import torch
     from bit_nf4_quantized_07_b200 import synthetic
     gen = torch.Generator(device=dev)
@@ -332,13 +333,26 @@ def measure_sweep(api, dev):
     quant_pass()
     deq_pass()
     torch.cuda.synchronize()
+    run_q, run_d = quant_pass, deq_pass
+    if use_graph:
+        gq, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gq):
+            quant_pass()
+        with torch.cuda.graph(gd):
+            deq_pass()
+        gq.replay()
+        gd.replay()
+        torch.cuda.synchronize()
+        run_q, run_d = gq.replay, gd.replay
     e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     e[0].record(stream)
-    quant_pass()
+    run_q()
     e[1].record(stream)
-    deq_pass()
+    run_d()
     e[2].record(stream)
     torch.cuda.synchronize()
+    if use_graph:
+        del gq, gd
     params = synthetic.sweep_params()
     qb, db = codec_bytes_per_param()
     tq, td = e[0].elapsed_time(e[1]) * 1e-3, e[1].elapsed_time(e[2]) * 1e-3
@@ -406,23 +420,59 @@ def run_ours(args):
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
-    def step(i, marks=None):
+    def step_body(i):
         W, X, A, B, dYs = sets[i % NSETS]
-        if marks is not None:
-            marks[0].record(stream)
         api.nf4_quantize(W, codes, absmax)
         api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)
-        if marks is not None:
-            marks[1].record(stream)
         api.nf4_dequant(wq, wdq)
-        if marks is not None:
-            marks[2].record(stream)
         api.qlora_linear_fwd(wq, X, A, B, cfg.s, Y=Y, U_out=U, ws=ws_f)
-        if marks is not None:
-            marks[3].record(stream)
         api.qlora_linear_bwd(wq, X, A, B, cfg.s, dYs, U=U, dX=dX, dA=dA, dB=dB, ws=ws_b)
-        if marks is not None:
-            marks[4].record(stream)
+
+    # Rows of the step, for the per-row times.
+    rows = {
+        "quantize_dq": lambda i: (api.nf4_quantize(sets[i % NSETS][0], codes, absmax),
+                                  api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)),
+        "quantize": lambda i: api.nf4_quantize(sets[i % NSETS][0], codes, absmax),
+        "double_quant": lambda i: api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq),
+        "dequant": lambda i: api.nf4_dequant(wq, wdq),
+        "fwd": lambda i: api.qlora_linear_fwd(wq, *sets[i % NSETS][1:4], cfg.s, Y=Y, U_out=U, ws=ws_f),
+        "bwd": lambda i: api.qlora_linear_bwd(wq, *sets[i % NSETS][1:4], cfg.s, sets[i % NSETS][4], U=U, dX=dX,
+                                              dA=dA, dB=dB, ws=ws_b),
+    }
+
+    # The step runs as a CUDA graph (one per input set): the library's calls
+    # are enqueued once, at capture, and every replay launches the same
+    # kernels.  --no-graph enqueues each call from Python instead.
+    captured = [0]
+
+    def capture(fn):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        l0 = api.launch_count()
+        with torch.cuda.graph(g):
+            fn()
+        captured[0] = api.launch_count() - l0  # kernels in the graph
+        torch.cuda.synchronize()
+        return g
+
+    graphs = None
+    launches_per_step = 0
+    if not args.no_graph:
+        graphs = []
+        for i in range(NSETS):
+            graphs.append(capture(lambda i=i: step_body(i)))
+            launches_per_step = captured[0]
+
+    def step(i):
+        if graphs is not None:
+            graphs[i % NSETS].replay()
+        else:
+            step_body(i)
         if world > 1:
             dp.allreduce_adapter_grads(dA, dB)
 
@@ -433,29 +483,41 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
 
-    marks = [[ev() for _ in range(5)] for _ in range(args.steps)]
     start, stop = ev(), ev()
     launches0 = api.launch_count()
     with ClockSampler(local) as clk:
         start.record(stream)
         for i in range(args.steps):
-            step(i, marks[i])
+            step(i)
         stop.record(stream)
         torch.cuda.synchronize()
-    launches = api.launch_count() - launches0
+    launches = api.launch_count() - launches0 if graphs is None else launches_per_step * args.steps
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     elapsed_ms = start.elapsed_time(stop)
-    sec = {"quantize_dq": 0.0, "dequant": 0.0, "fwd": 0.0, "bwd": 0.0}
-    for m in marks:
-        sec["quantize_dq"] += m[0].elapsed_time(m[1])
-        sec["dequant"] += m[1].elapsed_time(m[2])
-        sec["fwd"] += m[2].elapsed_time(m[3])
-        sec["bwd"] += m[3].elapsed_time(m[4])
-    sec = {k: v / args.steps for k, v in sec.items()}
     if world > 1:
         elapsed_ms = dp.max_over_ranks(elapsed_ms, device=dev)
+
+    # Per-row device times: each row alone, 2 * NSETS calls (rotating inputs)
+    # captured in one graph, replayed 3 times between CUDA events.
+    def row_ms(fn, reps=2 * NSETS):
+        g = capture(lambda: [fn(i) for i in range(reps)])
+        g.replay()
+        a0, a1 = ev(), ev()
+        a0.record(stream)
+        for _ in range(3):
+            g.replay()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return a0.elapsed_time(a1) / (3 * reps)
+
+    sec = {k: row_ms(f) for k, f in rows.items()}
+    codec_split = {"quantize_ms": sec.pop("quantize"), "double_quant_ms": sec.pop("double_quant")}
+    if graphs is not None:
+        del graphs
+        torch.cuda.synchronize()
 
     # End to end through the C ABI with host buffers: copies inside the timed region.
     W, X, A, B, dYs = sets[0]
@@ -506,6 +568,7 @@ def run_ours(args):
             "traffic": _recorded_traffic(cfg.name), "peak_source": peaks["source"] + " bf16 burst"}
     parts = {
         "quantize_dq_GBs": numel * qb / (sec["quantize_dq"] * 1e-3) / 1e9,
+        "quantize_dq_split": codec_split,
         "dequant_GBs": numel * db / (sec["dequant"] * 1e-3) / 1e9,
         "fwd_TFLOPs": fwd_tflops,
         "bwd_TFLOPs": cfg.bwd_flops() / (sec["bwd"] * 1e-3) / 1e12,
@@ -520,7 +583,9 @@ def run_ours(args):
            "config": {"workload": cfg.name, "dout": cfg.dout, "din": cfg.din, "n": cfg.n, "r": cfg.r, "s": cfg.s,
                       "global_batch": cfg.n * world, "parallelism": f"dp{world}",
                       "step": "nf4_quantize+nf4_double_quant+nf4_dequant+qlora_linear_fwd+qlora_linear_bwd",
-                      "l2": "3 rotating input sets (W0 fp32 alone 180 MB > 126 MB L2)"},
+                      "l2": "3 rotating input sets (W0 fp32 alone 180 MB > 126 MB L2)",
+                      "timing": "python-enqueued steps" if args.no_graph else
+                      "CUDA graph replay per step (one graph per input set)"},
            "gpu_launches": launches, "roofline": roof, "parts": parts, "clocks": clk.summary(),
            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}}
     if not args.no_extra:
@@ -529,7 +594,7 @@ def run_ours(args):
         parts["decode_4096x4096_r16"] = measure_decode(api, dev)
         for k, v in parts["decode_4096x4096_r16"].items():
             v["frac_hbm"] = v["GBs"] / peaks["hbm_gbs"]
-        sw = measure_sweep(api, dev)
+        sw = measure_sweep(api, dev, use_graph=not args.no_graph)
         sw["quantize_dq_frac_hbm"] = sw["quantize_dq_GBs"] / peaks["hbm_gbs"]
         sw["dequant_frac_hbm"] = sw["dequant_GBs"] / peaks["hbm_gbs"]
         parts["sweep_6.48B"] = sw
@@ -552,6 +617,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["prefill", "large", "pr1"], default="prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="enqueue every call from Python instead of replaying "
+                    "CUDA graphs of the step, the rows and the sweep")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode-shape and codec-sweep measurements")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the decode-shape measurement and print it (for profiling)")

@@ -25,8 +25,10 @@ STATUS_NAMES = {0: "QLN_OK", 1: "QLN_ERR_NULL", 2: "QLN_ERR_SHAPE", 3: "QLN_ERR_
 OP_DOUBLE_QUANT, OP_LINEAR_FWD, OP_LINEAR_BWD = 1, 2, 3
 
 #: Every symbol include/qlora_nf4.h declares.
-EXPORTS = ("nf4_quantize", "nf4_double_quant", "nf4_double_quant_noalloc", "nf4_dequant", "qlora_linear_fwd", "qlora_linear_bwd",
-           "qln_workspace_bytes", "qln_codebook", "qln_status_str", "qln_version", "qln_launch_count")
+EXPORTS = ("nf4_quantize", "nf4_quantize_ex", "nf4_double_quant", "nf4_double_quant_noalloc", "nf4_dequant",
+           "nf4_dequant_flat", "qlora_linear_fwd", "qlora_linear_bwd", "qln_workspace_bytes", "qln_codebook",
+           "qln_status_str", "qln_version", "qln_launch_count")
+DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
 
 
 class QLNError(RuntimeError):
@@ -55,9 +57,11 @@ def lib():
         WP = ctypes.POINTER(CNF4Weight)
         sig = {
             "nf4_quantize": ([P, I64, P, P, P], I32),
+            "nf4_quantize_ex": ([P, I32, I64, P, P, P], I32),
             "nf4_double_quant": ([P, I64, P, P, P, P, SZ, P], I32),
             "nf4_double_quant_noalloc": ([P, I64, P, P, P, P], I32),
             "nf4_dequant": ([WP, P, P], I32),
+            "nf4_dequant_flat": ([WP, I64, P, P], I32),
             "qlora_linear_fwd": ([WP, P, I64, P, P, I32, F, P, P, P, SZ, P], I32),
             "qlora_linear_bwd": ([WP, P, I64, P, P, I32, F, P, P, P, P, P, P, SZ, P], I32),
             "qln_workspace_bytes": ([I32, I64, I64, I64, I32], SZ),
@@ -144,15 +148,27 @@ class NF4Weight:
                           self.dq_mean.data_ptr() if self.dq_mean is not None else None, self.rows, self.cols)
 
 
+_DTYPES = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
+
+
 def nf4_quantize(W: torch.Tensor, codes: Optional[torch.Tensor] = None, absmax: Optional[torch.Tensor] = None):
-    """fp32 W (any shape, numel % 64 == 0) -> (codes uint8 [numel/2], absmax fp32 [numel/64])."""
+    """W (fp32, bf16 or fp16; any shape and numel) -> (codes uint8 [ceil(numel/2)],
+    absmax fp32 [ceil(numel/64)]).  fp32 weights in whole 64-blocks go through
+    nf4_quantize, everything else through nf4_quantize_ex (same bits for the
+    same values)."""
     n = W.numel()
+    if W.dtype not in _DTYPES:
+        raise ValueError(f"unsupported weight dtype {W.dtype}")
     if codes is None:
-        codes = torch.empty(n // 2, dtype=torch.uint8, device=W.device)
+        codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=W.device)
     if absmax is None:
-        absmax = torch.empty(n // 64, dtype=torch.float32, device=W.device)
+        absmax = torch.empty((n + 63) // 64, dtype=torch.float32, device=W.device)
     _need_cuda(W, codes, absmax)
-    _check("nf4_quantize", lib().nf4_quantize(_p(W), n, _p(codes), _p(absmax), _stream()))
+    if W.dtype == torch.float32 and n % 64 == 0:
+        _check("nf4_quantize", lib().nf4_quantize(_p(W), n, _p(codes), _p(absmax), _stream()))
+    else:
+        _check("nf4_quantize_ex", lib().nf4_quantize_ex(_p(W), _DTYPES[W.dtype], n, _p(codes), _p(absmax),
+                                                        _stream()))
     return codes, absmax
 
 
@@ -201,6 +217,17 @@ def nf4_dequant(w: NF4Weight, out: Optional[torch.Tensor] = None) -> torch.Tenso
     _need_cuda(w.codes, out)
     cw = w.c_struct()
     _check("nf4_dequant", lib().nf4_dequant(ctypes.byref(cw), _p(out), _stream()))
+    return out
+
+
+def nf4_dequant_flat(w: NF4Weight, numel: int, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """doubleDequant of a flat weight of any numel to BF16 [numel] (w.rows and
+    w.cols are not used)."""
+    if out is None:
+        out = torch.empty(numel, dtype=torch.bfloat16, device=w.codes.device)
+    _need_cuda(w.codes, out)
+    cw = w.c_struct()
+    _check("nf4_dequant_flat", lib().nf4_dequant_flat(ctypes.byref(cw), int(numel), _p(out), _stream()))
     return out
 
 

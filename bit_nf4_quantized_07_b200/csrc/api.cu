@@ -139,7 +139,19 @@ qln_status nf4_quantize(const float *W, int64_t numel, uint8_t *codes, float *ab
     int sms = 0;
     qln_status s = check_device(&sms);
     if (s != QLN_OK) return s;
-    return from_cuda(qln::launch_nf4_quantize(W, numel, codes, absmax, (cudaStream_t)stream, sms));
+    return from_cuda(qln::launch_nf4_quantize(W, QLN_DTYPE_F32, numel, codes, absmax, (cudaStream_t)stream, sms));
+}
+
+qln_status nf4_quantize_ex(const void *W, int32_t dtype, int64_t numel, uint8_t *codes, float *absmax,
+                           void *stream) {
+    if (!W || !codes || !absmax) return QLN_ERR_NULL;
+    if (numel <= 0) return QLN_ERR_SHAPE;
+    if (dtype != QLN_DTYPE_F32 && dtype != QLN_DTYPE_BF16 && dtype != QLN_DTYPE_F16) return QLN_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(absmax, 4)) return QLN_ERR_ALIGN;
+    int sms = 0;
+    qln_status s = check_device(&sms);
+    if (s != QLN_OK) return s;
+    return from_cuda(qln::launch_nf4_quantize(W, dtype, numel, codes, absmax, (cudaStream_t)stream, sms));
 }
 
 qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale, float *dq_mean,
@@ -177,6 +189,24 @@ qln_status nf4_dequant(const qln_nf4_weight *w, uint16_t *out, void *stream) {
     s = check_device(&sms);
     if (s != QLN_OK) return s;
     return from_cuda(qln::launch_nf4_dequant(w, out, (cudaStream_t)stream, sms));
+}
+
+qln_status nf4_dequant_flat(const qln_nf4_weight *w, int64_t numel, uint16_t *out, void *stream) {
+    if (!w || !w->codes || !out) return QLN_ERR_NULL;
+    if (w->qabs) {
+        if (!w->dq_scale || !w->dq_mean) return QLN_ERR_NULL;
+    } else if (!w->absmax) {
+        return QLN_ERR_NULL;
+    }
+    if (numel <= 0) return QLN_ERR_SHAPE;
+    if (!aligned(w->codes, 16) || !aligned(out, 16)) return QLN_ERR_ALIGN;
+    if (w->absmax && !aligned(w->absmax, 4)) return QLN_ERR_ALIGN;
+    if (w->dq_scale && !aligned(w->dq_scale, 4)) return QLN_ERR_ALIGN;
+    if (w->dq_mean && !aligned(w->dq_mean, 4)) return QLN_ERR_ALIGN;
+    int sms = 0;
+    qln_status s = check_device(&sms);
+    if (s != QLN_OK) return s;
+    return from_cuda(qln::launch_nf4_dequant_flat(w, numel, out, (cudaStream_t)stream, sms));
 }
 
 qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t n, const uint16_t *A,

@@ -53,6 +53,18 @@ __device__ __forceinline__ float nf4_threshold(int k) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel on the
+// stream is still running; pdl_wait() blocks until that kernel has completed
+// and its memory operations are visible, so every such kernel calls it before
+// its first access to global memory that another kernel reads or writes.
+// pdl_trigger() lets the next kernel on the stream be launched (it still
+// waits in its own pdl_wait()).  Both are no-ops without the attribute.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // Small conversions.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

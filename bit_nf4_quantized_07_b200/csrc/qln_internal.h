@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/qlora_nf4.h"
 
 namespace qln {
@@ -13,12 +15,34 @@ namespace qln {
 // Host-side count of kernels enqueued by this library (qln_launch_count).
 void note_launch();
 
+// Launch `kernel` with the programmatic stream-serialization attribute (the
+// kernel must call pdl_wait() before touching global memory that earlier
+// kernels on the stream read or write).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    note_launch();
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // codec.cu
-cudaError_t launch_nf4_quantize(const float *W, int64_t numel, uint8_t *codes, float *absmax,
+cudaError_t launch_nf4_quantize(const void *W, int dtype, int64_t numel, uint8_t *codes, float *absmax,
                                 cudaStream_t st, int num_sms);
 cudaError_t launch_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,
                                     void *ws, cudaStream_t st);
 cudaError_t launch_nf4_dequant(const qln_nf4_weight *w, uint16_t *out, cudaStream_t st, int num_sms);
+cudaError_t launch_nf4_dequant_flat(const qln_nf4_weight *w, int64_t numel, uint16_t *out, cudaStream_t st,
+                                    int num_sms);
 size_t dq_workspace_bytes(int64_t nb);
 // allocation-free variant: scratch in a file-scope device array (codec.cu)
 cudaError_t launch_nf4_double_quant_static(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,

@@ -78,6 +78,9 @@ typedef enum {
     QLN_ERR_INTERNAL = 8   /* device side: an internal consistency check failed*/
 } qln_status;
 
+/* Element types of the weights given to nf4_quantize_ex. */
+enum { QLN_DTYPE_F32 = 0, QLN_DTYPE_BF16 = 1, QLN_DTYPE_F16 = 2 };
+
 /* Workspace-sized operations (qln_workspace_bytes `op`). */
 enum { QLN_OP_DOUBLE_QUANT = 1, QLN_OP_LINEAR_FWD = 2, QLN_OP_LINEAR_BWD = 3 };
 
@@ -113,6 +116,25 @@ typedef struct {
  */
 QLN_API qln_status nf4_quantize(const float *W, int64_t numel, uint8_t *codes, float *absmax,
                         void *stream);
+
+/*
+ * nf4_quantize_ex -- nf4_quantize for 16-bit weights and for any numel.
+ * Checkpoints usually hold 16-bit weights ("LoRA 与 QLoRA", QLoRA usage notes:
+ * load the 16-bit model, then quantize).  Every bf16 or fp16 value is exactly
+ * an fp32 value, and that value is what gets quantized, so the result equals
+ * nf4_quantize of the weights widened to fp32, bit for bit.
+ *   W      [numel] in, element type `dtype` (QLN_DTYPE_F32, _BF16, _F16),
+ *          flattened row-major; numel >= 1, any value.
+ *   codes  [ceil(numel/2)] u8 out; absmax [ceil(numel/64)] fp32 out.
+ * Tails: the last block holds the numel mod 64 remaining weights (its absmax
+ * is over those); for odd numel the low nibble of the last byte is 7, the
+ * code a zero weight gets -- the same bytes as quantizing W zero-padded to
+ * whole blocks.  No byte of codes past ceil(numel/2) is written.
+ * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE if numel <= 0 or dtype is unknown;
+ * QLN_ERR_ALIGN if W or codes is not 16-byte aligned (absmax: 4-byte).
+ */
+QLN_API qln_status nf4_quantize_ex(const void *W, int32_t dtype, int64_t numel, uint8_t *codes, float *absmax,
+                                   void *stream);
 
 /*
  * nf4_double_quant -- quantize the block constants to 8 bits.
@@ -173,6 +195,16 @@ QLN_API qln_status nf4_double_quant_noalloc(const float *absmax, int64_t nb, int
  * QLN_ERR_ALIGN (codes, out).
  */
 QLN_API qln_status nf4_dequant(const qln_nf4_weight *w, uint16_t *out, void *stream);
+
+/*
+ * nf4_dequant_flat -- nf4_dequant of a flat weight of any numel (as written
+ * by nf4_quantize_ex).  w->rows and w->cols are ignored; blocks are 64
+ * consecutive weights of the flat array and the last may be partial.
+ *   out [numel] bf16 (uint16) out; nothing past numel is written.
+ * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE if numel <= 0; QLN_ERR_ALIGN (codes,
+ * out: 16-byte).
+ */
+QLN_API qln_status nf4_dequant_flat(const qln_nf4_weight *w, int64_t numel, uint16_t *out, void *stream);
 
 /*
  * qlora_linear_fwd -- fused QLoRA linear forward.

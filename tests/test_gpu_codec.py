@@ -68,6 +68,46 @@ def test_codec_crafted_edge_blocks():
     _check_all(w)
 
 
+def test_quantize_near_thresholds_with_inexact_reciprocals():
+    """Blocks whose absmax is not a power of two, filled with fp32 values a few
+    ulps either side of a * t_k for every threshold: the fast product w * (1/a)
+    and the exact quotient w / a disagree by an ulp or two there, so every
+    code checks the near-threshold fallback against the oracle's IEEE divide."""
+    cb = codec.cb32().astype(np.float64)
+    rng = np.random.Generator(np.random.PCG64(31))
+    blocks = []
+    for i in range(600):
+        a = np.float32(rng.uniform(0.01, 100.0))
+        b = np.empty(64, np.float32)
+        b[0] = a if i % 2 == 0 else -a
+        k = rng.integers(0, 15, 63)
+        t = np.float32(a * (cb[k] + cb[k + 1]) / 2)
+        steps = rng.integers(-3, 4, 63)
+        for j in range(63):
+            v = t[j]
+            for _ in range(abs(int(steps[j]))):
+                v = np.nextafter(v, np.float32(np.sign(steps[j]) * 1e9))
+            b[1 + j] = v
+        b[1:] = np.clip(b[1:], -a, a)
+        blocks.append(b)
+    _check_all(np.concatenate(blocks))
+
+
+def test_quantize_16_byte_aligned_input():
+    """W may be 16-byte but not 32-byte aligned (the wide-load path needs 32):
+    same codes and constants as from an aligned copy, ragged last chunk."""
+    w = synthetic.normal_f32((7 * 64 + 3 * 64,), 0.02, 41)
+    buf = torch.zeros(w.size + 8, dtype=torch.float32, device="cuda")
+    W = buf[4:4 + w.size]
+    assert W.data_ptr() % 32 == 16
+    W.copy_(torch.from_numpy(w))
+    codes, absmax = api.nf4_quantize(W)
+    torch.cuda.synchronize()
+    c_ref, a_ref = codec.quantize(w)
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+    assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+
+
 def test_dq_degenerate_groups():
     w = np.tile(np.r_[np.float32(0.25), np.zeros(63, np.float32)], 600)   # all a_j equal -> b == 0
     _check_all(w)
@@ -102,3 +142,61 @@ def test_large_size_codec_sampled():
         ah = codec.dq_restore(qabs[j:j + 1], scale[j // 256:j // 256 + 1], mu)[0]
         ref = codec.dequant(codes_s.reshape(-1, 32)[k], 64, absmax=np.array([ah], np.float32))
         assert np.array_equal(deq[k], ref)
+
+
+RAGGED = [1, 2, 7, 63, 64, 65, 130, 1000, 4096 + 37, (1 << 20) + 5, 3 * 1024 + 999]
+
+
+def _to_kind(w32: np.ndarray, kind: str):
+    """fp32 values -> (device tensor of that dtype, oracle input bits or values)."""
+    t = torch.from_numpy(w32)
+    if kind == "f32":
+        return t.cuda(), w32
+    dt = torch.bfloat16 if kind == "bf16" else torch.float16
+    d = t.to(dt)
+    return d.cuda(), d.view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("kind", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("n", RAGGED)
+def test_quantize_any_dtype_and_numel_bit_exact(kind, n):
+    """nf4_quantize_ex (and nf4_dequant_flat) against the oracle for 16-bit and
+    fp32 weights of any numel: codes, absmax, DQ and BF16 bits exact, and no
+    byte written past ceil(n/2) codes / n outputs."""
+    w32 = synthetic.normal_f32((n,), 0.02, 700 + n)
+    W, ref_in = _to_kind(w32, kind)
+    guard = 37
+    codes = torch.full(((n + 1) // 2 + guard,), 0xAB, dtype=torch.uint8, device="cuda")
+    absmax = torch.full(((n + 63) // 64 + 1,), -1.0, dtype=torch.float32, device="cuda")
+    api.nf4_quantize(W, codes=codes[:(n + 1) // 2], absmax=absmax[:(n + 63) // 64])
+    c_ref, a_ref = codec.quantize(ref_in) if kind == "f32" else codec.quantize16(ref_in, kind)
+    torch.cuda.synchronize()
+    cg = codes.cpu().numpy()
+    ag = absmax.cpu().numpy()
+    assert np.array_equal(cg[:(n + 1) // 2], c_ref), f"codes: {np.sum(cg[:(n + 1) // 2] != c_ref)} differ"
+    assert np.all(cg[(n + 1) // 2:] == 0xAB), "wrote past the codes"
+    assert np.array_equal(ag[:-1].view(np.uint32), a_ref.view(np.uint32)), "absmax"
+    assert ag[-1] == -1.0, "wrote past absmax"
+    # DQ + flat dequant of the ragged weight
+    am = absmax[:(n + 63) // 64]
+    qabs, scale, mu = api.nf4_double_quant(am)
+    q_ref, s_ref, mu_ref = codec.double_quant(a_ref)
+    wq = api.NF4Weight(codes=codes[:(n + 1) // 2], rows=1, cols=n, absmax=am, qabs=qabs, dq_scale=scale, dq_mean=mu)
+    out = torch.full((n + 24,), 0x7FC1, dtype=torch.int16, device="cuda")
+    api.nf4_dequant_flat(wq, n, out=out[:n].view(torch.bfloat16))
+    torch.cuda.synchronize()
+    assert np.array_equal(qabs.cpu().numpy(), q_ref) and np.float32(mu.item()) == np.float32(mu_ref)
+    og = out.cpu().numpy().view(np.uint16)
+    assert np.array_equal(og[:n], codec.dequant(c_ref, n, qabs=q_ref, scale=s_ref, mu=mu_ref)), "dequant"
+    assert np.all(og[n:] == 0x7FC1), "wrote past the dequant output"
+
+
+def test_quantize16_matches_fp32_path_on_prefill_weight():
+    """bf16 weights of the prefill layer: the 16-bit path gives the bytes the
+    fp32 path gives for the widened values."""
+    cfg = synthetic.PREFILL
+    w = torch.from_numpy(synthetic.weight_f32(cfg)).cuda().to(torch.bfloat16)
+    c16, a16 = api.nf4_quantize(w)
+    c32, a32 = api.nf4_quantize(w.float())
+    torch.cuda.synchronize()
+    assert torch.equal(c16, c32) and torch.equal(a16, a32)
