@@ -58,6 +58,18 @@ def lib():
         L.oracle_nf4_dequant.argtypes = [P, I64, P, P, P, P, P, P]
         L.oracle_nf4_dequant_f32.restype = None
         L.oracle_nf4_dequant_f32.argtypes = [P, I64, P, P, P, P, P, P]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_nf4_double_quant_e4m3.restype = None
+        L.oracle_nf4_double_quant_e4m3.argtypes = [P, I64, P, P, P]
+        L.oracle_dq_restore_e4m3.restype = ctypes.c_float
+        L.oracle_dq_restore_e4m3.argtypes = [ctypes.c_uint8, ctypes.c_float, ctypes.c_float]
+        L.oracle_nf4_dequant_fmt.restype = None
+        L.oracle_nf4_dequant_fmt.argtypes = [P, I64, P, P, ctypes.c_int, P, P, P, P]
+        L.oracle_nf4_dequant_f32_fmt.restype = None
+        L.oracle_nf4_dequant_f32_fmt.argtypes = [P, I64, P, P, ctypes.c_int, P, P, P, P]
         _lib = L
     return _lib
 
@@ -179,29 +191,53 @@ def dq_mean(absmax) -> np.float32:
     return np.float32(lib().oracle_dq_mean(_ptr(a), a.size))
 
 
-def double_quant(absmax):
-    """fp32 block constants -> (qabs int8 [nb], scale fp32 [ceil(nb/256)], mu fp32).
+def double_quant(absmax, fmt: str = "int8"):
+    """fp32 block constants -> (qabs [nb], scale fp32 [ceil(nb/256)], mu fp32).
 
     "LoRA 与 QLoRA" DQ: r_j = (a_j - mu)/b, 8-bit rhat_j, mu and b in 32 bits;
-    deck card 4 / jjjymmm.cn DQ: blocks of 256 constants."""
+    deck card 4 / jjjymmm.cn DQ: blocks of 256 constants.
+    fmt "int8": rhat = clamp(rint(r), -127, 127), b = max|d| / 127 (int8 array);
+    fmt "e4m3": deck card 4's "8-bit floats": rhat = E4M3(r) (nearest-even,
+    saturating), b = max|d| / 448 (uint8 array of E4M3 codes)."""
     a = _c(absmax, np.float32).reshape(-1)
     nb = a.size
     ng = (nb + DQ_GROUP - 1) // DQ_GROUP
-    qabs = np.zeros(nb, np.int8)
     scale = np.zeros(ng, np.float32)
     mu = np.zeros(1, np.float32)
-    lib().oracle_nf4_double_quant(_ptr(a), nb, _ptr(qabs), _ptr(scale), _ptr(mu))
+    if fmt == "int8":
+        qabs = np.zeros(nb, np.int8)
+        lib().oracle_nf4_double_quant(_ptr(a), nb, _ptr(qabs), _ptr(scale), _ptr(mu))
+    elif fmt == "e4m3":
+        qabs = np.zeros(nb, np.uint8)
+        lib().oracle_nf4_double_quant_e4m3(_ptr(a), nb, _ptr(qabs), _ptr(scale), _ptr(mu))
+    else:
+        raise ValueError(fmt)
     return qabs, scale, mu[0]
 
 
-def dq_restore(qabs, scale, mu):
+def e4m3_value(code: int) -> float:
+    """The value of an OCP FP8 E4M3 code (NaN for 0x7F / 0xFF)."""
+    return lib().oracle_e4m3_value(int(code) & 0xFF)
+
+
+def e4m3_encode(x: float) -> int:
+    """binary32 -> E4M3 code: nearest, ties to even mantissa, saturating at +-448."""
+    return int(lib().oracle_e4m3_encode(ctypes.c_float(x)))
+
+
+def dq_restore(qabs, scale, mu, fmt: str = "int8"):
     """ahat_j = fp32(mu + fp32(b_g * rhat_j)) for every j (vector form)."""
-    qabs = _c(qabs, np.int8).reshape(-1)
     scale = _c(scale, np.float32).reshape(-1)
-    out = np.empty(qabs.size, np.float32)
     L = lib()
-    for j in range(qabs.size):
-        out[j] = L.oracle_dq_restore(int(qabs[j]), float(scale[j // DQ_GROUP]), float(mu))
+    if fmt == "e4m3":
+        q = _c(qabs, np.uint8).reshape(-1)
+        f = lambda j: L.oracle_dq_restore_e4m3(int(q[j]), float(scale[j // DQ_GROUP]), float(mu))
+    else:
+        q = _c(qabs, np.int8).reshape(-1)
+        f = lambda j: L.oracle_dq_restore(int(q[j]), float(scale[j // DQ_GROUP]), float(mu))
+    out = np.empty(q.size, np.float32)
+    for j in range(q.size):
+        out[j] = f(j)
     return out
 
 
@@ -209,33 +245,36 @@ def bf16_rn(x: float) -> int:
     return lib().oracle_bf16_rn(ctypes.c_float(x))
 
 
-def dequant(codes, numel, absmax=None, qabs=None, scale=None, mu=None):
+def dequant(codes, numel, absmax=None, qabs=None, scale=None, mu=None, fmt: str = "int8"):
     """doubleDequant to BF16 bits (uint16 [numel]).
 
     jjjymmm.cn "QLoRA": restore the constant first, then the weight with it;
     deck card 1: weights are dequantized to BFloat16 for every matmul.
-    Pass ``absmax`` for plain NF4, or ``qabs, scale, mu`` for NF4 + DQ."""
+    Pass ``absmax`` for plain NF4, or ``qabs, scale, mu`` (and the DQ format)
+    for NF4 + DQ."""
     codes = _c(codes, np.uint8).reshape(-1)
     out = np.empty(numel, np.uint16)
     mu_arr = None if mu is None else np.array([mu], np.float32)
-    lib().oracle_nf4_dequant(
+    q = None if qabs is None else np.ascontiguousarray(qabs).view(np.uint8).reshape(-1)
+    lib().oracle_nf4_dequant_fmt(
         _ptr(codes), numel,
         _ptr(None if absmax is None else _c(absmax, np.float32)),
-        _ptr(None if qabs is None else _c(qabs, np.int8)),
+        _ptr(q), 1 if fmt == "e4m3" else 0,
         _ptr(None if scale is None else _c(scale, np.float32)),
         _ptr(mu_arr), _ptr(cb32()), _ptr(out))
     return out
 
 
-def dequant_f32(codes, numel, absmax=None, qabs=None, scale=None, mu=None):
+def dequant_f32(codes, numel, absmax=None, qabs=None, scale=None, mu=None, fmt: str = "int8"):
     """As :func:`dequant`, returning the fp32 product before BF16 rounding."""
     codes = _c(codes, np.uint8).reshape(-1)
     out = np.empty(numel, np.float32)
     mu_arr = None if mu is None else np.array([mu], np.float32)
-    lib().oracle_nf4_dequant_f32(
+    q = None if qabs is None else np.ascontiguousarray(qabs).view(np.uint8).reshape(-1)
+    lib().oracle_nf4_dequant_f32_fmt(
         _ptr(codes), numel,
         _ptr(None if absmax is None else _c(absmax, np.float32)),
-        _ptr(None if qabs is None else _c(qabs, np.int8)),
+        _ptr(q), 1 if fmt == "e4m3" else 0,
         _ptr(None if scale is None else _c(scale, np.float32)),
         _ptr(mu_arr), _ptr(cb32()), _ptr(out))
     return out

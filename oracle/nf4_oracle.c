@@ -199,10 +199,79 @@ void oracle_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs,
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* O3'. Double quantization with 8-bit floats (FP8 E4M3).                   */
+/* ------------------------------------------------------------------------ */
+
+/* [P2 card 4] quantizes the constants to "8-bit floats".  The 8-bit float
+ * format here is OCP FP8 E4M3 (the "fn" variant): 1 sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits, no infinities, NaN only at S.1111.111.
+ *   exponent field 0:      value = (m / 8) * 2^-6      (subnormals, +-0)
+ *   exponent field e > 0:  value = (1 + m / 8) * 2^(e-7)
+ * so the largest finite value is 1.75 * 2^8 = 448. */
+double oracle_e4m3_value(uint8_t code) {
+    int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Round a binary32 to E4M3: the nearest finite code, ties to the code with an
+ * even mantissa, and anything beyond +-448 saturated to +-448 ("satfinite").
+ * Brute force over the 127 non-negative finite codes; the sign is applied
+ * after (the format is sign-magnitude).  Distances are exact in binary64. */
+uint8_t oracle_e4m3_encode(float x) {
+    double ax = fabs((double)x);
+    uint8_t best = 0;
+    double bestd = INFINITY;
+    for (int c = 0; c <= 0x7e; ++c) {
+        double d = fabs(ax - oracle_e4m3_value((uint8_t)c));
+        if (d < bestd || (d == bestd && (c & 1) == 0)) {
+            bestd = d;
+            best = (uint8_t)c;
+        }
+    }
+    if (ax >= 448.0) best = 0x7e;
+    return (uint8_t)(best | (signbit(x) ? 0x80 : 0x00));
+}
+
+/* [P2 card 4] "8-bit floats" reading of the DQ step, otherwise as the INT8
+ * reading above (same mu, same groups of 256):
+ *   d_j   = fp32(a_j - mu)
+ *   b_g   = fp32(max_{j in g} |d_j| / 448)        (448: the largest E4M3 value)
+ *   rhat  = E4M3(fp32(d_j / b_g)), nearest-even, saturating; code 0 if b_g == 0. */
+void oracle_nf4_double_quant_e4m3(const float *absmax, int64_t nb, uint8_t *qabs,
+                                  float *scale, float *mu_out) {
+    float mu = oracle_dq_mean(absmax, nb);
+    *mu_out = mu;
+    int64_t ng = (nb + 255) / 256;
+    for (int64_t g = 0; g < ng; ++g) {
+        int64_t j0 = g * 256, j1 = j0 + 256 < nb ? j0 + 256 : nb;
+        float B = 0.0f;
+        for (int64_t j = j0; j < j1; ++j) {
+            float d = fabsf(absmax[j] - mu);
+            if (d > B) B = d;
+        }
+        float b = B / 448.0f;
+        scale[g] = b;
+        for (int64_t j = j0; j < j1; ++j) {
+            if (b == 0.0f) { qabs[j] = 0; continue; }
+            float r = (absmax[j] - mu) / b;
+            qabs[j] = oracle_e4m3_encode(r);
+        }
+    }
+}
+
 /* ahat_j = fp32(mu + fp32(b_g * rhat_j)) [P1 DQ reconstruction, in the written
  * order: the product first, then the sum]. */
 float oracle_dq_restore(int8_t rhat, float b, float mu) {
     float prod = b * (float)rhat;
+    return mu + prod;
+}
+
+/* The same with an E4M3 code (its value is exact in binary32). */
+float oracle_dq_restore_e4m3(uint8_t code, float b, float mu) {
+    float prod = b * (float)oracle_e4m3_value(code);
     return mu + prod;
 }
 
@@ -226,12 +295,14 @@ uint16_t oracle_bf16_rn(float f) {
  * value] [P2 card 1: weights are dequantized to BFloat16 for the matmul]
  *   w' = bf16_RN( fp32( ahat_j * cb[q] ) ),  for the numel weights (any numel)
  * With qabs == NULL the block constants are the plain fp32 absmax (no DQ). */
-void oracle_nf4_dequant(const uint8_t *codes, int64_t numel, const float *absmax,
-                        const int8_t *qabs, const float *scale, const float *mu,
-                        const float cb[16], uint16_t *out) {
+void oracle_nf4_dequant_fmt(const uint8_t *codes, int64_t numel, const float *absmax,
+                            const uint8_t *qabs, int e4m3, const float *scale, const float *mu,
+                            const float cb[16], uint16_t *out) {
     int64_t nb = (numel + 63) / 64;
     for (int64_t j = 0; j < nb; ++j) {
-        float a = qabs ? oracle_dq_restore(qabs[j], scale[j / 256], *mu) : absmax[j];
+        float a = !qabs ? absmax[j]
+                  : e4m3 ? oracle_dq_restore_e4m3(qabs[j], scale[j / 256], *mu)
+                         : oracle_dq_restore((int8_t)qabs[j], scale[j / 256], *mu);
         for (int i = 0; i < 64 && j * 64 + i < numel; ++i) {
             int64_t e = j * 64 + i;
             uint8_t byte = codes[e / 2];
@@ -242,13 +313,21 @@ void oracle_nf4_dequant(const uint8_t *codes, int64_t numel, const float *absmax
     }
 }
 
+void oracle_nf4_dequant(const uint8_t *codes, int64_t numel, const float *absmax,
+                        const int8_t *qabs, const float *scale, const float *mu,
+                        const float cb[16], uint16_t *out) {
+    oracle_nf4_dequant_fmt(codes, numel, absmax, (const uint8_t *)qabs, 0, scale, mu, cb, out);
+}
+
 /* Same as above but returns the binary32 value before the BF16 rounding. */
-void oracle_nf4_dequant_f32(const uint8_t *codes, int64_t numel, const float *absmax,
-                            const int8_t *qabs, const float *scale, const float *mu,
-                            const float cb[16], float *out) {
+void oracle_nf4_dequant_f32_fmt(const uint8_t *codes, int64_t numel, const float *absmax,
+                                const uint8_t *qabs, int e4m3, const float *scale, const float *mu,
+                                const float cb[16], float *out) {
     int64_t nb = (numel + 63) / 64;
     for (int64_t j = 0; j < nb; ++j) {
-        float a = qabs ? oracle_dq_restore(qabs[j], scale[j / 256], *mu) : absmax[j];
+        float a = !qabs ? absmax[j]
+                  : e4m3 ? oracle_dq_restore_e4m3(qabs[j], scale[j / 256], *mu)
+                         : oracle_dq_restore((int8_t)qabs[j], scale[j / 256], *mu);
         for (int i = 0; i < 64 && j * 64 + i < numel; ++i) {
             int64_t e = j * 64 + i;
             uint8_t byte = codes[e / 2];
@@ -256,4 +335,10 @@ void oracle_nf4_dequant_f32(const uint8_t *codes, int64_t numel, const float *ab
             out[e] = a * cb[q];
         }
     }
+}
+
+void oracle_nf4_dequant_f32(const uint8_t *codes, int64_t numel, const float *absmax,
+                            const int8_t *qabs, const float *scale, const float *mu,
+                            const float cb[16], float *out) {
+    oracle_nf4_dequant_f32_fmt(codes, numel, absmax, (const uint8_t *)qabs, 0, scale, mu, cb, out);
 }

@@ -131,3 +131,73 @@ def test_dequant_definition_and_special_codes():
     # without DQ the plain absmax is the constant
     plain = codec.dequant_f32(codes, n, absmax=absmax).reshape(-1, 64)
     assert np.array_equal(plain, absmax[:, None] * cb[q])
+
+
+# --- the "8-bit floats" reading of DQ (deck card 4): OCP FP8 E4M3 codes -----
+
+def test_e4m3_decode_against_torch_and_the_format_definition():
+    """Every code against torch.float8_e4m3fn's conversion (a library routine),
+    plus values fixed by the format: 1.0, the largest 448, the smallest
+    subnormal 2^-9, the smallest normal 2^-6, signed zero, the NaN codes."""
+    vals = np.array([codec.e4m3_value(c) for c in range(256)])
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    both_nan = np.isnan(vals) & np.isnan(ref)
+    assert np.all(both_nan | (vals == ref))
+    assert vals[0x38] == 1.0 and vals[0x7E] == 448.0 and vals[0xFE] == -448.0
+    assert vals[0x01] == 2.0 ** -9 and vals[0x08] == 2.0 ** -6 and vals[0x07] == 7 * 2.0 ** -9
+    assert vals[0x00] == 0.0 and math.copysign(1.0, vals[0x80]) == -1.0
+    assert np.isnan(vals[0x7F]) and np.isnan(vals[0xFF]) and np.isnan(vals).sum() == 2
+    finite = vals[:0x7F]
+    assert np.all(np.diff(finite) > 0), "non-negative codes increase with value"
+
+
+def test_e4m3_encode_nearest_even_and_saturating():
+    g = np.random.Generator(np.random.PCG64(17))
+    x = np.concatenate([g.uniform(-448, 448, 4000), g.standard_normal(4000) * 0.01,
+                        g.uniform(-2, 2, 4000)]).astype(np.float32)
+    enc = np.array([codec.e4m3_encode(v) for v in x], np.uint8)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(enc, ref)
+    # ties go to the even mantissa: 1.0625 lies halfway between 1.0 (0x38) and
+    # 1.125 (0x39); 1.1875 halfway between 1.125 and 1.25 (0x3A)
+    assert codec.e4m3_encode(1.0625) == 0x38 and codec.e4m3_encode(1.1875) == 0x3A
+    assert codec.e4m3_encode(-1.0625) == 0xB8
+    # halfway between the two smallest subnormals (2^-9 and 2^-8): to 2^-8 (code 2)
+    assert codec.e4m3_encode(1.5 * 2.0 ** -9) == 0x02
+    # beyond the largest finite value: saturate (no infinities in E4M3)
+    for v, c in ((448.0, 0x7E), (460.0, 0x7E), (500.0, 0x7E), (1e30, 0x7E), (-1e30, 0xFE)):
+        assert codec.e4m3_encode(v) == c
+
+
+def test_e4m3_dq_group_extremes_error_bound_and_shared_mean():
+    """Each group with b > 0 holds +-448 at its farthest constant; every
+    restored constant is within half an E4M3 step of its true value (relative
+    2^-4 in the normal range, 2^-10 absolute among subnormals) scaled by b,
+    plus binary32 rounding; mu is the INT8 reading's mu."""
+    a = np.abs(synthetic.normal_f32(256 * 40 + 77, 0.02, 23))
+    q, b, mu = codec.double_quant(a, fmt="e4m3")
+    q8, b8, mu8 = codec.double_quant(a, fmt="int8")
+    assert np.float32(mu) == np.float32(mu8)
+    assert q.dtype == np.uint8 and b.size == b8.size
+    for g in range(b.size):
+        grp = q[g * 256:(g + 1) * 256]
+        assert b[g] > 0 and np.any((grp & 0x7F) == 0x7E)
+    ah = codec.dq_restore(q, b, mu, fmt="e4m3").astype(np.float64)
+    r = (a.astype(np.float64) - float(mu)) / np.repeat(b.astype(np.float64), 256)[:a.size]
+    half_step = np.where(np.abs(r) >= 2.0 ** -6, np.abs(r) * 2.0 ** -4, 2.0 ** -10)
+    bound = np.repeat(b.astype(np.float64), 256)[:a.size] * (half_step + 1e-6) + 2.0 ** -22 * np.abs(a)
+    assert np.all(np.abs(ah - a) <= bound)
+
+
+def test_e4m3_dq_degenerate_group_and_dequant_format():
+    a = np.full(300, np.float32(0.25))                        # all equal -> b == 0 -> code 0
+    q, b, mu = codec.double_quant(a, fmt="e4m3")
+    assert np.all(q == 0) and np.all(b == 0) and mu == np.float32(0.25)
+    # dequant reads the E4M3 codes through the same restore as dq_restore
+    w = synthetic.normal_f32((64 * 600,), 0.02, 29)
+    codes, absmax = codec.quantize(w)
+    q, b, mu = codec.double_quant(absmax, fmt="e4m3")
+    ah = codec.dq_restore(q, b, mu, fmt="e4m3")
+    full = codec.dequant(codes, w.size, qabs=q, scale=b, mu=mu, fmt="e4m3")
+    plain = codec.dequant(codes, w.size, absmax=ah)
+    assert np.array_equal(full, plain)
