@@ -25,10 +25,12 @@ STATUS_NAMES = {0: "QLN_OK", 1: "QLN_ERR_NULL", 2: "QLN_ERR_SHAPE", 3: "QLN_ERR_
 OP_DOUBLE_QUANT, OP_LINEAR_FWD, OP_LINEAR_BWD = 1, 2, 3
 
 #: Every symbol include/qlora_nf4.h declares.
-EXPORTS = ("nf4_quantize", "nf4_quantize_ex", "nf4_double_quant", "nf4_double_quant_noalloc", "nf4_dequant",
+EXPORTS = ("nf4_quantize", "nf4_quantize_ex", "nf4_double_quant", "nf4_double_quant_ex", "nf4_double_quant_noalloc",
+           "nf4_dequant",
            "nf4_dequant_flat", "qlora_linear_fwd", "qlora_linear_bwd", "qln_workspace_bytes", "qln_codebook",
            "qln_status_str", "qln_version", "qln_launch_count")
 DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
+DQ_FORMATS = {"int8": 0, "e4m3": 1}
 
 
 class QLNError(RuntimeError):
@@ -40,7 +42,7 @@ class QLNError(RuntimeError):
 class CNF4Weight(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p), ("qabs", ctypes.c_void_p),
                 ("dq_scale", ctypes.c_void_p), ("dq_mean", ctypes.c_void_p), ("rows", ctypes.c_int64),
-                ("cols", ctypes.c_int64)]
+                ("cols", ctypes.c_int64), ("dq_format", ctypes.c_int32)]
 
 
 _lib = None
@@ -59,6 +61,7 @@ def lib():
             "nf4_quantize": ([P, I64, P, P, P], I32),
             "nf4_quantize_ex": ([P, I32, I64, P, P, P], I32),
             "nf4_double_quant": ([P, I64, P, P, P, P, SZ, P], I32),
+            "nf4_double_quant_ex": ([P, I64, I32, P, P, P, P, SZ, P], I32),
             "nf4_double_quant_noalloc": ([P, I64, P, P, P, P], I32),
             "nf4_dequant": ([WP, P, P], I32),
             "nf4_dequant_flat": ([WP, I64, P, P], I32),
@@ -140,12 +143,14 @@ class NF4Weight:
     qabs: Optional[torch.Tensor] = None    # int8 [nb]
     dq_scale: Optional[torch.Tensor] = None
     dq_mean: Optional[torch.Tensor] = None
+    dq_format: str = "int8"                # how qabs is stored: "int8" or "e4m3"
 
     def c_struct(self) -> CNF4Weight:
         return CNF4Weight(self.codes.data_ptr(), self.absmax.data_ptr() if self.absmax is not None else None,
                           self.qabs.data_ptr() if self.qabs is not None else None,
                           self.dq_scale.data_ptr() if self.dq_scale is not None else None,
-                          self.dq_mean.data_ptr() if self.dq_mean is not None else None, self.rows, self.cols)
+                          self.dq_mean.data_ptr() if self.dq_mean is not None else None, self.rows, self.cols,
+                          DQ_FORMATS[self.dq_format])
 
 
 _DTYPES = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
@@ -172,12 +177,15 @@ def nf4_quantize(W: torch.Tensor, codes: Optional[torch.Tensor] = None, absmax: 
     return codes, absmax
 
 
-def nf4_double_quant(absmax: torch.Tensor, qabs=None, dq_scale=None, dq_mean=None, ws=None):
-    """fp32 absmax [nb] -> (qabs int8 [nb], dq_scale fp32 [ceil(nb/256)], dq_mean fp32 [1])."""
+def nf4_double_quant(absmax: torch.Tensor, qabs=None, dq_scale=None, dq_mean=None, ws=None, fmt: str = "int8"):
+    """fp32 absmax [nb] -> (qabs [nb], dq_scale fp32 [ceil(nb/256)], dq_mean fp32 [1]).
+
+    fmt "int8": qabs int8 (nf4_double_quant); "e4m3": qabs uint8 E4M3 codes
+    (nf4_double_quant_ex) -- set NF4Weight.dq_format to match."""
     nb = absmax.numel()
     dev = absmax.device
     if qabs is None:
-        qabs = torch.empty(nb, dtype=torch.int8, device=dev)
+        qabs = torch.empty(nb, dtype=torch.int8 if fmt == "int8" else torch.uint8, device=dev)
     if dq_scale is None:
         dq_scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
     if dq_mean is None:
@@ -185,8 +193,13 @@ def nf4_double_quant(absmax: torch.Tensor, qabs=None, dq_scale=None, dq_mean=Non
     if ws is None:
         ws = alloc_workspace(workspace_bytes(OP_DOUBLE_QUANT, nb), dev)
     _need_cuda(absmax, qabs, dq_scale, dq_mean, ws)
-    _check("nf4_double_quant", lib().nf4_double_quant(_p(absmax), nb, _p(qabs), _p(dq_scale), _p(dq_mean), _p(ws),
-                                                      ws.numel(), _stream()))
+    if fmt == "int8":
+        _check("nf4_double_quant", lib().nf4_double_quant(_p(absmax), nb, _p(qabs), _p(dq_scale), _p(dq_mean),
+                                                          _p(ws), ws.numel(), _stream()))
+    else:
+        _check("nf4_double_quant_ex", lib().nf4_double_quant_ex(_p(absmax), nb, DQ_FORMATS[fmt], _p(qabs),
+                                                                _p(dq_scale), _p(dq_mean), _p(ws), ws.numel(),
+                                                                _stream()))
     return qabs, dq_scale, dq_mean
 
 
@@ -200,13 +213,15 @@ def nf4_double_quant_noalloc(absmax: torch.Tensor, qabs, dq_scale, dq_mean):
     return qabs, dq_scale, dq_mean
 
 
-def quantize_weight(W: torch.Tensor, double_quant: bool = True, ws=None) -> NF4Weight:
-    """nf4_quantize (+ nf4_double_quant) of a [rows][cols] fp32 weight."""
+def quantize_weight(W: torch.Tensor, double_quant: bool = True, ws=None, dq_format: str = "int8") -> NF4Weight:
+    """nf4_quantize (+ nf4_double_quant in the given 8-bit format) of a
+    [rows][cols] weight (fp32, bf16 or fp16)."""
     rows, cols = W.shape
     codes, absmax = nf4_quantize(W)
     w = NF4Weight(codes=codes, rows=rows, cols=cols, absmax=absmax)
     if double_quant:
-        w.qabs, w.dq_scale, w.dq_mean = nf4_double_quant(absmax, ws=ws)
+        w.qabs, w.dq_scale, w.dq_mean = nf4_double_quant(absmax, ws=ws, fmt=dq_format)
+        w.dq_format = dq_format
     return w
 
 

@@ -99,6 +99,7 @@ qln_status check_weight(const qln_nf4_weight *w) {
         return QLN_ERR_NULL;
     }
     if (w->rows <= 0 || w->cols <= 0 || (w->cols % 64) != 0) return QLN_ERR_SHAPE;
+    if (w->dq_format != QLN_DQ_INT8 && w->dq_format != QLN_DQ_E4M3) return QLN_ERR_SHAPE;
     if (!aligned(w->codes, 16)) return QLN_ERR_ALIGN;
     if (w->absmax && !aligned(w->absmax, 4)) return QLN_ERR_ALIGN;
     if (w->dq_scale && !aligned(w->dq_scale, 4)) return QLN_ERR_ALIGN;
@@ -154,8 +155,10 @@ qln_status nf4_quantize_ex(const void *W, int32_t dtype, int64_t numel, uint8_t 
     return from_cuda(qln::launch_nf4_quantize(W, dtype, numel, codes, absmax, (cudaStream_t)stream, sms));
 }
 
-qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale, float *dq_mean,
-                            void *ws, size_t ws_bytes, void *stream) {
+qln_status nf4_double_quant_ex(const float *absmax, int64_t nb, int32_t dq_format, void *qabs_v, float *dq_scale,
+                               float *dq_mean, void *ws, size_t ws_bytes, void *stream) {
+    int8_t *qabs = static_cast<int8_t *>(qabs_v);
+    if (dq_format != QLN_DQ_INT8 && dq_format != QLN_DQ_E4M3) return QLN_ERR_SHAPE;
     if (!absmax || !qabs || !dq_scale || !dq_mean || !ws) return QLN_ERR_NULL;
     if (nb <= 0 || nb > qln::dq_max_blocks()) return QLN_ERR_SHAPE;
     if (!aligned(absmax, 16) || !aligned(qabs, 4) || !aligned(dq_scale, 4) || !aligned(dq_mean, 4))
@@ -165,7 +168,13 @@ qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float
     int sms = 0;
     qln_status s = check_device(&sms);
     if (s != QLN_OK) return s;
-    return from_cuda(qln::launch_nf4_double_quant(absmax, nb, qabs, dq_scale, dq_mean, ws, (cudaStream_t)stream));
+    return from_cuda(qln::launch_nf4_double_quant(absmax, nb, qabs, dq_scale, dq_mean, ws, dq_format == QLN_DQ_E4M3,
+                                                     (cudaStream_t)stream));
+}
+
+qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale, float *dq_mean,
+                            void *ws, size_t ws_bytes, void *stream) {
+    return nf4_double_quant_ex(absmax, nb, QLN_DQ_INT8, qabs, dq_scale, dq_mean, ws, ws_bytes, stream);
 }
 
 qln_status nf4_double_quant_noalloc(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale,
@@ -199,6 +208,7 @@ qln_status nf4_dequant_flat(const qln_nf4_weight *w, int64_t numel, uint16_t *ou
         return QLN_ERR_NULL;
     }
     if (numel <= 0) return QLN_ERR_SHAPE;
+    if (w->dq_format != QLN_DQ_INT8 && w->dq_format != QLN_DQ_E4M3) return QLN_ERR_SHAPE;
     if (!aligned(w->codes, 16) || !aligned(out, 16)) return QLN_ERR_ALIGN;
     if (w->absmax && !aligned(w->absmax, 4)) return QLN_ERR_ALIGN;
     if (w->dq_scale && !aligned(w->dq_scale, 4)) return QLN_ERR_ALIGN;

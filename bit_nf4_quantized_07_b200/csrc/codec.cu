@@ -485,7 +485,8 @@ constexpr int kDqThreads = 256;
 __global__ void __launch_bounds__(kDqThreads) dq_quant_kernel(const float *__restrict__ a, int64_t nb,
                                                               const double *__restrict__ partial, int np,
                                                               int P, int8_t *__restrict__ qabs,
-                                                              float *__restrict__ scale, float *__restrict__ mu_out) {
+                                                              float *__restrict__ scale, float *__restrict__ mu_out,
+                                                              bool e4m3) {
     __shared__ double slice[kDqThreads / 32];
     __shared__ float mu_s;
     pdl_wait();
@@ -535,14 +536,18 @@ __global__ void __launch_bounds__(kDqThreads) dq_quant_kernel(const float *__res
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const float b = __fdiv_rn(m, 127.0f);
+    const float b = __fdiv_rn(m, e4m3 ? 448.0f : 127.0f);  // 448: the largest E4M3 value
     if (lane == 0) scale[g] = b;
     uint32_t w[2] = {0u, 0u};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        int r = 0;
-        if (b != 0.f) r = (int)fminf(fmaxf(rintf(__fdiv_rn(d[i], b)), -127.f), 127.f);
-        w[i >> 2] |= ((uint32_t)(r & 0xff)) << (8 * (i & 3));
+        uint32_t r = 0;
+        if (b != 0.f) {
+            const float x = __fdiv_rn(d[i], b);
+            r = e4m3 ? (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3)  // nearest-even, saturating
+                     : (uint32_t)((int)fminf(fmaxf(rintf(x), -127.f), 127.f) & 0xff);
+        }
+        w[i >> 2] |= (r & 0xffu) << (8 * (i & 3));
     }
     if (j0 + 8 <= nb) {
         *reinterpret_cast<uint32_t *>(qabs + j0) = w[0];
@@ -575,7 +580,7 @@ int64_t dq_max_blocks() { return kMeanMaxBlocks; }
 
 // K2 then K3, each launched as a programmatic dependent of the kernel before it.
 static cudaError_t launch_dq_pair(const float *absmax, int64_t nb, double *partial, int8_t *qabs, float *scale,
-                                  float *mu, cudaStream_t st) {
+                                  float *mu, bool e4m3, cudaStream_t st) {
     const int NG = dq_groups_per_thread(nb);
     const int np = (int)dq_partial_count(nb);
     int P = 8;
@@ -593,13 +598,13 @@ static cudaError_t launch_dq_pair(const float *absmax, int64_t nb, double *parti
     const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
     const int64_t grid = (ng + (kDqThreads / 32) - 1) / (kDqThreads / 32);
     return launch_pdl(dq_quant_kernel, dim3((unsigned)grid), dim3(kDqThreads), 0, st, absmax, nb,
-                      (const double *)partial, np, P, qabs, scale, mu);
+                      (const double *)partial, np, P, qabs, scale, mu, e4m3);
 }
 
 cudaError_t launch_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,
-                                    void *ws, cudaStream_t st) {
+                                    void *ws, bool e4m3, cudaStream_t st) {
     double *partial = reinterpret_cast<double *>(reinterpret_cast<char *>(ws) + 256);
-    return launch_dq_pair(absmax, nb, partial, qabs, scale, mu, st);
+    return launch_dq_pair(absmax, nb, partial, qabs, scale, mu, e4m3, st);
 }
 
 // ===========================================================================
@@ -645,7 +650,7 @@ cudaError_t launch_nf4_double_quant_static(const float *absmax, int64_t nb, int8
     double *partial = nullptr;
     cudaError_t e = dq_static_partials(&partial);
     if (e != cudaSuccess) return e;
-    return launch_dq_pair(absmax, nb, partial, qabs, scale, mu, st);
+    return launch_dq_pair(absmax, nb, partial, qabs, scale, mu, false, st);
 }
 
 // ===========================================================================
@@ -671,7 +676,7 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4 *__restric
                                                           const int8_t *__restrict__ qabs,
                                                           const float *__restrict__ scale,
                                                           const float *__restrict__ mu_p, int64_t nchunks,
-                                                          uint4 *__restrict__ out) {
+                                                          uint4 *__restrict__ out, bool e4m3) {
     __shared__ __align__(16) uint4 stage[8][128];  // per warp 2 KB
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     uint4 *buf = stage[wib];
@@ -697,7 +702,7 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4 *__restric
     fetch(ch + nwarps, d1);
     for (; ch < nchunks; ch += nwarps) {
         fetch(ch + 2 * nwarps, d2);
-        const float ah = qabs ? dq_restore(d0.q, d0.v, mu) : d0.v;
+        const float ah = qabs ? dq_restore((uint32_t)d0.q, d0.v, mu, e4m3) : d0.v;
         const NF4Table t = nf4_table(ah);
         // piece w of lane l (bytes 64 l + 16 w of the chunk) sits at slot 4 l + ((w + l/2) & 3)
         const int rot = lane >> 1;
@@ -723,11 +728,12 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4 *__restric
 __global__ void nf4_dequant_tail_kernel(const uint4 *__restrict__ codes128, const float *__restrict__ absmax,
                                         const int8_t *__restrict__ qabs, const float *__restrict__ scale,
                                         const float *__restrict__ mu_p, int64_t g0, int64_t ng,
-                                        uint4 *__restrict__ out) {
+                                        uint4 *__restrict__ out, bool e4m3) {
     const int64_t k = threadIdx.x;
     if (k >= ng) return;
     const int64_t i = g0 + k, j = i >> 1;
-    const float ah = qabs ? dq_restore(__ldg(qabs + j), __ldg(scale + (j >> 8)), __ldg(mu_p)) : __ldg(absmax + j);
+    const float ah = qabs ? dq_restore((uint32_t)__ldg(qabs + j), __ldg(scale + (j >> 8)), __ldg(mu_p), e4m3)
+                          : __ldg(absmax + j);
     const NF4Table t = nf4_table(ah);
     const uint4 cw = __ldg(codes128 + i);
     out[4 * i + 0] = nf4_decode8(cw.x, t);
@@ -740,11 +746,12 @@ __global__ void nf4_dequant_tail_kernel(const uint4 *__restrict__ codes128, cons
 __global__ void nf4_dequant_elem_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ absmax,
                                         const int8_t *__restrict__ qabs, const float *__restrict__ scale,
                                         const float *__restrict__ mu_p, int64_t e0, int64_t numel,
-                                        uint16_t *__restrict__ out) {
+                                        uint16_t *__restrict__ out, bool e4m3) {
     const int64_t e = e0 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= numel) return;
     const int64_t j = e >> 6;
-    const float ah = qabs ? dq_restore(__ldg(qabs + j), __ldg(scale + (j >> 8)), __ldg(mu_p)) : __ldg(absmax + j);
+    const float ah = qabs ? dq_restore((uint32_t)__ldg(qabs + j), __ldg(scale + (j >> 8)), __ldg(mu_p), e4m3)
+                          : __ldg(absmax + j);
     const uint32_t byte = __ldg(codes + (e >> 1));
     const int q = (e & 1) ? (int)(byte & 15u) : (int)(byte >> 4);
     const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(ah, nf4_value(q)));
@@ -765,6 +772,7 @@ cudaError_t launch_nf4_dequant_flat(const qln_nf4_weight *w, int64_t numel, uint
 
 static cudaError_t launch_dequant_numel(const qln_nf4_weight *w, int64_t numel, uint16_t *out, cudaStream_t st,
                                         int num_sms) {
+    const bool e4m3 = w->dq_format == QLN_DQ_E4M3;
     const int64_t nchunks = numel / 1024;  // weights come in whole 64-blocks; chunks of 1024 + a tail below
     const int64_t tail = numel - nchunks * 1024;
     int64_t grid = (nchunks + 7) / 8;
@@ -774,7 +782,7 @@ static cudaError_t launch_dequant_numel(const qln_nf4_weight *w, int64_t numel, 
     if (nchunks > 0) {
         nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(w->codes), w->absmax,
                                                           w->qabs, w->dq_scale, w->dq_mean, nchunks,
-                                                          reinterpret_cast<uint4 *>(out));
+                                                          reinterpret_cast<uint4 *>(out), e4m3);
         note_launch();
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
@@ -783,14 +791,15 @@ static cudaError_t launch_dequant_numel(const qln_nf4_weight *w, int64_t numel, 
     if (whole > 0) {
         const int64_t g0 = nchunks * 32, ng = whole / 32;
         nf4_dequant_tail_kernel<<<1, 64, 0, st>>>(reinterpret_cast<const uint4 *>(w->codes), w->absmax, w->qabs,
-                                                   w->dq_scale, w->dq_mean, g0, ng, reinterpret_cast<uint4 *>(out));
+                                                   w->dq_scale, w->dq_mean, g0, ng, reinterpret_cast<uint4 *>(out),
+                                                   e4m3);
         note_launch();
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     if (tail > whole) {  // fewer than 32 weights: one thread each
         nf4_dequant_elem_kernel<<<1, 32, 0, st>>>(w->codes, w->absmax, w->qabs, w->dq_scale, w->dq_mean,
-                                                   nchunks * 1024 + whole, numel, out);
+                                                   nchunks * 1024 + whole, numel, out, e4m3);
         note_launch();
         return cudaGetLastError();
     }

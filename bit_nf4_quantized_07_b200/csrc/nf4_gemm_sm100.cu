@@ -64,6 +64,7 @@ struct Cfg {
 
 struct Params {
     const int8_t *qabs;
+    bool e4m3;  // qabs holds E4M3 codes (QLN_DQ_E4M3), else int8
     const float *absmax;
     const float *dq_scale;
     const float *dq_mean;
@@ -270,7 +271,7 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         for (int kt = 0; kt < nsteps; ++kt) {
             const int s = kt % S;
             const uint32_t ph = (uint32_t)(kt / S) & 1u;
-            const float ah = p.qabs ? dq_restore((int8_t)r0.q, r0.v, mu) : r0.v;
+            const float ah = p.qabs ? dq_restore((uint32_t)r0.q, r0.v, mu, p.e4m3) : r0.v;
             r0 = r1;
             r1 = fetch(kt + 2);
             if (!mbar_wait_bounded(empty(s), ph ^ 1u, abort_flag, kWaitLimitNs)) {
@@ -480,6 +481,7 @@ cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16
 
     Params p;
     p.qabs = w->qabs;
+    p.e4m3 = w->dq_format == QLN_DQ_E4M3;
     p.absmax = w->absmax;
     p.dq_scale = w->dq_scale;
     p.dq_mean = w->dq_mean;

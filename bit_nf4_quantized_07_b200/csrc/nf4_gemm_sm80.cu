@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(128) nf4_mma_gemm_kernel(const uint8_t *__rest
                                                            int64_t cols, const uint16_t *__restrict__ act, int64_t n,
                                                            const uint16_t *__restrict__ lact,
                                                            const uint16_t *__restrict__ lw, int r,
-                                                           uint16_t *__restrict__ out) {
+                                                           uint16_t *__restrict__ out, bool e4m3) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     SmemSm80 &S = *reinterpret_cast<SmemSm80 *>(smem_raw);
     const int rpad = (r + 15) & ~15;
@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(128) nf4_mma_gemm_kernel(const uint8_t *__rest
     auto block_const = [&](int kt) -> float {
         const int row = tid >> 1;
         const int64_t jb = (wtile_row0(kt) + row) * bpr + wtile_col0(kt) / 64;
-        if (qabs) return dq_restore(__ldg(qabs + jb), __ldg(dq_scale + (jb >> 8)), mu);
+        if (qabs) return dq_restore((uint32_t)__ldg(qabs + jb), __ldg(dq_scale + (jb >> 8)), mu, e4m3);
         return __ldg(absmax + jb);
     };
 
@@ -237,13 +237,15 @@ cudaError_t launch_nf4_mma_gemm(const qln_nf4_weight *w, bool trans, const uint1
         e = cudaFuncSetAttribute(nf4_mma_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         nf4_mma_gemm_kernel<true><<<grid, 128, smem, st>>>(w->codes, w->absmax, w->qabs, w->dq_scale, w->dq_mean,
-                                                          w->rows, w->cols, act, n, lact, lw, r, out);
+                                                          w->rows, w->cols, act, n, lact, lw, r, out,
+                                                          w->dq_format == QLN_DQ_E4M3);
         note_launch();
     } else {
         e = cudaFuncSetAttribute(nf4_mma_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         nf4_mma_gemm_kernel<false><<<grid, 128, smem, st>>>(w->codes, w->absmax, w->qabs, w->dq_scale, w->dq_mean,
-                                                           w->rows, w->cols, act, n, lact, lw, r, out);
+                                                           w->rows, w->cols, act, n, lact, lw, r, out,
+                                                          w->dq_format == QLN_DQ_E4M3);
         note_launch();
     }
     return cudaGetLastError();

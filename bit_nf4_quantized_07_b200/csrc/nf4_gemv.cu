@@ -76,6 +76,7 @@ constexpr uint64_t kDvWaitNs = 2000000000ull;  // bounded waits
 struct DvParams {
     const float *absmax;
     const int8_t *qabs;
+    bool e4m3;  // qabs holds E4M3 codes (QLN_DQ_E4M3), else int8
     const float *dq_scale;
     const float *dq_mean;
     int64_t rows, cols, KB, T;
@@ -361,7 +362,7 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
                         float ah[2];
     #pragma unroll
                         for (int h = 0; h < 2; ++h)
-                            ah[h] = dq ? dq_restore((int8_t)kc.raw[b][h], (kc.lo[h] + b >= 256) ? kc.sc[h][1] : kc.sc[h][0], mu)
+                            ah[h] = dq ? dq_restore(kc.raw[b][h], (kc.lo[h] + b >= 256) ? kc.sc[h][1] : kc.sc[h][0], mu, p.e4m3)
                                        : __uint_as_float(kc.raw[b][h]);
                         float tmp[NT][4];
     #pragma unroll
@@ -680,6 +681,7 @@ cudaError_t launch_nf4_gemv(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     DvParams p;
     p.absmax = w->absmax;
     p.qabs = w->qabs;
+    p.e4m3 = w->dq_format == QLN_DQ_E4M3;
     p.dq_scale = w->dq_scale;
     p.dq_mean = w->dq_mean;
     p.rows = w->rows;

@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -76,10 +78,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
+// The value of an OCP FP8 E4M3 code (exact in fp32): the hardware conversion
+// to half, then to float.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+    const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)(code & 0xffu), __NV_E4M3);
+    return __half2float(__half(h));
+}
+
 // doubleDequant of one block constant: ahat = fp32(mu + fp32(b * rhat)), the
 // product first, then the sum ("LoRA 与 QLoRA" section 2, reconstruction).
-__device__ __forceinline__ float dq_restore(int8_t rhat, float b, float mu) {
-    return __fadd_rn(mu, __fmul_rn(b, (float)rhat));
+// The low byte of `code` is rhat: an int8 (QLN_DQ_INT8) or an E4M3 code
+// (QLN_DQ_E4M3, the "8-bit floats" of deck card 4).
+__device__ __forceinline__ float dq_restore(uint32_t code, float b, float mu, bool e4m3) {
+    const float r = e4m3 ? e4m3_to_f32(code) : (float)(int8_t)(code & 0xffu);
+    return __fadd_rn(mu, __fmul_rn(b, r));
 }
 
 // ---------------------------------------------------------------------------

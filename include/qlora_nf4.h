@@ -78,6 +78,9 @@ typedef enum {
     QLN_ERR_INTERNAL = 8   /* device side: an internal consistency check failed*/
 } qln_status;
 
+/* Formats of the 8-bit double-quantized block constants (qabs). */
+enum { QLN_DQ_INT8 = 0, QLN_DQ_E4M3 = 1 };
+
 /* Element types of the weights given to nf4_quantize_ex. */
 enum { QLN_DTYPE_F32 = 0, QLN_DTYPE_BF16 = 1, QLN_DTYPE_F16 = 2 };
 
@@ -88,7 +91,10 @@ enum { QLN_OP_DOUBLE_QUANT = 1, QLN_OP_LINEAR_FWD = 2, QLN_OP_LINEAR_BWD = 3 };
  * are device pointers owned by the caller.  With qabs != NULL the weight is
  * double-quantized (qabs, dq_scale, dq_mean are used, absmax is ignored);
  * with qabs == NULL the plain fp32 absmax is used (bnb_4bit_use_double_quant
- * off).  cols must be a multiple of 64, so blocks never straddle rows. */
+ * off).  cols must be a multiple of 64, so blocks never straddle rows.
+ * dq_format says how qabs is stored: QLN_DQ_INT8 (0, signed int8, as written
+ * by nf4_double_quant) or QLN_DQ_E4M3 (1, OCP FP8 E4M3 codes, as written by
+ * nf4_double_quant_ex with that format); a zero-initialized struct is INT8. */
 typedef struct {
     const uint8_t *codes;
     const float *absmax;
@@ -97,6 +103,7 @@ typedef struct {
     const float *dq_mean;
     int64_t rows; /* dout */
     int64_t cols; /* din  */
+    int32_t dq_format;
 } qln_nf4_weight;
 
 /*
@@ -157,6 +164,22 @@ QLN_API qln_status nf4_quantize_ex(const void *W, int32_t dtype, int64_t numel, 
  */
 QLN_API qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale,
                             float *dq_mean, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * nf4_double_quant_ex -- nf4_double_quant with a choice of 8-bit format.
+ * The pages disagree on the 8-bit format of the quantized constants: deck
+ * "3 QLoRA Finetuning" card 4 says 8-bit floats, jjjymmm.cn "Double
+ * Quantization" says INT8.  dq_format QLN_DQ_INT8 is nf4_double_quant;
+ * QLN_DQ_E4M3 stores OCP FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, largest finite value 448, no infinities):
+ *   b_g = fp32(max|d_j| / 448), rhat_j = E4M3(fp32(d_j / b_g)) rounded to
+ *   nearest-even and saturated to +-448; code 0 when b_g == 0.
+ * mu is the same as for INT8.  Set qln_nf4_weight.dq_format to the same value
+ * when the result is used.  qabs [nb] bytes out; other arguments, workspace
+ * and errors as nf4_double_quant, plus QLN_ERR_SHAPE for an unknown format.
+ */
+QLN_API qln_status nf4_double_quant_ex(const float *absmax, int64_t nb, int32_t dq_format, void *qabs,
+                                       float *dq_scale, float *dq_mean, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * nf4_double_quant_noalloc -- nf4_double_quant without a caller workspace.

@@ -22,14 +22,15 @@ def f64(bits):
 class OracleWeight:
     """NF4 + DQ of a fp32 weight by the oracle, with W' as BF16 bits."""
 
-    def __init__(self, w: np.ndarray, double_quant: bool = True):
+    def __init__(self, w: np.ndarray, double_quant: bool = True, dq_format: str = "int8"):
         self.rows, self.cols = w.shape
         self.numel = w.size
         self.codes, self.absmax = codec.quantize(w)
         self.dq = double_quant
         if double_quant:
-            self.qabs, self.scale, self.mu = codec.double_quant(self.absmax)
-            self.wp_bits = codec.dequant(self.codes, self.numel, qabs=self.qabs, scale=self.scale, mu=self.mu)
+            self.qabs, self.scale, self.mu = codec.double_quant(self.absmax, fmt=dq_format)
+            self.wp_bits = codec.dequant(self.codes, self.numel, qabs=self.qabs, scale=self.scale, mu=self.mu,
+                                         fmt=dq_format)
         else:
             self.wp_bits = codec.dequant(self.codes, self.numel, absmax=self.absmax)
         self.wp_bits = self.wp_bits.reshape(self.rows, self.cols)

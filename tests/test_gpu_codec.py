@@ -200,3 +200,27 @@ def test_quantize16_matches_fp32_path_on_prefill_weight():
     c32, a32 = api.nf4_quantize(w.float())
     torch.cuda.synchronize()
     assert torch.equal(c16, c32) and torch.equal(a16, a32)
+
+
+@pytest.mark.parametrize("shape,seed", [((512, 512), 51), ((3, 320), 52), ((1000, 192), 53), ((11008, 4096), 54)])
+def test_e4m3_double_quant_and_dequant_bit_exact(shape, seed):
+    """The "8-bit floats" DQ format: E4M3 codes, group scales, mu and the BF16
+    dequant (tiled and flat) bit-exact against the oracle."""
+    w = synthetic.normal_f32(shape, 0.02, seed)
+    W = torch.from_numpy(w).cuda()
+    codes, absmax = api.nf4_quantize(W)
+    q, b, mu = api.nf4_double_quant(absmax, fmt="e4m3")
+    rows, cols = w.reshape(-1, 64).shape[0], 64
+    wq = api.NF4Weight(codes=codes, rows=rows, cols=cols, absmax=absmax, qabs=q, dq_scale=b, dq_mean=mu,
+                       dq_format="e4m3")
+    deq = api.nf4_dequant(wq)
+    flat = api.nf4_dequant_flat(wq, w.size)
+    torch.cuda.synchronize()
+    c_ref, a_ref = codec.quantize(w)
+    q_ref, b_ref, mu_ref = codec.double_quant(a_ref, fmt="e4m3")
+    assert np.array_equal(q.cpu().numpy(), q_ref), f"{np.sum(q.cpu().numpy() != q_ref)} E4M3 codes differ"
+    assert np.array_equal(b.cpu().numpy().view(np.uint32), b_ref.view(np.uint32))
+    assert np.float32(mu.item()).view(np.uint32) == np.float32(mu_ref).view(np.uint32)
+    ref = codec.dequant(c_ref, w.size, qabs=q_ref, scale=b_ref, mu=mu_ref, fmt="e4m3")
+    assert np.array_equal(dev_bf16_bits(deq).reshape(-1), ref)
+    assert np.array_equal(dev_bf16_bits(flat).reshape(-1), ref)

@@ -14,12 +14,12 @@ pytestmark = pytest.mark.gpu
 TOL = 2e-2
 
 
-def _gpu_weight(w, double_quant=True):
-    return api.quantize_weight(torch.from_numpy(w).cuda(), double_quant=double_quant)
+def _gpu_weight(w, double_quant=True, dq_format="int8"):
+    return api.quantize_weight(torch.from_numpy(w).cuda(), double_quant=double_quant, dq_format=dq_format)
 
 
-def _run(cfg, w, X, A, B, dY, double_quant=True, backward=True):
-    wq = _gpu_weight(w, double_quant)
+def _run(cfg, w, X, A, B, dY, double_quant=True, backward=True, dq_format="int8"):
+    wq = _gpu_weight(w, double_quant, dq_format)
     Xd, Ad, Bd = bf16_to_dev(X), bf16_to_dev(A), bf16_to_dev(B)
     Y, U = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s)
     out = {"Y": f64(dev_bf16_bits(Y)), "U": f64(dev_bf16_bits(U))}
@@ -202,3 +202,27 @@ def test_prefill_sampled():
 @pytest.mark.slow
 def test_large_sampled():
     _sampled(synthetic.LARGE)
+
+
+E4M3_SHAPES = [
+    synthetic.custom("e4m3_tc_512x768_n256_r16", 512, 768, 256, 16, s=2.0, index=31),    # tcgen05 path
+    synthetic.custom("e4m3_mma_256x320_n40_r8", 256, 320, 40, 8, s=1.0, index=32),       # mma.sync path
+    synthetic.custom("e4m3_dec_1024x2048_n4_r16", 1024, 2048, 4, 16, s=2.0, index=33),  # decode kernel
+]
+
+
+@pytest.mark.parametrize("cfg", E4M3_SHAPES, ids=lambda c: c.name)
+def test_linear_with_e4m3_double_quant(cfg):
+    """Every fused path restores the block constants from E4M3 codes when the
+    weight says so: forward and backward within the tolerance of the oracle's
+    E4M3-restored W'."""
+    w, X, A, B, dY = workload(cfg)
+    ow = OracleWeight(w, dq_format="e4m3")
+    got = _run(cfg, w, X, A, B, dY, dq_format="e4m3")
+    Y, U = forward_ref(ow, X, A, B, cfg.s)
+    dX, dA, dB = backward_ref(ow, X, A, B, cfg.s, dY)
+    _compare("U", got["U"], U)
+    _compare("Y", got["Y"], Y)
+    _compare("dX", got["dX"], dX)
+    _compare("dA", got["dA"], dA)
+    _compare("dB", got["dB"], dB)
