@@ -12,10 +12,11 @@ Parity status:
              invariants), double quantization (closed-form bit count, exact
              mean, error bound), dequant (definition + BF16 rounding vs torch),
              forward/backward (finite differences, special cases, merged-weight
-             identity, rank bound).
+             identity, rank bound), the E4M3 codec (torch's float8_e4m3fn),
+             AdamW (torch.optim.AdamW and closed forms).
   unpinned - the exact 8-bit format of the double-quantized constants (the
              pages disagree: 8-bit floats vs INT8; INT8 absmax is our reading),
              the nibble order inside a byte, and the codebook offset delta
              beyond the 4-decimal window the printed table fixes.
 """
-from . import codec, linear  # noqa: F401
+from . import adamw, codec, linear  # noqa: F401
