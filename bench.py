@@ -410,8 +410,6 @@ def run_ours(args):
     Y = torch.empty(cfg.n, cfg.dout, dtype=torch.bfloat16, device=dev)
     U = torch.empty(cfg.n, cfg.r, dtype=torch.bfloat16, device=dev)
     dX = torch.empty(cfg.n, cfg.din, dtype=torch.bfloat16, device=dev)
-    dA = torch.empty(cfg.r, cfg.din, dtype=torch.float32, device=dev)
-    dB = torch.empty(cfg.dout, cfg.r, dtype=torch.float32, device=dev)
     ws_dq = api.alloc_workspace(api.workspace_bytes(api.OP_DOUBLE_QUANT, nb), dev)
     ws_f = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_FWD, cfg.dout, cfg.din, cfg.n, cfg.r), dev)
     ws_b = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_BWD, cfg.dout, cfg.din, cfg.n, cfg.r), dev)
@@ -420,6 +418,23 @@ def run_ours(args):
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
+    # AdamW state of the LoRA factors (one per input set): fp32 masters, the
+    # 32-bit moments and the device step counter; the update writes the BF16
+    # copies the next forward of that set reads.
+    # A and B live in one flat buffer per set (masters, BF16 copies, moments),
+    # and dA/dB in one flat gradient buffer, so one launch updates both.
+    nA, nB = cfg.r * cfg.din, cfg.dout * cfg.r
+    grad_flat = torch.empty(nA + nB, dtype=torch.float32, device=dev)
+    dA, dB = grad_flat[:nA].view(cfg.r, cfg.din), grad_flat[nA:].view(cfg.dout, cfg.r)
+    opt = []
+    for k, (W_, X_, A, B, dY_) in enumerate(sets):
+        flat16 = torch.cat([A.reshape(-1), B.reshape(-1)])
+        A16, B16 = flat16[:nA].view(cfg.r, cfg.din), flat16[nA:].view(cfg.dout, cfg.r)
+        sets[k] = (W_, X_, A16, B16, dY_)
+        opt.append({"p32": flat16.float(), "p16": flat16, "m": torch.zeros(nA + nB, device=dev),
+                    "v": torch.zeros(nA + nB, device=dev), "t": torch.zeros(1, dtype=torch.int64, device=dev)})
+    ADAMW = dict(lr=1e-4, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0)
+
     def step_body(i):
         W, X, A, B, dYs = sets[i % NSETS]
         api.nf4_quantize(W, codes, absmax)
@@ -427,6 +442,12 @@ def run_ours(args):
         api.nf4_dequant(wq, wdq)
         api.qlora_linear_fwd(wq, X, A, B, cfg.s, Y=Y, U_out=U, ws=ws_f)
         api.qlora_linear_bwd(wq, X, A, B, cfg.s, dYs, U=U, dX=dX, dA=dA, dB=dB, ws=ws_b)
+
+    def optim_body(i, p16=None):
+        o = opt[i % NSETS]
+        o["t"].add_(1)
+        api.adamw_step(o["p32"], grad_flat, o["m"], o["v"], o["t"], param_bf16=o["p16"] if p16 is None else p16,
+                       **ADAMW)
 
     # Rows of the step, for the per-row times.
     rows = {
@@ -438,6 +459,7 @@ def run_ours(args):
         "fwd": lambda i: api.qlora_linear_fwd(wq, *sets[i % NSETS][1:4], cfg.s, Y=Y, U_out=U, ws=ws_f),
         "bwd": lambda i: api.qlora_linear_bwd(wq, *sets[i % NSETS][1:4], cfg.s, sets[i % NSETS][4], U=U, dX=dX,
                                               dA=dA, dB=dB, ws=ws_b),
+        "adamw": lambda i: optim_body(i),
     }
 
     # The step runs as a CUDA graph (one per input set): the library's calls
@@ -465,16 +487,25 @@ def run_ours(args):
     if not args.no_graph:
         graphs = []
         for i in range(NSETS):
-            graphs.append(capture(lambda i=i: step_body(i)))
-            launches_per_step = captured[0]
+            g_main = capture(lambda i=i: step_body(i))
+            n_main = captured[0]
+            g_opt = capture(lambda i=i: optim_body(i))
+            graphs.append((g_main, g_opt))
+            launches_per_step = n_main + captured[0]
 
     def step(i):
+        # codec + forward + backward, the data-parallel all-reduce of dA/dB
+        # (N > 1), then the optimizer
         if graphs is not None:
-            graphs[i % NSETS].replay()
+            graphs[i % NSETS][0].replay()
         else:
             step_body(i)
         if world > 1:
             dp.allreduce_adapter_grads(dA, dB)
+        if graphs is not None:
+            graphs[i % NSETS][1].replay()
+        else:
+            optim_body(i)
 
     for i in range(args.warmup):
         step(i)
@@ -522,7 +553,9 @@ def run_ours(args):
     # End to end through the C ABI with host buffers: copies inside the timed region.
     W, X, A, B, dYs = sets[0]
     hW, hX, hA, hB, hdY = (t.cpu().pin_memory() for t in (W, X, A, B, dYs))
-    dW, dXi, dAi, dBi, ddY = (torch.empty_like(t) for t in (W, X, A, B, dYs))
+    dW, dXi, ddY = (torch.empty_like(t) for t in (W, X, dYs))
+    dflat16 = torch.empty(nA + nB, dtype=torch.bfloat16, device=dev)
+    dAi, dBi = dflat16[:nA].view(cfg.r, cfg.din), dflat16[nA:].view(cfg.dout, cfg.r)
     oY, odX, odA, odB = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (Y, dX, dA, dB))
 
     def e2e_step():
@@ -535,6 +568,7 @@ def run_ours(args):
         api.qlora_linear_bwd(wq, dXi, dAi, dBi, cfg.s, ddY, U=U, dX=dX, dA=dA, dB=dB, ws=ws_b)
         if world > 1:
             dp.allreduce_adapter_grads(dA, dB)
+        optim_body(0, p16=dflat16)
         for h, d in ((oY, Y), (odX, dX), (odA, dA), (odB, dB)):
             h.copy_(d, non_blocking=True)
 
@@ -572,6 +606,7 @@ def run_ours(args):
         "dequant_GBs": numel * db / (sec["dequant"] * 1e-3) / 1e9,
         "fwd_TFLOPs": fwd_tflops,
         "bwd_TFLOPs": cfg.bwd_flops() / (sec["bwd"] * 1e-3) / 1e12,
+        "adamw_GBs": 30 * cfg.r * (cfg.din + cfg.dout) / (sec["adamw"] * 1e-3) / 1e9,
         "ms": sec,
         "hbm_peak_GBs": peaks["hbm_gbs"],
     }
@@ -582,7 +617,8 @@ def run_ours(args):
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
            "config": {"workload": cfg.name, "dout": cfg.dout, "din": cfg.din, "n": cfg.n, "r": cfg.r, "s": cfg.s,
                       "global_batch": cfg.n * world, "parallelism": f"dp{world}",
-                      "step": "nf4_quantize+nf4_double_quant+nf4_dequant+qlora_linear_fwd+qlora_linear_bwd",
+                      "step": "nf4_quantize+nf4_double_quant+nf4_dequant+qlora_linear_fwd+qlora_linear_bwd"
+                              "+qln_adamw_step(A,B)",
                       "l2": "3 rotating input sets (W0 fp32 alone 180 MB > 126 MB L2)",
                       "timing": "python-enqueued steps" if args.no_graph else
                       "CUDA graph replay per step (one graph per input set)"},

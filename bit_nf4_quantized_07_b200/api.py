@@ -28,7 +28,7 @@ OP_DOUBLE_QUANT, OP_LINEAR_FWD, OP_LINEAR_BWD = 1, 2, 3
 EXPORTS = ("nf4_quantize", "nf4_quantize_ex", "nf4_double_quant", "nf4_double_quant_ex", "nf4_double_quant_noalloc",
            "nf4_dequant",
            "nf4_dequant_flat", "qlora_linear_fwd", "qlora_linear_bwd", "qln_workspace_bytes", "qln_codebook",
-           "qln_status_str", "qln_version", "qln_launch_count")
+           "qln_status_str", "qln_version", "qln_launch_count", "qln_adamw_step")
 DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
 DQ_FORMATS = {"int8": 0, "e4m3": 1}
 
@@ -37,6 +37,14 @@ class QLNError(RuntimeError):
     def __init__(self, fn, status):
         super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
         self.status = status
+
+
+class CAdamWConfig(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("weight_decay", ctypes.c_float)]
+
+
+ADAMW_PAGE_IN, ADAMW_PAGE_OUT = 1, 2
 
 
 class CNF4Weight(ctypes.Structure):
@@ -72,6 +80,7 @@ def lib():
             "qln_status_str": ([I32], ctypes.c_char_p),
             "qln_version": ([], I32),
             "qln_launch_count": ([], ctypes.c_uint64),
+            "qln_adamw_step": ([P, P, P, P, P, I64, ctypes.POINTER(CAdamWConfig), P, I32, P], I32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -287,3 +296,15 @@ def qlora_linear_bwd(w: NF4Weight, X, A, B, s: float, dY, U=None, dX=None, dA=No
 def device_status(ws: torch.Tensor) -> int:
     """The int32 status word at workspace offset 0 (synchronises the current stream)."""
     return int(ws[:4].view(torch.int32).item())
+
+
+def adamw_step(param: torch.Tensor, grad: torch.Tensor, m: torch.Tensor, v: torch.Tensor, step: torch.Tensor,
+               lr: float, betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.0,
+               param_bf16: Optional[torch.Tensor] = None, flags: int = 0):
+    """One AdamW update of an fp32 master tensor in place (qln_adamw_step).
+    ``step`` is a device int64 tensor holding the step number t >= 1."""
+    n = param.numel()
+    _need_cuda(param, grad, m, v, step, param_bf16)
+    cfg = CAdamWConfig(lr, betas[0], betas[1], eps, weight_decay)
+    _check("qln_adamw_step", lib().qln_adamw_step(_p(param), _p(grad), _p(m), _p(v), _p(param_bf16), n,
+                                                  ctypes.byref(cfg), _p(step), flags, _stream()))

@@ -200,6 +200,19 @@ qln_status nf4_dequant(const qln_nf4_weight *w, uint16_t *out, void *stream) {
     return from_cuda(qln::launch_nf4_dequant(w, out, (cudaStream_t)stream, sms));
 }
 
+qln_status qln_adamw_step(float *param, const float *grad, float *m, float *v, uint16_t *param_bf16, int64_t n,
+                          const qln_adamw_config *cfg, const int64_t *step, int32_t flags, void *stream) {
+    if (!param || !grad || !m || !v || !cfg || !step) return QLN_ERR_NULL;
+    if (n <= 0) return QLN_ERR_SHAPE;
+    if (!aligned(param, 16) || !aligned(grad, 16) || !aligned(m, 16) || !aligned(v, 16)) return QLN_ERR_ALIGN;
+    if (param_bf16 && !aligned(param_bf16, 8)) return QLN_ERR_ALIGN;
+    int sms = 0;
+    qln_status s = check_device(&sms);
+    if (s != QLN_OK) return s;
+    return from_cuda(qln::launch_adamw(param, grad, m, v, param_bf16, n, cfg->lr, cfg->beta1, cfg->beta2, cfg->eps,
+                                       cfg->weight_decay, step, flags, (cudaStream_t)stream, sms));
+}
+
 qln_status nf4_dequant_flat(const qln_nf4_weight *w, int64_t numel, uint16_t *out, void *stream) {
     if (!w || !w->codes || !out) return QLN_ERR_NULL;
     if (w->qabs) {

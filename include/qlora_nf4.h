@@ -276,6 +276,49 @@ QLN_API qln_status qlora_linear_bwd(const qln_nf4_weight *w, const uint16_t *X, 
                             const uint16_t *dY, const uint16_t *U, uint16_t *dX, float *dA,
                             float *dB, void *ws, size_t ws_bytes, void *stream);
 
+/* AdamW hyper-parameters (fp32, as the update computes in fp32). */
+typedef struct {
+    float lr;
+    float beta1;
+    float beta2;
+    float eps;
+    float weight_decay;
+} qln_adamw_config;
+
+/* qln_adamw_step flags. */
+enum { QLN_ADAMW_PAGE_IN = 1, QLN_ADAMW_PAGE_OUT = 2 };
+
+/*
+ * qln_adamw_step -- one AdamW update of a LoRA factor (the paged optimizer).
+ * Defined by: deck "3 QLoRA Finetuning" card 5 (paged optimizers keep the
+ * optimizer states in NVIDIA unified memory, paged out to CPU RAM when the
+ * GPU runs short and paged back for the update) and card 1 (only the adapter
+ * parameters are updated); "LoRA 与 QLoRA" QLoRA usage notes
+ * (paged_adamw_32bit).  The pages do not write AdamW out; this is the
+ * published one (Loshchilov & Hutter, ICLR 2019), decay first:
+ *   m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2;  p = p (1 - lr wd);
+ *   p = p - (lr / (1 - b1^t)) m / (sqrt(v / (1 - b2^t)) + eps),
+ * evaluated in fp32 per element (bias corrections in binary64).
+ *   param  [n] fp32 in/out: the factor's master copy (A or B, flattened).
+ *   grad   [n] fp32 in: its gradient (dA or dB from qlora_linear_bwd).
+ *   m, v   [n] fp32 in/out: the 32-bit AdamW states, zero before step 1.
+ *   param_bf16 [n] bf16 out or NULL: RN(param) after the update, the copy the
+ *          forward reads.
+ *   step   device pointer to the step number t >= 1 being taken (read by the
+ *          kernel, so a captured CUDA graph can be replayed step after step
+ *          while the caller increments it).
+ *   flags  QLN_ADAMW_PAGE_IN: operands that live in managed memory are
+ *          prefetched to the current device before the update;
+ *          QLN_ADAMW_PAGE_OUT: m and v, if managed, are prefetched back to
+ *          host RAM after it.  Memory of any other kind is left alone.
+ * Any pointer may be managed (cudaMallocManaged) or device memory.
+ * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE if n <= 0; QLN_ERR_ALIGN if param,
+ * grad, m or v is not 16-byte aligned (param_bf16: 8-byte).
+ */
+QLN_API qln_status qln_adamw_step(float *param, const float *grad, float *m, float *v, uint16_t *param_bf16,
+                                  int64_t n, const qln_adamw_config *cfg, const int64_t *step, int32_t flags,
+                                  void *stream);
+
 /* Device workspace, in bytes, that `op` needs for these sizes (nb for
  * QLN_OP_DOUBLE_QUANT is passed as `rows`).  Returns 0 for an unknown op. */
 QLN_API size_t qln_workspace_bytes(int32_t op, int64_t rows, int64_t cols, int64_t n, int32_t r);

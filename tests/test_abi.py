@@ -135,3 +135,15 @@ def test_linear_argument_errors(L):
     bwd = L.qlora_linear_bwd(ctypes.byref(w), A16, 4, A16, A16, 16, 1.0, A16, None, A16, A16, A16, ws, need - 1,
                              None)
     assert bwd == 4
+
+
+def test_adamw_argument_errors(L):
+    cfg = api.CAdamWConfig(1e-3, 0.9, 0.999, 1e-8, 0.0)
+    c = ctypes.byref(cfg)
+    assert L.qln_adamw_step(None, A16, A16, A16, None, 64, c, A16, 0, None) == 1
+    assert L.qln_adamw_step(A16, A16, A16, A16, None, 64, None, A16, 0, None) == 1
+    assert L.qln_adamw_step(A16, A16, A16, A16, None, 64, c, None, 0, None) == 1
+    assert L.qln_adamw_step(A16, A16, A16, A16, None, 0, c, A16, 0, None) == 2
+    assert L.qln_adamw_step(A4, A16, A16, A16, None, 64, c, A16, 0, None) == 3
+    assert L.qln_adamw_step(A16, A16, A16, A4, None, 64, c, A16, 0, None) == 3
+    assert L.qln_adamw_step(A16, A16, A16, A16, A4, 64, c, A16, 0, None) == 3
