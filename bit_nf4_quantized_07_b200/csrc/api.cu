@@ -255,10 +255,10 @@ qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
         // the status word itself, so no memset precedes it
         return from_cuda(qln::launch_nf4_gemv(w, X, n, A, B, r, s, Y, U_out, ws, cs));
     }
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
-    if (e != cudaSuccess) return QLN_ERR_CUDA;
-    // U = X A^T (and s*U for the adapter MMA), then the fused weight GEMM.
-    e = qln::launch_lora_down(X, n, w->cols, A, false, r, s, U, sU, pU, cs, kSplitTargetSms);
+    // U = X A^T (and s*U for the adapter MMA; its first kernel also clears the
+    // status word), then the fused weight GEMM.  No memset between kernels:
+    // the launches chain by programmatic dependent launch.
+    cudaError_t e = qln::launch_lora_down(X, n, w->cols, A, false, r, s, U, sU, pU, cs, kSplitTargetSms, status);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     e = fused_gemm(w, false, X, n, sU, B, r, Y, status, cs, sms);
     return from_cuda(e);
@@ -286,17 +286,18 @@ qln_status qlora_linear_bwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     float *pGU = reinterpret_cast<float *>(wsb + L.pGU);
     float *pA = reinterpret_cast<float *>(wsb + L.pA);
     float *pB = reinterpret_cast<float *>(wsb + L.pB);
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
-    if (e != cudaSuccess) return QLN_ERR_CUDA;
+    cudaError_t e;
+    int *reset = status;  // the call's first kernel clears the status word
     if (!U) {
         uint16_t *Uw = reinterpret_cast<uint16_t *>(wsb + L.U);
-        e = qln::launch_lora_down(X, n, w->cols, A, false, r, s, Uw, nullptr, pGU, cs, kSplitTargetSms);
+        e = qln::launch_lora_down(X, n, w->cols, A, false, r, s, Uw, nullptr, pGU, cs, kSplitTargetSms, reset);
         if (e != cudaSuccess) return QLN_ERR_CUDA;
         U = Uw;
+        reset = nullptr;
     }
     // G = dY B (and s*G; B read as stored, [dout][r]), dX = dY W' + (s G) A,
     // dA = s G^T X (the transpose of s X^T G), dB = s dY^T U.
-    e = qln::launch_lora_down(dY, n, w->rows, B, true, r, s, G, sG, pGU, cs, kSplitTargetSms);
+    e = qln::launch_lora_down(dY, n, w->rows, B, true, r, s, G, sG, pGU, cs, kSplitTargetSms, reset);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     e = fused_gemm(w, true, dY, n, sG, A, r, dX, status, cs, sms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;

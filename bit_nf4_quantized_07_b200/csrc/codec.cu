@@ -678,6 +678,8 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4 *__restric
                                                           const float *__restrict__ mu_p, int64_t nchunks,
                                                           uint4 *__restrict__ out, bool e4m3) {
     __shared__ __align__(16) uint4 stage[8][128];  // per warp 2 KB
+    pdl_wait();  // the weight may come from the previous kernel on the stream
+    pdl_trigger();
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     uint4 *buf = stage[wib];
     const float mu = qabs ? __ldg(mu_p) : 0.f;
@@ -780,11 +782,9 @@ static cudaError_t launch_dequant_numel(const qln_nf4_weight *w, int64_t numel, 
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
     if (nchunks > 0) {
-        nf4_dequant_kernel<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(w->codes), w->absmax,
-                                                          w->qabs, w->dq_scale, w->dq_mean, nchunks,
-                                                          reinterpret_cast<uint4 *>(out), e4m3);
-        note_launch();
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_pdl(nf4_dequant_kernel, dim3((unsigned)grid), dim3(256), 0, st,
+                                   reinterpret_cast<const uint4 *>(w->codes), w->absmax, w->qabs, w->dq_scale,
+                                   w->dq_mean, nchunks, reinterpret_cast<uint4 *>(out), e4m3);
         if (e != cudaSuccess) return e;
     }
     const int64_t whole = (tail / 32) * 32;  // 32-weight groups of the tail: 16-byte stores

@@ -43,8 +43,11 @@ constexpr int kDnLd = 72;  // padded row (bf16) of the staged tiles
 template <int NT, bool WKM>
 __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t *__restrict__ in, int64_t n, int64_t K,
                                                         const uint16_t *__restrict__ wt, int r, int cps,
-                                                        float *__restrict__ partial) {
+                                                        float *__restrict__ partial, int *status_reset) {
     extern __shared__ __align__(16) uint16_t dsm[];
+    pdl_wait();  // every input may come from the previous kernel on the stream
+    pdl_trigger();
+    if (status_reset && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status_reset = QLN_OK;
     constexpr int WR = NT * 8;                              // adapter rows staged (r rounded up to 8)
     constexpr int WKLD = WR + 8;                            // padded row of a K-major wt stage
     constexpr int STAGE = 64 * kDnLd + (WKM ? 64 * WKLD : WR * kDnLd);  // elements per stage
@@ -169,6 +172,8 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t *__restri
 
 __global__ void lora_fold_kernel(const float *__restrict__ partial, int splits, int64_t total, float scale,
                                  uint16_t *__restrict__ out, uint16_t *__restrict__ out_scaled) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
         const float v = fold_splits(partial + i, total, splits);
@@ -198,7 +203,7 @@ size_t lora_down_partial_bytes(int64_t n, int64_t K, int r, int num_sms) {
 
 template <int NT, bool WKM>
 static cudaError_t launch_down_t(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, int splits,
-                                 int cps, float *partial, cudaStream_t st) {
+                                 int cps, float *partial, int *status_reset, cudaStream_t st) {
     const size_t smem =
         (size_t)kDnStages * (64 * kDnLd + (WKM ? 64 * (NT * 8 + 8) : NT * 8 * kDnLd)) * sizeof(uint16_t);
     auto kern = lora_down_kernel<NT, WKM>;
@@ -207,51 +212,48 @@ static cudaError_t launch_down_t(const uint16_t *in, int64_t n, int64_t K, const
         if (e != cudaSuccess) return e;
     }
     dim3 grid((unsigned)((n + 63) / 64), (unsigned)splits);
-    kern<<<grid, 128, smem, st>>>(in, n, K, wt, r, cps, partial);
-    note_launch();
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(128), smem, st, in, n, K, wt, r, cps, partial, status_reset);
 }
 
 template <bool WKM>
 static cudaError_t launch_down_nt(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, int splits,
-                                  int cps, float *partial, cudaStream_t st) {
+                                  int cps, float *partial, int *sr, cudaStream_t st) {
     const int nt = (r + 7) / 8;
     cudaError_t e;
     switch (nt) {
-        case 1: e = launch_down_t<1, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 2: e = launch_down_t<2, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 3: e = launch_down_t<3, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 4: e = launch_down_t<4, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 5: e = launch_down_t<5, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 6: e = launch_down_t<6, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 7: e = launch_down_t<7, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 8: e = launch_down_t<8, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 9: e = launch_down_t<9, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 10: e = launch_down_t<10, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 11: e = launch_down_t<11, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 12: e = launch_down_t<12, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 13: e = launch_down_t<13, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 14: e = launch_down_t<14, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        case 15: e = launch_down_t<15, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
-        default: e = launch_down_t<16, WKM>(in, n, K, wt, r, splits, cps, partial, st); break;
+        case 1: e = launch_down_t<1, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 2: e = launch_down_t<2, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 3: e = launch_down_t<3, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 4: e = launch_down_t<4, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 5: e = launch_down_t<5, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 6: e = launch_down_t<6, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 7: e = launch_down_t<7, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 8: e = launch_down_t<8, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 9: e = launch_down_t<9, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 10: e = launch_down_t<10, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 11: e = launch_down_t<11, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 12: e = launch_down_t<12, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 13: e = launch_down_t<13, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 14: e = launch_down_t<14, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        case 15: e = launch_down_t<15, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
+        default: e = launch_down_t<16, WKM>(in, n, K, wt, r, splits, cps, partial, sr, st); break;
     }
     return e;
 }
 
 cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, bool wt_kmajor, int r,
                              float scale, uint16_t *out, uint16_t *out_scaled, float *partial, cudaStream_t st,
-                             int num_sms) {
+                             int num_sms, int *status_reset) {
     int splits, cps;
     lora_down_plan(n, K, num_sms, &splits, &cps);
-    cudaError_t e = wt_kmajor ? launch_down_nt<true>(in, n, K, wt, r, splits, cps, partial, st)
-                              : launch_down_nt<false>(in, n, K, wt, r, splits, cps, partial, st);
+    cudaError_t e = wt_kmajor ? launch_down_nt<true>(in, n, K, wt, r, splits, cps, partial, status_reset, st)
+                              : launch_down_nt<false>(in, n, K, wt, r, splits, cps, partial, status_reset, st);
     if (e != cudaSuccess) return e;
     const int64_t total = n * r;
     int64_t blocks = (total + 255) / 256;
     if (blocks > 4096) blocks = 4096;
-    lora_fold_kernel<<<(unsigned)blocks, 256, 0, st>>>(partial, splits, total, scale, out, out_scaled);
-    note_launch();
-    return cudaGetLastError();
+    return launch_pdl(lora_fold_kernel, dim3((unsigned)blocks), dim3(256), 0, st, (const float *)partial, splits, total,
+                      scale, out, out_scaled);
 }
 
 // ===========================================================================
@@ -273,6 +275,8 @@ __global__ void __launch_bounds__(128) tn_skinny_kernel(const uint16_t *__restri
     extern __shared__ __align__(16) uint16_t sk[];
     uint16_t *Ps = sk;                                   // [stages][32][kSkPad]
     uint16_t *Qs = sk + kSkStages * kSkBK * kSkPad;      // [stages][32][QLD]
+    pdl_wait();  // P and Q may come from the previous kernel on the stream
+    pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int64_t m0 = (int64_t)blockIdx.x * kSkBM;
@@ -374,6 +378,8 @@ __global__ void __launch_bounds__(128) tn_skinny_kernel(const uint16_t *__restri
 
 __global__ void tn_skinny_fold_kernel(const float *__restrict__ partials, int splits, int64_t M, int R, float scale,
                                       bool transpose, float *__restrict__ C) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t MR = M * R;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < MR; i += stride) {
@@ -410,9 +416,8 @@ static cudaError_t launch_skinny_t(const uint16_t *P, const uint16_t *Q, int64_t
         if (e != cudaSuccess) return e;
     }
     dim3 grid((unsigned)((M + kSkBM - 1) / kSkBM), (unsigned)splits);
-    kern<<<grid, 128, smem, st>>>(P, Q, n, M, R, scale, transpose, C, splits > 1 ? partials : nullptr);
-    note_launch();
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(128), smem, st, P, Q, n, M, R, scale, transpose, C,
+                      splits > 1 ? partials : nullptr);
 }
 
 cudaError_t launch_tn_skinny(const uint16_t *P, const uint16_t *Q, int64_t n, int64_t M, int R, float scale,
@@ -440,9 +445,8 @@ cudaError_t launch_tn_skinny(const uint16_t *P, const uint16_t *Q, int64_t n, in
     const int64_t MR = M * R;
     int64_t blocks = (MR + 255) / 256;
     if (blocks > 4096) blocks = 4096;
-    tn_skinny_fold_kernel<<<(unsigned)blocks, 256, 0, st>>>(partials, splits, M, R, scale, transpose, C);
-    note_launch();
-    return cudaGetLastError();
+    return launch_pdl(tn_skinny_fold_kernel, dim3((unsigned)blocks), dim3(256), 0, st, (const float *)partials, splits,
+                      M, R, scale, transpose, C);
 }
 
 }  // namespace qln

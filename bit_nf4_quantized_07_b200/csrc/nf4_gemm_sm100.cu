@@ -127,6 +127,10 @@ nf4_tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_d = *tmem_slot;
+    // Barriers, descriptors and TMEM are set up while the previous kernel on
+    // the stream finishes; every global access comes after this wait.
+    qln::pdl_wait();
+    qln::pdl_trigger();
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -440,9 +444,8 @@ static cudaError_t launch_t(const CUtensorMap &m_codes, const CUtensorMap &m_act
     cudaError_t e = cudaFuncSetAttribute(nf4_tc_gemm_kernel<TRANS, MT, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    nf4_tc_gemm_kernel<TRANS, MT, NT><<<grid, C::kThreads, C::kSmemBytes, st>>>(m_codes, m_act, m_lw, m_lact, p);
-    note_launch();
-    return cudaGetLastError();
+    return qln::launch_pdl(nf4_tc_gemm_kernel<TRANS, MT, NT>, grid, dim3(C::kThreads), (size_t)C::kSmemBytes, st,
+                           m_codes, m_act, m_lw, m_lact, p);
 }
 
 }  // namespace tc

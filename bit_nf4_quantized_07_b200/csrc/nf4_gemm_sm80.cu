@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(128) nf4_mma_gemm_kernel(const uint8_t *__rest
                                                            const uint16_t *__restrict__ lw, int r,
                                                            uint16_t *__restrict__ out, bool e4m3) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
+    pdl_wait();  // every input may come from the previous kernel on the stream
+    pdl_trigger();
     SmemSm80 &S = *reinterpret_cast<SmemSm80 *>(smem_raw);
     const int rpad = (r + 15) & ~15;
     // adapter tiles after the main structure
@@ -232,23 +234,12 @@ cudaError_t launch_nf4_mma_gemm(const qln_nf4_weight *w, bool trans, const uint1
     const size_t smem = sizeof(SmemSm80) + (size_t)ls_rows * ls_ld * 2 + (size_t)64 * (rpad + 8) * 2;
     const int64_t M = trans ? w->cols : w->rows;
     dim3 grid((unsigned)((n + kSmBN - 1) / kSmBN), (unsigned)(M / kSmBM));
-    cudaError_t e;
-    if (trans) {
-        e = cudaFuncSetAttribute(nf4_mma_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        nf4_mma_gemm_kernel<true><<<grid, 128, smem, st>>>(w->codes, w->absmax, w->qabs, w->dq_scale, w->dq_mean,
-                                                          w->rows, w->cols, act, n, lact, lw, r, out,
-                                                          w->dq_format == QLN_DQ_E4M3);
-        note_launch();
-    } else {
-        e = cudaFuncSetAttribute(nf4_mma_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        nf4_mma_gemm_kernel<false><<<grid, 128, smem, st>>>(w->codes, w->absmax, w->qabs, w->dq_scale, w->dq_mean,
-                                                           w->rows, w->cols, act, n, lact, lw, r, out,
-                                                          w->dq_format == QLN_DQ_E4M3);
-        note_launch();
-    }
-    return cudaGetLastError();
+    const bool e4m3 = w->dq_format == QLN_DQ_E4M3;
+    auto kern = trans ? nf4_mma_gemm_kernel<true> : nf4_mma_gemm_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, grid, dim3(128), smem, st, w->codes, w->absmax, w->qabs, w->dq_scale, w->dq_mean, w->rows,
+                      w->cols, act, n, lact, lw, r, out, e4m3);
 }
 
 }  // namespace qln

@@ -165,6 +165,8 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
     int *ucount = reinterpret_cast<int *>(reinterpret_cast<char *>(p.status) + kWsUCountOffset);
     int *uflag = reinterpret_cast<int *>(reinterpret_cast<char *>(p.status) + kWsUFlagOffset);
     int *udone = reinterpret_cast<int *>(reinterpret_cast<char *>(p.status) + kWsDoneOffset);
+    pdl_wait();  // X, the weight and the workspace may all be touched by the previous kernel on the stream
+    pdl_trigger();
 
     // ---- U CTAs: U = X A^T, once for the grid ------------------------------------
     if ((int)blockIdx.x >= p.Q * S) {
@@ -658,17 +660,19 @@ static cudaError_t launch_dv(DvParams p, const qln_nf4_weight *w, cudaStream_t s
     p.off_su = L.off_su;
     p.off_bar = L.off_bar;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)L.S;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // the kernel waits before any global access
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3((unsigned)((bestQ + kDvUParts / L.S) * L.S));
     cfg.blockDim = dim3(kDvThreads);
     cfg.dynamicSmemBytes = L.smem;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, nf4_decode_fwd_kernel<NT>, tm, p);
     note_launch();
     if (e != cudaSuccess) return e;

@@ -60,7 +60,7 @@ int64_t dq_max_blocks();
 //   wt_kmajor: wt is stored [K][r] instead (out[t][j] = sum_k in[t][k] * wt[k][j]).
 cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, bool wt_kmajor, int r,
                              float scale, uint16_t *out, uint16_t *out_scaled, float *partial, cudaStream_t st,
-                             int num_sms);
+                             int num_sms, int *status_reset = nullptr);
 size_t lora_down_partial_bytes(int64_t n, int64_t K, int r, int num_sms);
 //   C = scale * P^T Q with Q [n][R] narrow (R <= 128): C[m][j], or C[j][m] with
 //   `transpose`; fp32 partials of tn_skinny_partials_bytes(M, R, splits).
