@@ -41,7 +41,8 @@ __device__ __forceinline__ void adamw_elem(float &p, float g, float &m, float &v
 __global__ void __launch_bounds__(256) adamw_kernel(const AdamWArgs a) {
     pdl_wait();
     // bias corrections of step t, in binary64 once per thread
-    const double t = (double)*a.step;
+    const int64_t tv = *a.step;
+    const double t = (double)(tv < 1 ? 1 : tv);  // a step below 1 is taken as the first
     const double bc1 = 1.0 - pow((double)a.b1, t), bc2 = 1.0 - pow((double)a.b2, t);
     const float step_size = (float)((double)a.lr / bc1);
     const float inv_sqrt_bc2 = (float)(1.0 / sqrt(bc2));

@@ -307,10 +307,13 @@ enum { QLN_ADAMW_PAGE_IN = 1, QLN_ADAMW_PAGE_OUT = 2 };
  *   step   device pointer to the step number t >= 1 being taken (read by the
  *          kernel, so a captured CUDA graph can be replayed step after step
  *          while the caller increments it).
+ *   step   values below 1 are taken as 1.
  *   flags  QLN_ADAMW_PAGE_IN: operands that live in managed memory are
  *          prefetched to the current device before the update;
  *          QLN_ADAMW_PAGE_OUT: m and v, if managed, are prefetched back to
- *          host RAM after it.  Memory of any other kind is left alone.
+ *          host RAM after it.  Memory of any other kind is left alone.  The
+ *          prefetches are stream operations of their own: pass 0 while the
+ *          stream is being captured into a CUDA graph.
  * Any pointer may be managed (cudaMallocManaged) or device memory.
  * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE if n <= 0; QLN_ERR_ALIGN if param,
  * grad, m or v is not 16-byte aligned (param_bf16: 8-byte).
