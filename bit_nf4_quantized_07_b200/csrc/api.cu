@@ -83,8 +83,8 @@ BwdWs bwd_layout(int64_t rows, int64_t cols, int64_t n, int r) {
     L.pGU = L.U + nr;
     const size_t pg = qln::lora_down_partial_bytes(n, rows, r, kSplitTargetSms);
     const size_t pu = qln::lora_down_partial_bytes(n, cols, r, kSplitTargetSms);
-    L.splitA = qln::tn_skinny_splits(n, cols, kSplitTargetSms);
-    L.splitB = qln::tn_skinny_splits(n, rows, kSplitTargetSms);
+    L.splitA = qln::tn_skinny_splits(n, cols, r, kSplitTargetSms);
+    L.splitB = qln::tn_skinny_splits(n, rows, r, kSplitTargetSms);
     L.pA = L.pGU + round256(pg > pu ? pg : pu);
     L.pB = L.pA + round256(qln::tn_skinny_partials_bytes(cols, r, L.splitA));
     L.total = L.pB + round256(qln::tn_skinny_partials_bytes(rows, r, L.splitB));

@@ -182,11 +182,29 @@ __global__ void lora_fold_kernel(const float *__restrict__ partial, int splits, 
     }
 }
 
-// Splits of the K range: about 6 CTAs per SM, at least 4 chunks of 64 per CTA.
-void lora_down_plan(int64_t n, int64_t K, int num_sms, int *splits, int *cps) {
+// CTAs of `smem` bytes that fit on one SM (228 KB per SM, 1 KB reserved per
+// CTA, at most 16 CTAs of 128 threads); registers are not the limit for these
+// kernels at their launch bounds.
+static int64_t ctas_per_sm(size_t smem) {
+    const int64_t k = (int64_t)(228 * 1024) / (int64_t)(smem + 1024);
+    return k < 1 ? 1 : (k > 16 ? 16 : k);
+}
+
+static size_t lora_down_smem(int r, bool wkm) {
+    const int nt = (r + 7) / 8;
+    return (size_t)kDnStages * (64 * kDnLd + (wkm ? 64 * (nt * 8 + 8) : nt * 8 * kDnLd)) * sizeof(uint16_t);
+}
+
+// Splits of the K range: one full wave of resident CTAs (rounded down, so the
+// grid never spills into a second, mostly empty wave), at least 4 chunks of
+// 64 per CTA.  The staged-tile size is the same for both operand layouts to
+// within a few KB, so the plan uses the larger (k-major) one.
+void lora_down_plan(int64_t n, int64_t K, int r, int num_sms, int *splits, int *cps) {
     const int64_t nch = K / 64;
     const int64_t ttiles = (n + 63) / 64;
-    int64_t sp = (6 * (int64_t)num_sms + ttiles - 1) / ttiles;
+    const size_t smem = lora_down_smem(r, true) > lora_down_smem(r, false) ? lora_down_smem(r, true)
+                                                                            : lora_down_smem(r, false);
+    int64_t sp = ctas_per_sm(smem) * (int64_t)num_sms / ttiles;
     const int64_t maxsp = nch / 4 > 0 ? nch / 4 : 1;
     if (sp > maxsp) sp = maxsp;
     if (sp < 1) sp = 1;
@@ -197,15 +215,14 @@ void lora_down_plan(int64_t n, int64_t K, int num_sms, int *splits, int *cps) {
 
 size_t lora_down_partial_bytes(int64_t n, int64_t K, int r, int num_sms) {
     int sp, cps;
-    lora_down_plan(n, K, num_sms, &sp, &cps);
+    lora_down_plan(n, K, r, num_sms, &sp, &cps);
     return (size_t)sp * (size_t)n * (size_t)r * sizeof(float);
 }
 
 template <int NT, bool WKM>
 static cudaError_t launch_down_t(const uint16_t *in, int64_t n, int64_t K, const uint16_t *wt, int r, int splits,
                                  int cps, float *partial, int *status_reset, cudaStream_t st) {
-    const size_t smem =
-        (size_t)kDnStages * (64 * kDnLd + (WKM ? 64 * (NT * 8 + 8) : NT * 8 * kDnLd)) * sizeof(uint16_t);
+    const size_t smem = lora_down_smem(NT * 8, WKM);
     auto kern = lora_down_kernel<NT, WKM>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -245,7 +262,7 @@ cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uin
                              float scale, uint16_t *out, uint16_t *out_scaled, float *partial, cudaStream_t st,
                              int num_sms, int *status_reset) {
     int splits, cps;
-    lora_down_plan(n, K, num_sms, &splits, &cps);
+    lora_down_plan(n, K, r, num_sms, &splits, &cps);
     cudaError_t e = wt_kmajor ? launch_down_nt<true>(in, n, K, wt, r, splits, cps, partial, status_reset, st)
                               : launch_down_nt<false>(in, n, K, wt, r, splits, cps, partial, status_reset, st);
     if (e != cudaSuccess) return e;
@@ -391,10 +408,14 @@ __global__ void tn_skinny_fold_kernel(const float *__restrict__ partials, int sp
 }
 
 // About 6 CTAs per SM, each with at least 4 token steps (128 tokens).
-int tn_skinny_splits(int64_t n, int64_t M, int num_sms) {
+// Token splits: one full wave of resident CTAs (rounded down), at least 4
+// token steps per CTA, at most 64 splits.
+int tn_skinny_splits(int64_t n, int64_t M, int R, int num_sms) {
     const int64_t tiles = (M + kSkBM - 1) / kSkBM;
     const int64_t steps = (n + kSkBK - 1) / kSkBK;
-    int64_t splits = (6 * (int64_t)num_sms + tiles - 1) / tiles;
+    const int ntj = (R + 7) / 8;
+    const size_t smem = (size_t)kSkStages * kSkBK * (kSkPad + ntj * 8 + 8) * sizeof(uint16_t);
+    int64_t splits = ctas_per_sm(smem) * (int64_t)num_sms / tiles;
     const int64_t maxsp = steps / 4 > 0 ? steps / 4 : 1;
     if (splits > maxsp) splits = maxsp;
     if (splits > 64) splits = 64;

@@ -67,7 +67,7 @@ size_t lora_down_partial_bytes(int64_t n, int64_t K, int r, int num_sms);
 cudaError_t launch_tn_skinny(const uint16_t *P, const uint16_t *Q, int64_t n, int64_t M, int R, float scale,
                              bool transpose, float *C, float *partials, int splits, cudaStream_t st);
 size_t tn_skinny_partials_bytes(int64_t M, int R, int splits);
-int tn_skinny_splits(int64_t n, int64_t M, int num_sms);
+int tn_skinny_splits(int64_t n, int64_t M, int R, int num_sms);
 
 // nf4_gemm_sm80.cu: fused NF4 decode + legacy mma.sync GEMM (small n).
 //   trans = false: out[t][m] = bf16(sum_k act[t][k] W'[m][k] + sum_j lact[t][j] lw[m][j])   (forward)
