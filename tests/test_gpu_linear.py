@@ -226,3 +226,32 @@ def test_linear_with_e4m3_double_quant(cfg):
     _compare("dX", got["dX"], dX)
     _compare("dA", got["dA"], dA)
     _compare("dB", got["dB"], dB)
+
+
+def test_decode_wait_runs_out_reports_timeout_and_recovers():
+    """Failure detection without a GPU fault: a workspace whose U counter can
+    never reach its last arrival means the U-ready flag is never raised.  The
+    decode CTAs' bounded wait (2 s) runs out, the kernel records
+    QLN_ERR_TIMEOUT in the status word and finishes; its last CTA leaves the
+    counters at zero, so the next call on the same workspace is correct."""
+    import time
+    cfg = synthetic.custom("timeout_1024x2048_n4_r16", 1024, 2048, 4, 16, s=2.0, index=41)
+    w, X, A, B, dY = workload(cfg)
+    wq = _gpu_weight(w)
+    Xd, Ad, Bd = bf16_to_dev(X), bf16_to_dev(A), bf16_to_dev(B)
+    ws = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_FWD, cfg.dout, cfg.din, cfg.n, cfg.r))
+    ws[64:68].view(torch.int32).fill_(1 << 20)  # the U arrival counter (header offset 64)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s, ws=ws)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert api.device_status(ws) == 7, "QLN_ERR_TIMEOUT expected"
+    assert 1.0 < elapsed < 60.0, elapsed
+    assert int(ws[64:68].view(torch.int32).item()) == 0 and int(ws[128:132].view(torch.int32).item()) == 0
+    Y, U = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s, ws=ws)
+    torch.cuda.synchronize()
+    assert api.device_status(ws) == 0
+    Yr, Ur = forward_ref(OracleWeight(w), X, A, B, cfg.s)
+    _compare("U", f64(dev_bf16_bits(U)), Ur)
+    _compare("Y", f64(dev_bf16_bits(Y)), Yr)
