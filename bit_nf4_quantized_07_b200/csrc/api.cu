@@ -169,7 +169,7 @@ qln_status nf4_double_quant_ex(const float *absmax, int64_t nb, int32_t dq_forma
     qln_status s = check_device(&sms);
     if (s != QLN_OK) return s;
     return from_cuda(qln::launch_nf4_double_quant(absmax, nb, qabs, dq_scale, dq_mean, ws, dq_format == QLN_DQ_E4M3,
-                                                     (cudaStream_t)stream));
+                                                     (cudaStream_t)stream, sms));
 }
 
 qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale, float *dq_mean,

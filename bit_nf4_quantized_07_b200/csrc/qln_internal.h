@@ -39,7 +39,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 cudaError_t launch_nf4_quantize(const void *W, int dtype, int64_t numel, uint8_t *codes, float *absmax,
                                 cudaStream_t st, int num_sms);
 cudaError_t launch_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,
-                                    void *ws, bool e4m3, cudaStream_t st);
+                                    void *ws, bool e4m3, cudaStream_t st, int num_sms);
 cudaError_t launch_nf4_dequant(const qln_nf4_weight *w, uint16_t *out, cudaStream_t st, int num_sms);
 cudaError_t launch_adamw(float *p, const float *g, float *m, float *v, uint16_t *p_bf16, int64_t n, float lr,
                          float b1, float b2, float eps, float wd, const int64_t *step, int flags, cudaStream_t st,

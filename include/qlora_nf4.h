@@ -45,8 +45,9 @@
  *   give up after a bounded number of polls and write QLN_ERR_TIMEOUT into the
  *   int32 status word at byte offset 0 of the workspace; read it after the
  *   stream has synchronised (0 = QLN_OK).  Each workspace call clears it.
- * - Bytes 4..255 of a workspace hold counters of the decode-sized forward
- *   (n <= 32).  Zero-fill a workspace once before its first use; every call
+ * - Bytes 4..255 of a workspace hold counters (the decode-sized forward,
+ *   n <= 32; the single-launch double quantization's grid barrier).
+ *   Zero-fill a workspace once before its first use; every call
  *   leaves the counters at zero again (also across CUDA graph replays).  After
  *   a call that reported QLN_ERR_TIMEOUT, zero the first 256 bytes again.
  */
@@ -157,7 +158,11 @@ QLN_API qln_status nf4_quantize_ex(const void *W, int32_t dtype, int64_t numel, 
  * b_g == 0.  The last group may be partial.
  *   ws / ws_bytes: device scratch of at least
  *   qln_workspace_bytes(QLN_OP_DOUBLE_QUANT, nb, 0, 0, 0) bytes, 256-byte
- *   aligned; contents on entry are ignored.
+ *   aligned.  Its first 256 bytes are a header: a status word at offset 0
+ *   (QLN_OK, or QLN_ERR_TIMEOUT when a bounded device wait gave up) and
+ *   counters of the single-launch path's grid barrier.  Zero the header once
+ *   before the first call; every call leaves it zeroed again (zero it anew
+ *   after a QLN_ERR_TIMEOUT).  The rest is scratch.
  * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE if nb <= 0 or nb > 2^25 (numel above
  * 2^31); QLN_ERR_WORKSPACE; QLN_ERR_ALIGN if absmax is not 16-byte aligned or
  * ws is not 256-byte aligned.

@@ -224,3 +224,66 @@ def test_e4m3_double_quant_and_dequant_bit_exact(shape, seed):
     ref = codec.dequant(c_ref, w.size, qabs=q_ref, scale=b_ref, mu=mu_ref, fmt="e4m3")
     assert np.array_equal(dev_bf16_bits(deq).reshape(-1), ref)
     assert np.array_equal(dev_bf16_bits(flat).reshape(-1), ref)
+
+
+@pytest.mark.parametrize("fmt", ["int8", "e4m3"])
+def test_single_launch_dq_repeats_replays_and_leaves_header_zeroed(fmt):
+    """The single-launch double quantization (grid barrier on counters in the
+    workspace header): back-to-back calls and CUDA graph replays on one
+    workspace give the oracle's bits, and every call leaves the header at zero."""
+    w = synthetic.normal_f32((11008 // 4, 4096), 0.02, 61)
+    codes, absmax = api.nf4_quantize(torch.from_numpy(w).cuda())
+    nb = absmax.numel()
+    ws = api.alloc_workspace(api.workspace_bytes(api.OP_DOUBLE_QUANT, nb))
+    _, a_ref = codec.quantize(w)
+    q_ref, b_ref, mu_ref = codec.double_quant(a_ref, fmt=fmt)
+    q, b, mu = api.nf4_double_quant(absmax, ws=ws, fmt=fmt)
+    for _ in range(3):
+        q2, b2, mu2 = api.nf4_double_quant(absmax, ws=ws, fmt=fmt)
+        assert torch.equal(q, q2) and torch.equal(b, b2) and torch.equal(mu, mu2)
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy().view(np.uint8), q_ref.view(np.uint8))
+    assert np.array_equal(b.cpu().numpy().view(np.uint32), b_ref.view(np.uint32))
+    assert np.float32(mu.item()).view(np.uint32) == np.float32(mu_ref).view(np.uint32)
+    assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        api.nf4_double_quant(absmax, q, b, mu, ws=ws, fmt=fmt)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(3):
+            api.nf4_double_quant(absmax, q, b, mu, ws=ws, fmt=fmt)
+    q.zero_()
+    for _ in range(4):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy().view(np.uint8), q_ref.view(np.uint8))
+    assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0
+
+
+def test_single_launch_dq_barrier_runs_out_and_reports_timeout():
+    """Failure detection without a GPU fault: an arrival counter that can
+    never reach the grid size makes every CTA's bounded barrier wait (2 s) run
+    out; the kernel records QLN_ERR_TIMEOUT and finishes.  With the header
+    zeroed again the next call is exact."""
+    import time
+    w = synthetic.normal_f32((1024, 4096), 0.02, 62)
+    codes, absmax = api.nf4_quantize(torch.from_numpy(w).cuda())
+    nb = absmax.numel()
+    ws = api.alloc_workspace(api.workspace_bytes(api.OP_DOUBLE_QUANT, nb))
+    ws[64:68].view(torch.int32).fill_(-(1 << 30))  # the barrier's arrival counter
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    api.nf4_double_quant(absmax, ws=ws)
+    torch.cuda.synchronize()
+    assert 1.0 < time.perf_counter() - t0 < 60.0
+    assert api.device_status(ws) == 7, "QLN_ERR_TIMEOUT expected"
+    ws[:256].zero_()
+    q, b, mu = api.nf4_double_quant(absmax, ws=ws)
+    torch.cuda.synchronize()
+    assert api.device_status(ws) == 0
+    q_ref, b_ref, mu_ref = codec.double_quant(codec.quantize(w)[1])
+    assert np.array_equal(q.cpu().numpy(), q_ref) and np.float32(mu.item()) == np.float32(mu_ref)
