@@ -147,3 +147,34 @@ def test_adamw_argument_errors(L):
     assert L.qln_adamw_step(A4, A16, A16, A16, None, 64, c, A16, 0, None) == 3
     assert L.qln_adamw_step(A16, A16, A16, A4, None, 64, c, A16, 0, None) == 3
     assert L.qln_adamw_step(A16, A16, A16, A16, A4, 64, c, A16, 0, None) == 3
+
+
+def test_quantize_ex_argument_errors(L):
+    assert L.nf4_quantize_ex(None, api.DTYPE_BF16, 65, A16, A16, None) == 1
+    assert L.nf4_quantize_ex(A16, api.DTYPE_BF16, 0, A16, A16, None) == 2
+    assert L.nf4_quantize_ex(A16, 7, 64, A16, A16, None) == 2                    # unknown element type
+    assert L.nf4_quantize_ex(A4, api.DTYPE_F16, 65, A16, A16, None) == 3
+    assert L.nf4_quantize_ex(A16, api.DTYPE_F32, 65, A4, A16, None) == 3
+    assert L.nf4_quantize_ex(A16, api.DTYPE_F32, 65, A16, P(0x10002), None) == 3
+
+
+def test_double_quant_ex_argument_errors(L):
+    ws = P(0x20000)
+    need = api.workspace_bytes(api.OP_DOUBLE_QUANT, 100)
+    assert L.nf4_double_quant_ex(None, 100, 0, A16, A16, A16, ws, need, None) == 1
+    assert L.nf4_double_quant_ex(A16, 100, 2, A16, A16, A16, ws, need, None) == 2   # unknown 8-bit format
+    assert L.nf4_double_quant_ex(A16, 0, 1, A16, A16, A16, ws, need, None) == 2
+    assert L.nf4_double_quant_ex(A16, 100, 1, A16, A16, A16, P(0x20010), need, None) == 3
+    assert L.nf4_double_quant_ex(A16, 100, 1, A16, A16, A16, ws, need - 1, None) == 4
+
+
+def test_dequant_flat_and_format_argument_errors(L):
+    out = A16
+    w = _w()
+    assert L.nf4_dequant_flat(None, 65, out, None) == 1
+    assert L.nf4_dequant_flat(ctypes.byref(w), 0, out, None) == 2
+    assert L.nf4_dequant_flat(ctypes.byref(w), 65, P(0x10002), None) == 3
+    bad = _w()
+    bad.dq_format = 9                                                            # neither INT8 nor E4M3
+    assert L.nf4_dequant(ctypes.byref(bad), out, None) == 2
+    assert L.nf4_dequant_flat(ctypes.byref(bad), 64, out, None) == 2
