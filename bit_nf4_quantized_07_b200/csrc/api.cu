@@ -1,9 +1,13 @@
 // C ABI of libqlora_nf4: argument checks, workspace layout, kernel dispatch.
 // Every entry point validates synchronously, then only enqueues work on the
-// caller's stream: no allocation, no synchronisation, no host-device copies.
+// caller's stream: no device-memory allocation, no synchronisation, no
+// host-device copies.  The backward may fork part of its work onto one
+// internal stream per device (created on first use) and joins it back onto
+// the caller's stream before returning.
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "qln_common.cuh"
 #include "qln_internal.h"
@@ -128,6 +132,46 @@ cudaError_t fused_gemm(const qln_nf4_weight *w, bool trans, const uint16_t *act,
         return qln::launch_nf4_tc_gemm(w, trans, act, n, lact, lw, r, out, status, st, num_sms);
     return qln::launch_nf4_mma_gemm(w, trans, act, n, lact, lw, r, out, status, st, num_sms);
 }
+
+// ---------------------------------------------------------------------------
+// The internal side stream of a device and the events that fork work onto it
+// and join it back: created on first use, kept until the process exits.  The
+// lock covers only the host-side enqueue of one fork/join.
+// ---------------------------------------------------------------------------
+struct SideCtx {
+    cudaStream_t stream;
+    cudaEvent_t fork, join;
+};
+std::mutex g_side_mu;
+SideCtx g_side[kMaxDevices];
+int g_side_state[kMaxDevices];  // 0 not tried, 1 ready, -1 unavailable
+
+// Caller holds g_side_mu.
+SideCtx *side_ctx() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (g_side_state[dev] == 0) {
+        SideCtx c{};
+        const bool ok = cudaStreamCreateWithFlags(&c.stream, cudaStreamNonBlocking) == cudaSuccess &&
+                        cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming) == cudaSuccess &&
+                        cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) cudaGetLastError();  // e.g. refused during stream capture: try again on a later call
+        else {
+            g_side[dev] = c;
+            g_side_state[dev] = 1;
+        }
+    }
+    return g_side_state[dev] == 1 ? &g_side[dev] : nullptr;
+}
+
+// dA and dB beside the dX GEMM: when the GEMM leaves at least this many SMs
+// idle (one wave of fewer CTAs than SMs), one persistent launch of as many
+// CTAs as idle SMs computes both on those SMs, so they can never delay the
+// GEMM's CTAs whichever launches first.
+constexpr int64_t kSideMinCtas = 8;
 
 }  // namespace
 
@@ -299,6 +343,23 @@ qln_status qlora_linear_bwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     // dA = s G^T X (the transpose of s X^T G), dB = s dY^T U.
     e = qln::launch_lora_down(dY, n, w->rows, B, true, r, s, G, sG, pGU, cs, kSplitTargetSms, reset);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
+    const int64_t gemm_ctas = qln::nf4_tc_gemm_ctas(w, true, n, r, sms);
+    const int64_t idle = gemm_ctas > 0 && gemm_ctas < sms ? sms - gemm_ctas : 0;
+    if (idle >= kSideMinCtas) {
+        std::lock_guard<std::mutex> lock(g_side_mu);
+        if (SideCtx *sc = side_ctx()) {
+            // fork: dA, dB on the idle SMs once G is ready; the GEMM on the caller's stream; join
+            e = cudaEventRecord(sc->fork, cs);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(sc->stream, sc->fork, 0);
+            if (e == cudaSuccess)
+                e = qln::launch_tn_skinny_side(dY, U, w->rows, X, G, w->cols, n, r, s, dA, dB, (int)idle, sc->stream);
+            if (e == cudaSuccess) e = cudaEventRecord(sc->join, sc->stream);
+            if (e != cudaSuccess) return QLN_ERR_CUDA;
+            e = fused_gemm(w, true, dY, n, sG, A, r, dX, status, cs, sms);
+            const cudaError_t j = cudaStreamWaitEvent(cs, sc->join, 0);
+            return from_cuda(e != cudaSuccess ? e : j);
+        }
+    }
     e = fused_gemm(w, true, dY, n, sG, A, r, dX, status, cs, sms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;
     e = qln::launch_tn_skinny(X, G, n, w->cols, r, s, true, dA, pA, L.splitA, cs);

@@ -284,20 +284,21 @@ cudaError_t launch_lora_down(const uint16_t *in, int64_t n, int64_t K, const uin
 // ===========================================================================
 constexpr int kSkBM = 128, kSkBK = 32, kSkPad = 136, kSkStages = 4;
 
-template <int NTJ>  // R <= 8 NTJ
-__global__ void __launch_bounds__(128) tn_skinny_kernel(const uint16_t *__restrict__ P, const uint16_t *__restrict__ Q,
-                                                        int64_t n, int64_t M, int R, float scale, bool transpose,
-                                                        float *__restrict__ C, float *__restrict__ partials) {
+// One 128-row tile of C over the token steps split, split + nsplit, ...:
+// accumulate P^T Q for rows [m0, m0 + 128) and all R columns, then store the
+// fp32 partial (partials != null) or scale * sum into C.  STG-stage cp.async
+// ring; the caller's CTA has 128 threads and STG * kSkBK * (kSkPad + QLD)
+// bf16 of shared memory.
+template <int NTJ, int STG>
+__device__ __forceinline__ void skinny_tile(const uint16_t *__restrict__ P, const uint16_t *__restrict__ Q, int64_t n,
+                                            int64_t M, int R, float scale, bool transpose, float *__restrict__ C,
+                                            float *__restrict__ partials, int64_t m0, int split, int nsplit,
+                                            uint16_t *sk) {
     constexpr int QW = NTJ * 8, QLD = QW + 8;
-    extern __shared__ __align__(16) uint16_t sk[];
-    uint16_t *Ps = sk;                                   // [stages][32][kSkPad]
-    uint16_t *Qs = sk + kSkStages * kSkBK * kSkPad;      // [stages][32][QLD]
-    pdl_wait();  // P and Q may come from the previous kernel on the stream
-    pdl_trigger();
+    uint16_t *Ps = sk;                             // [stages][32][kSkPad]
+    uint16_t *Qs = sk + STG * kSkBK * kSkPad;      // [stages][32][QLD]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
-    const int64_t m0 = (int64_t)blockIdx.x * kSkBM;
-    const int split = blockIdx.y, nsplit = gridDim.y;
     const int64_t nsteps = (n + kSkBK - 1) / kSkBK;
 
     float acc[2][NTJ][4];
@@ -327,19 +328,19 @@ __global__ void __launch_bounds__(128) tn_skinny_kernel(const uint16_t *__restri
 
     const int64_t mysteps = split < nsteps ? (nsteps - split + nsplit - 1) / nsplit : 0;
 #pragma unroll
-    for (int i = 0; i < kSkStages - 1; ++i) {
+    for (int i = 0; i < STG - 1; ++i) {
         if (i < mysteps) load(i, split + (int64_t)i * nsplit);
         cp_async_commit();
     }
     for (int64_t it = 0; it < mysteps; ++it) {
         {
-            const int64_t nx = it + kSkStages - 1;
-            if (nx < mysteps) load((int)(nx % kSkStages), split + nx * nsplit);
+            const int64_t nx = it + STG - 1;
+            if (nx < mysteps) load((int)(nx % STG), split + nx * nsplit);
             cp_async_commit();
         }
-        cp_async_wait<kSkStages - 1>();
+        cp_async_wait<STG - 1>();
         __syncthreads();
-        const int buf = (int)(it % kSkStages);
+        const int buf = (int)(it % STG);
         const uint16_t *Pb = Ps + buf * kSkBK * kSkPad;
         const uint16_t *Qb = Qs + buf * kSkBK * QLD;
 #pragma unroll
@@ -391,6 +392,43 @@ __global__ void __launch_bounds__(128) tn_skinny_kernel(const uint16_t *__restri
                         C[transpose ? (int64_t)j * M + m : m * R + j] = __fmul_rn(scale, acc[mt][nt][e]);
                 }
             }
+}
+
+template <int NTJ>  // R <= 8 NTJ
+__global__ void __launch_bounds__(128) tn_skinny_kernel(const uint16_t *__restrict__ P, const uint16_t *__restrict__ Q,
+                                                        int64_t n, int64_t M, int R, float scale, bool transpose,
+                                                        float *__restrict__ C, float *__restrict__ partials) {
+    extern __shared__ __align__(16) uint16_t sk[];
+    pdl_wait();  // P and Q may come from the previous kernel on the stream
+    pdl_trigger();
+    skinny_tile<NTJ, kSkStages>(P, Q, n, M, R, scale, transpose, C, partials, (int64_t)blockIdx.x * kSkBM, blockIdx.y,
+                                gridDim.y, sk);
+}
+
+// dB = s dY^T U and dA = s (X^T G)^T as one persistent launch of few CTAs,
+// for SMs the dX GEMM leaves idle: CTA b takes tiles b, b + gridDim.x, ... of
+// the list [dB tiles | dA tiles], each over all tokens (no split, no partials,
+// no fold: the order of every sum is fixed).  More stages than the split
+// kernel, since each CTA has an SM to itself.
+constexpr int kSideStages = 8;
+
+template <int NTJ>
+__global__ void __launch_bounds__(128) tn_skinny_side_kernel(const uint16_t *__restrict__ dY,
+                                                             const uint16_t *__restrict__ U, int64_t dout,
+                                                             const uint16_t *__restrict__ X,
+                                                             const uint16_t *__restrict__ G, int64_t din, int64_t n,
+                                                             int R, float scale, float *__restrict__ dA,
+                                                             float *__restrict__ dB) {
+    extern __shared__ __align__(16) uint16_t sk[];
+    pdl_wait();
+    const int64_t tB = (dout + kSkBM - 1) / kSkBM, tA = (din + kSkBM - 1) / kSkBM;
+    for (int64_t v = blockIdx.x; v < tB + tA; v += gridDim.x) {
+        __syncthreads();  // the previous tile's buffers are free
+        if (v < tB)
+            skinny_tile<NTJ, kSideStages>(dY, U, n, dout, R, scale, false, dB, nullptr, v * kSkBM, 0, 1, sk);
+        else
+            skinny_tile<NTJ, kSideStages>(X, G, n, din, R, scale, true, dA, nullptr, (v - tB) * kSkBM, 0, 1, sk);
+    }
 }
 
 __global__ void tn_skinny_fold_kernel(const float *__restrict__ partials, int splits, int64_t M, int R, float scale,
@@ -468,6 +506,42 @@ cudaError_t launch_tn_skinny(const uint16_t *P, const uint16_t *Q, int64_t n, in
     if (blocks > 4096) blocks = 4096;
     return launch_pdl(tn_skinny_fold_kernel, dim3((unsigned)blocks), dim3(256), 0, st, (const float *)partials, splits,
                       M, R, scale, transpose, C);
+}
+
+template <int NTJ>
+static cudaError_t launch_side_t(const uint16_t *dY, const uint16_t *U, int64_t dout, const uint16_t *X,
+                                 const uint16_t *G, int64_t din, int64_t n, int R, float scale, float *dA, float *dB,
+                                 int nside, cudaStream_t st) {
+    const size_t smem = (size_t)kSideStages * kSkBK * (kSkPad + NTJ * 8 + 8) * sizeof(uint16_t);
+    auto kern = tn_skinny_side_kernel<NTJ>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<nside, 128, smem, st>>>(dY, U, dout, X, G, din, n, R, scale, dA, dB);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tn_skinny_side(const uint16_t *dY, const uint16_t *U, int64_t dout, const uint16_t *X,
+                                  const uint16_t *G, int64_t din, int64_t n, int R, float scale, float *dA, float *dB,
+                                  int nside, cudaStream_t st) {
+    switch ((R + 7) / 8) {
+        case 1: return launch_side_t<1>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 2: return launch_side_t<2>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 3: return launch_side_t<3>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 4: return launch_side_t<4>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 5: return launch_side_t<5>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 6: return launch_side_t<6>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 7: return launch_side_t<7>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 8: return launch_side_t<8>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 9: return launch_side_t<9>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 10: return launch_side_t<10>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 11: return launch_side_t<11>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 12: return launch_side_t<12>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 13: return launch_side_t<13>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 14: return launch_side_t<14>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        case 15: return launch_side_t<15>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+        default: return launch_side_t<16>(dY, U, dout, X, G, din, n, R, scale, dA, dB, nside, st);
+    }
 }
 
 }  // namespace qln

@@ -457,6 +457,14 @@ bool nf4_tc_gemm_supported(const qln_nf4_weight *w, bool trans, int64_t n, int r
            tc::encode_fn() != nullptr;
 }
 
+int64_t nf4_tc_gemm_ctas(const qln_nf4_weight *w, bool trans, int64_t n, int r, int num_sms) {
+    if (!nf4_tc_gemm_supported(w, trans, n, r)) return 0;
+    const int64_t M = trans ? w->cols : w->rows;
+    const int64_t K = trans ? w->rows : w->cols;
+    const tc::TileShape shape = tc::choose_shape(M, K, n, num_sms > 0 ? num_sms : 148);
+    return ((n + (int64_t)shape.NT * shape.BN - 1) / ((int64_t)shape.NT * shape.BN)) * (M / (tc::kBM * shape.MT));
+}
+
 cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16_t *act, int64_t n,
                                const uint16_t *lact, const uint16_t *lw, int r, uint16_t *out, int *status,
                                cudaStream_t st, int num_sms) {

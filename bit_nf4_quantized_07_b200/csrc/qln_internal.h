@@ -67,6 +67,13 @@ size_t lora_down_partial_bytes(int64_t n, int64_t K, int r, int num_sms);
 cudaError_t launch_tn_skinny(const uint16_t *P, const uint16_t *Q, int64_t n, int64_t M, int R, float scale,
                              bool transpose, float *C, float *partials, int splits, cudaStream_t st);
 size_t tn_skinny_partials_bytes(int64_t M, int R, int splits);
+// dA and dB as one persistent launch of `nside` CTAs (for SMs a concurrent
+// kernel leaves idle); no partials.
+cudaError_t launch_tn_skinny_side(const uint16_t *dY, const uint16_t *U, int64_t dout, const uint16_t *X,
+                                  const uint16_t *G, int64_t din, int64_t n, int R, float scale, float *dA, float *dB,
+                                  int nside, cudaStream_t st);
+// CTAs the tcgen05 GEMM launches for this call (0 when it does not take the call).
+int64_t nf4_tc_gemm_ctas(const qln_nf4_weight *w, bool trans, int64_t n, int r, int num_sms);
 int tn_skinny_splits(int64_t n, int64_t M, int R, int num_sms);
 
 // nf4_gemm_sm80.cu: fused NF4 decode + legacy mma.sync GEMM (small n).
