@@ -47,6 +47,10 @@ SMALL = [
     synthetic.custom("r128_128x256_n33_r128", 128, 256, 33, 128, s=2.0, index=14),
     synthetic.custom("tokens_tile_512x256_n256_r16", 512, 256, 256, 16, s=2.0, index=15),
     synthetic.custom("wide_384x1024_n640_r32", 384, 1024, 640, 32, s=1.5, index=16, outlier_rate=0.001),
+    # tcgen05 path with r = 128: dA and dB beside the dX GEMM with 16 fragment columns
+    synthetic.custom("side_r128_256x512_n128_r128", 256, 512, 128, 128, s=0.5, index=42),
+    # ragged token tiles on the tcgen05 path, side kernel with r = 24
+    synthetic.custom("side_r24_640x768_n200_r24", 640, 768, 200, 24, s=1.0, index=43),
 ]
 
 
