@@ -165,11 +165,36 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
     int *ucount = reinterpret_cast<int *>(reinterpret_cast<char *>(p.status) + kWsUCountOffset);
     int *uflag = reinterpret_cast<int *>(reinterpret_cast<char *>(p.status) + kWsUFlagOffset);
     int *udone = reinterpret_cast<int *>(reinterpret_cast<char *>(p.status) + kWsDoneOffset);
+    const bool ucta = (int)blockIdx.x >= p.Q * S;
+    const uint32_t wbar = bars + (uint32_t)warp * 16u;  // stage st's barrier at + 8 st
+    if (!ucta) {
+        // Before the dependency wait only shared memory and the launch's own
+        // parameters are touched, nothing an earlier kernel on the stream can
+        // change: the barriers and the decode table are ready while that
+        // kernel finishes.
+        if (lane == 0) {
+            tc::mbar_init(wbar, 1);
+            tc::mbar_init(wbar + 8, 1);
+            tc::mbar_fence_init();
+            tc::tma_prefetch_map(&tm_codes);
+        }
+        {   // table: warp w writes the rows e = 16 k + w, so c[e >> 4] = c[k] is a constant
+            float clo = 0.f;
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+                if (q == warp) clo = nf4_value(q);
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                *reinterpret_cast<uint32_t *>(tab + (16 * k + warp) * 256 + lane * 4) =
+                    pack_bf16x2(nf4_value(k), clo);
+        }
+        __syncwarp();
+    }
     pdl_wait();  // X, the weight and the workspace may all be touched by the previous kernel on the stream
     pdl_trigger();
 
     // ---- U CTAs: U = X A^T, once for the grid ------------------------------------
-    if ((int)blockIdx.x >= p.Q * S) {
+    if (ucta) {
         const int u = (int)blockIdx.x - p.Q * S;  // 0 .. UG-1; U clusters hold U CTAs only
         const int64_t ub0 = KB * u / p.UG, ub1 = KB * (u + 1) / p.UG;  // this CTA's K range of U
         const int njt = r / 8, nsubu = kDvWarps / njt;
@@ -244,15 +269,7 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
     if (blockIdx.x == 0 && tid == 0) *p.status = QLN_OK;
     cluster_arrive_relaxed();  // "started": no peer writes here before every CTA of the cluster runs
 
-    // ---- 1. requests: two units of codes per warp, X chunk, constants, table ---
-    const uint32_t wbar = bars + (uint32_t)warp * 16u;  // stage st's barrier at + 8 st
-    if (lane == 0) {
-        tc::mbar_init(wbar, 1);
-        tc::mbar_init(wbar + 8, 1);
-        tc::mbar_fence_init();
-        tc::tma_prefetch_map(&tm_codes);
-    }
-    __syncwarp();
+    // ---- 1. requests: two units of codes per warp, X chunk, constants --------------
     const uint32_t ring_s = smem_u32(ring) + (uint32_t)(warp * kDvStageBytes);  // stage st at + st * 16 stages
     auto issue_codes = [&](int k, int st) {  // round k's unit of this warp -> stage st
         const int64_t tl = t0 + (int64_t)(kDvWarps * k + warp) / nsub;
@@ -305,16 +322,6 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DvPara
         for (int64_t l = rank * kDvThreads + tid; l < lines; l += (int64_t)S * kDvThreads)
             asm volatile("prefetch.global.L2 [%0];" ::"l"(bb + l * 128));
     }
-    {   // table: warp w writes the rows e = 16 k + w, so c[e >> 4] = c[k] is a constant
-        float clo = 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-            if (q == warp) clo = nf4_value(q);
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-            *reinterpret_cast<uint32_t *>(tab + (16 * k + warp) * 256 + lane * 4) = pack_bf16x2(nf4_value(k), clo);
-    }
-
     cp_async_wait<0>();  // X
     __syncthreads();
     cluster_wait();      // every CTA of the cluster has started
