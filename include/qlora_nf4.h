@@ -163,6 +163,11 @@ QLN_API qln_status nf4_quantize_ex(const void *W, int32_t dtype, int64_t numel, 
  *   counters of the single-launch path's grid barrier.  Zero the header once
  *   before the first call; every call leaves it zeroed again (zero it anew
  *   after a QLN_ERR_TIMEOUT).  The rest is scratch.
+ * Weights of up to about 116 M parameters take a single launch whose CTAs
+ * meet at a grid-wide barrier; its grid is sized so that the whole device
+ * holds it at once.  A kernel on another stream that keeps SMs busy only
+ * delays it, and a wait longer than 2 s ends with QLN_ERR_TIMEOUT in the
+ * status word instead of a hang.
  * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE if nb <= 0 or nb > 2^25 (numel above
  * 2^31); QLN_ERR_WORKSPACE; QLN_ERR_ALIGN if absmax is not 16-byte aligned or
  * ws is not 256-byte aligned.
