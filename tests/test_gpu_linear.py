@@ -1,5 +1,5 @@
 """GPU parity of the fused QLoRA linear (forward and backward) against the
-float64 oracle.  Tolerance (the benchmark spec): normwise max relative error
+float64 oracle.  Tolerance (the stated target): normwise max relative error
 max|T - T*| / max|T*| <= 2e-2 per output tensor."""
 import numpy as np
 import pytest
