@@ -51,6 +51,7 @@
 // host picks S per shape and device), so results do not depend on timing.
 // Remote shared-memory accesses are stores only and all land before the
 // epoch's cluster barrier.
+#include <atomic>
 #include <type_traits>
 
 #include "qln_common.cuh"
@@ -596,13 +597,18 @@ size_t nf4_gemv_ws_bytes(int64_t n, int r) {
 
 template <int NT>
 static cudaError_t dv_max_clusters(int S, int *out) {
-    static int cache[64][9];  // per device and cluster size: co-resident clusters (0 = not asked yet)
+    // per device and cluster size: co-resident clusters (0 = not asked yet);
+    // host threads may launch at once, so the entries are atomics
+    static std::atomic<int> cache[64][9];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && cache[dev][S] > 0) {
-        *out = cache[dev][S];
-        return cudaSuccess;
+    if (dev >= 0 && dev < 64) {
+        const int c = cache[dev][S].load(std::memory_order_relaxed);
+        if (c > 0) {
+            *out = c;
+            return cudaSuccess;
+        }
     }
     e = cudaFuncSetAttribute(nf4_decode_fwd_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDvSmemMax);
     if (e != cudaSuccess) return e;
@@ -621,7 +627,7 @@ static cudaError_t dv_max_clusters(int S, int *out) {
     e = cudaOccupancyMaxActiveClusters(&nclus, (const void *)nf4_decode_fwd_kernel<NT>, &q);
     if (e != cudaSuccess) return e;
     if (nclus < 1) return cudaErrorInvalidConfiguration;
-    if (dev >= 0 && dev < 64) cache[dev][S] = nclus;
+    if (dev >= 0 && dev < 64) cache[dev][S].store(nclus, std::memory_order_relaxed);
     *out = nclus;
     return cudaSuccess;
 }
