@@ -91,6 +91,14 @@ def codec_bytes_per_param():
     return q, d
 
 
+def decode_bytes_per_call(rows, cols, n, r):
+    """Algorithmic bytes of one decode-sized forward with a double-quantized
+    weight: codes, rhat, group scales and mu, then X, A, B, U and Y (bf16)."""
+    nb = rows * cols // 64
+    wbytes = rows * cols // 2 + nb + 4 * ((nb + 255) // 256) + 4
+    return wbytes + 2 * n * cols + 2 * r * cols + 2 * rows * r + 2 * n * r + 2 * n * rows
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -282,9 +290,7 @@ def measure_decode(api, dev, copies=64, reps=5):
         torch.cuda.synchronize()
         per_call = e0.elapsed_time(e1) / (reps * copies) * 1e-3
         del graph
-        nb = rows * cols // 64
-        wbytes = rows * cols // 2 + nb + 4 * ((nb + 255) // 256) + 4
-        bytes_call = wbytes + 2 * n * cols + 2 * r * cols + 2 * rows * r + 2 * n * r + 2 * n * rows
+        bytes_call = decode_bytes_per_call(rows, cols, n, r)
         out[f"n{n}"] = {"us_per_call": per_call * 1e6, "GBs": bytes_call / per_call / 1e9,
                         "TFLOPs": 2 * n * (rows * cols + r * cols + rows * r) / per_call / 1e12,
                         "timing": f"CUDA graph of {copies} calls on {copies} weight copies, {reps} replays"}

@@ -66,3 +66,19 @@ def test_sweep_size_and_bytes():
     q, d = bench.codec_bytes_per_param()
     assert abs(q * params / 1e9 - 29.25) < 0.01  # 29.2448 GB, quoted to four figures
     assert abs(d * params / 1e9 - 16.29) < 0.01
+
+
+def test_decode_bytes_per_call():
+    """Decode layer 4096 x 4096, r = 16: 8.93 / 8.98 / 9.18 MB per call at
+    n = 1 / 4 / 16, of which the weight is 8.65 MB (codes 8.39 MB, rhat
+    0.26 MB, scales 4 KB); the parts are the sizes of the arrays read and
+    written."""
+    rows = cols = 4096
+    r = 16
+    weight = rows * cols // 2 + rows * cols // 64 + 4 * (rows * cols // (64 * 256)) + 4
+    assert abs(weight / 1e6 - 8.65) < 0.005
+    for n, mb in ((1, 8.93), (4, 8.98), (16, 9.18)):
+        acts = 2 * (n * cols + r * cols + rows * r + n * r + n * rows)
+        got = bench.decode_bytes_per_call(rows, cols, n, r)
+        assert got == weight + acts
+        assert abs(got / 1e6 - mb) < 0.005
