@@ -1,13 +1,10 @@
 // C ABI of libqlora_nf4: argument checks, workspace layout, kernel dispatch.
 // Every entry point validates synchronously, then only enqueues work on the
 // caller's stream: no device-memory allocation, no synchronisation, no
-// host-device copies.  The backward may fork part of its work onto one
-// internal stream per device (created on first use) and joins it back onto
-// the caller's stream before returning.
+// host-device copies, no streams or events of its own.
 #include <string.h>
 
 #include <atomic>
-#include <mutex>
 
 #include "qln_common.cuh"
 #include "qln_internal.h"
@@ -48,11 +45,10 @@ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int kSplitTargetSms = 148;
 
 // Workspace layout of the linear calls (all offsets 256-byte aligned):
-//   [0, 256)        header: int32 device status word (0 = QLN_OK) at 0, the
-//                   decode-sized forward's counters at 64 and 128
+//   [0, 256)        header: int32 device status word (0 = QLN_OK) at 0
 //   fwd: sU [n][r] bf16, U [n][r] bf16 (used when U_out is NULL),
-//        split-K partials of U (fp32) -- or, for decode-sized n, the parts of
-//        U and bf16(s U) of the one-launch forward
+//        split-K partials of U (fp32); the decode-sized forward uses only the
+//        header
 //   bwd: G [n][r] bf16, sG [n][r] bf16, U [n][r] bf16, split-K partials of
 //        G / U (fp32, reused), dA partials, dB partials
 // Split counts are planned for a fixed SM count so that the workspace size
@@ -72,9 +68,7 @@ FwdWs fwd_layout(int64_t rows, int64_t cols, int64_t n, int r) {
     L.sU = qln::kWsHeaderBytes;
     L.U = L.sU + nr;
     L.pU = L.U + nr;
-    const size_t generic = L.pU + round256(qln::lora_down_partial_bytes(n, cols, r, kSplitTargetSms));
-    const size_t decode = qln::kWsHeaderBytes + round256(qln::nf4_gemv_ws_bytes(n, r));
-    L.total = generic > decode ? generic : decode;
+    L.total = L.pU + round256(qln::lora_down_partial_bytes(n, cols, r, kSplitTargetSms));
     return L;
 }
 
@@ -133,44 +127,11 @@ cudaError_t fused_gemm(const qln_nf4_weight *w, bool trans, const uint16_t *act,
     return qln::launch_nf4_mma_gemm(w, trans, act, n, lact, lw, r, out, status, st, num_sms);
 }
 
-// ---------------------------------------------------------------------------
-// The internal side stream of a device and the events that fork work onto it
-// and join it back: created on first use, kept until the process exits.  The
-// lock covers only the host-side enqueue of one fork/join.
-// ---------------------------------------------------------------------------
-struct SideCtx {
-    cudaStream_t stream;
-    cudaEvent_t fork, join;
-};
-std::mutex g_side_mu;
-SideCtx g_side[kMaxDevices];
-int g_side_state[kMaxDevices];  // 0 not tried, 1 ready, -1 unavailable
-
-// Caller holds g_side_mu.
-SideCtx *side_ctx() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        cudaGetLastError();
-        return nullptr;
-    }
-    if (g_side_state[dev] == 0) {
-        SideCtx c{};
-        const bool ok = cudaStreamCreateWithFlags(&c.stream, cudaStreamNonBlocking) == cudaSuccess &&
-                        cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming) == cudaSuccess &&
-                        cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming) == cudaSuccess;
-        if (!ok) cudaGetLastError();  // e.g. refused during stream capture: try again on a later call
-        else {
-            g_side[dev] = c;
-            g_side_state[dev] = 1;
-        }
-    }
-    return g_side_state[dev] == 1 ? &g_side[dev] : nullptr;
-}
-
 // dA and dB beside the dX GEMM: when the GEMM leaves at least this many SMs
 // idle (one wave of fewer CTAs than SMs), one persistent launch of as many
-// CTAs as idle SMs computes both on those SMs, so they can never delay the
-// GEMM's CTAs whichever launches first.
+// CTAs as idle SMs computes both on those SMs.  It is the GEMM's programmatic
+// dependent, so it starts only once every GEMM CTA is resident and can never
+// hold an SM the GEMM needs.
 constexpr int64_t kSideMinCtas = 8;
 
 }  // namespace
@@ -294,10 +255,10 @@ qln_status qlora_linear_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     uint16_t *sU = reinterpret_cast<uint16_t *>(wsb + L.sU);
     uint16_t *U = U_out ? U_out : reinterpret_cast<uint16_t *>(wsb + L.U);
     float *pU = reinterpret_cast<float *>(wsb + L.pU);
-    if (qln::nf4_gemv_supported(w, n, r)) {
+    if (qln::nf4_decode_fwd_supported(w, n, r)) {
         // decode-sized n: one launch forms U and the whole forward; it clears
         // the status word itself, so no memset precedes it
-        return from_cuda(qln::launch_nf4_gemv(w, X, n, A, B, r, s, Y, U_out, ws, cs));
+        return from_cuda(qln::launch_nf4_decode_fwd(w, X, n, A, B, r, s, Y, U_out, status, cs));
     }
     // U = X A^T (and s*U for the adapter MMA; its first kernel also clears the
     // status word), then the fused weight GEMM.  No memset between kernels:
@@ -346,19 +307,11 @@ qln_status qlora_linear_bwd(const qln_nf4_weight *w, const uint16_t *X, int64_t 
     const int64_t gemm_ctas = qln::nf4_tc_gemm_ctas(w, true, n, r, sms);
     const int64_t idle = gemm_ctas > 0 && gemm_ctas < sms ? sms - gemm_ctas : 0;
     if (idle >= kSideMinCtas) {
-        std::lock_guard<std::mutex> lock(g_side_mu);
-        if (SideCtx *sc = side_ctx()) {
-            // fork: dA, dB on the idle SMs once G is ready; the GEMM on the caller's stream; join
-            e = cudaEventRecord(sc->fork, cs);
-            if (e == cudaSuccess) e = cudaStreamWaitEvent(sc->stream, sc->fork, 0);
-            if (e == cudaSuccess)
-                e = qln::launch_tn_skinny_side(dY, U, w->rows, X, G, w->cols, n, r, s, dA, dB, (int)idle, sc->stream);
-            if (e == cudaSuccess) e = cudaEventRecord(sc->join, sc->stream);
-            if (e != cudaSuccess) return QLN_ERR_CUDA;
-            e = fused_gemm(w, true, dY, n, sG, A, r, dX, status, cs, sms);
-            const cudaError_t j = cudaStreamWaitEvent(cs, sc->join, 0);
-            return from_cuda(e != cudaSuccess ? e : j);
-        }
+        // the GEMM, then dA and dB on the SMs it leaves idle: launched on the
+        // same stream as the GEMM's programmatic dependent, so the two overlap
+        e = fused_gemm(w, true, dY, n, sG, A, r, dX, status, cs, sms);
+        if (e != cudaSuccess) return QLN_ERR_CUDA;
+        return from_cuda(qln::launch_tn_skinny_side(dY, U, w->rows, X, G, w->cols, n, r, s, dA, dB, (int)idle, cs));
     }
     e = fused_gemm(w, true, dY, n, sG, A, r, dX, status, cs, sms);
     if (e != cudaSuccess) return QLN_ERR_CUDA;

@@ -410,6 +410,17 @@ __global__ void __launch_bounds__(128) tn_skinny_kernel(const uint16_t *__restri
 // the list [dB tiles | dA tiles], each over all tokens (no split, no partials,
 // no fold: the order of every sum is fixed).  More stages than the split
 // kernel, since each CTA has an SM to itself.
+//
+// It is launched on the caller's stream right after the dX GEMM, as its
+// programmatic dependent, and runs beside it.  It reads dY, U, X and G before
+// any dependency wait.  That is safe because a dependent can start only once
+// every CTA of the GEMM has released it, and every kernel of this library
+// releases its dependents only after its own dependency wait; so when this
+// kernel starts, every kernel before the GEMM (those that wrote G, U, dY, X)
+// has completed, and its writes are in L2, which is where the cp.async.cg
+// copies read.  The GEMM writes none of these inputs and reads neither dA nor
+// dB.  The kernel waits on the GEMM before it exits, so it never completes
+// before the GEMM does, and a kernel that follows it on the stream sees dX.
 constexpr int kSideStages = 8;
 
 template <int NTJ>
@@ -420,7 +431,6 @@ __global__ void __launch_bounds__(128) tn_skinny_side_kernel(const uint16_t *__r
                                                              int R, float scale, float *__restrict__ dA,
                                                              float *__restrict__ dB) {
     extern __shared__ __align__(16) uint16_t sk[];
-    pdl_wait();
     const int64_t tB = (dout + kSkBM - 1) / kSkBM, tA = (din + kSkBM - 1) / kSkBM;
     for (int64_t v = blockIdx.x; v < tB + tA; v += gridDim.x) {
         __syncthreads();  // the previous tile's buffers are free
@@ -429,6 +439,7 @@ __global__ void __launch_bounds__(128) tn_skinny_side_kernel(const uint16_t *__r
         else
             skinny_tile<NTJ, kSideStages>(X, G, n, din, R, scale, true, dA, nullptr, (v - tB) * kSkBM, 0, 1, sk);
     }
+    pdl_wait();  // complete only after the dX GEMM
 }
 
 __global__ void tn_skinny_fold_kernel(const float *__restrict__ partials, int splits, int64_t M, int R, float scale,
@@ -516,8 +527,8 @@ static cudaError_t launch_side_t(const uint16_t *dY, const uint16_t *U, int64_t 
     auto kern = tn_skinny_side_kernel<NTJ>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<nside, 128, smem, st>>>(dY, U, dout, X, G, din, n, R, scale, dA, dB);
-    note_launch();
+    e = launch_pdl(kern, dim3((unsigned)nside), dim3(128), smem, st, dY, U, dout, X, G, din, n, R, scale, dA, dB);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -87,27 +87,16 @@ cudaError_t launch_nf4_mma_gemm(const qln_nf4_weight *w, bool trans, const uint1
 bool make_tensor_map_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t inner,
                         uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
 
-// Workspace header of the linear calls: the int32 status word at byte 0 and
-// three counters of the decode-sized forward.  The counters must be zero when a
-// workspace is first used; every launch that uses them leaves them at zero.
+// Workspace header of the linear calls: the int32 device status word at byte 0.
 constexpr int kWsHeaderBytes = 256;
-constexpr int kWsUCountOffset = 64;   // int32: CTAs that have published their part of U
-constexpr int kWsUFlagOffset = 128;   // int32: 1 once bf16(s U) of the call is in the workspace
-constexpr int kWsDoneOffset = 192;    // int32: CTAs that have read bf16(s U)
-// SM count the decode-sized forward sizes its workspace for (B200); its grid
-// never exceeds it.
-constexpr int kDvPlanSms = 148;
 
-// nf4_gemv.cu: the whole forward for decode-sized n (<= 32) in one launch of
+// nf4_decode.cu: the whole forward for decode-sized n (<= 32) in one launch of
 // thread-block clusters: U = X A^T, Y = bf16(X W'^T + bf16(s U) B^T),
-// U_out = bf16(U).
-//   ws: the workspace (header as above); scratch from byte kWsHeaderBytes on,
-//   nf4_gemv_ws_bytes(...) of it.
-bool nf4_gemv_supported(const qln_nf4_weight *w, int64_t n, int r);
-size_t nf4_gemv_ws_bytes(int64_t n, int r);
-cudaError_t launch_nf4_gemv(const qln_nf4_weight *w, const uint16_t *X, int64_t n, const uint16_t *A,
-                            const uint16_t *B, int r, float s, uint16_t *Y, uint16_t *U_out, void *ws,
-                            cudaStream_t st);
+// U_out = bf16(U) (if not null).  Needs no workspace beyond the status word.
+bool nf4_decode_fwd_supported(const qln_nf4_weight *w, int64_t n, int r);
+cudaError_t launch_nf4_decode_fwd(const qln_nf4_weight *w, const uint16_t *X, int64_t n, const uint16_t *A,
+                                  const uint16_t *B, int r, float s, uint16_t *Y, uint16_t *U_out, int *status,
+                                  cudaStream_t st);
 
 // nf4_gemm_sm100.cu: fused NF4 decode + tcgen05 GEMM (TMA, TMEM accumulators).
 cudaError_t launch_nf4_tc_gemm(const qln_nf4_weight *w, bool trans, const uint16_t *act, int64_t n,
