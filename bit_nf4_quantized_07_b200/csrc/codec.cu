@@ -286,14 +286,18 @@ constexpr int kQzLutBytes = 256 * 128;                                    // 256
 template <typename T, typename Idx>
 __global__ void __launch_bounds__(kQzThreads, kQzCtasPerSm) nf4_quantize_kernel(const T *__restrict__ W, Idx numel,
                                                                                 uint8_t *__restrict__ codes,
-                                                                                float *__restrict__ absmax) {
+                                                                                float *__restrict__ absmax,
+                                                                                bool release_early) {
     constexpr int kB = QzIn<T>::kBytes;
     extern __shared__ __align__(16) unsigned char qz_smem[];
     for (int i = threadIdx.x; i < kQzLutBytes / 4; i += kQzThreads)  // bucket i/32, lane i%32
         reinterpret_cast<uint32_t *>(qz_smem)[i] = kSnapTable.e[i >> 5];
     __syncthreads();
     pdl_wait();  // W may come from the previous kernel; codes/absmax may still be read by it
-    pdl_trigger();
+    // This kernel writes a weight (codes, absmax), and a forward may read its
+    // weight before its own dependency wait; so the next kernel is released
+    // early only when it is known to wait first.
+    if (release_early) pdl_trigger();
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -381,7 +385,7 @@ static cudaError_t launch_quantize_t(const T *W, int64_t numel, uint8_t *codes, 
         cudaFuncSetAttribute(nf4_quantize_kernel<T, Idx>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(nf4_quantize_kernel<T, Idx>, dim3((unsigned)grid), dim3(kQzThreads), (size_t)smem, st, W,
-                      (Idx)numel, codes, absmax);
+                      (Idx)numel, codes, absmax, false);
 }
 
 template <typename T>
@@ -527,7 +531,7 @@ __global__ void __launch_bounds__(kDqThreads) dq_quant_kernel(const float *__res
     __shared__ double slice[kDqThreads / 32];
     __shared__ float mu_s;
     pdl_wait();
-    pdl_trigger();
+    // writes the DQ constants of a weight: no early release (see the quantize kernel)
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int64_t g = (int64_t)blockIdx.x * (kDqThreads / 32) + warp;
@@ -613,7 +617,7 @@ __global__ void __launch_bounds__(kDqThreads) dq_fused_kernel(const float *__res
     int *leave = reinterpret_cast<int *>(ws + kDqfLeaveOffset);
     double *partial = reinterpret_cast<double *>(ws + 256);
     pdl_wait();  // the constants come from the previous kernel (the quantize)
-    pdl_trigger();
+    // writes the DQ constants of a weight: no early release (see the quantize kernel)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
     const int64_t g0 = ((int64_t)blockIdx.x * (kDqThreads / 32) + warp) * GPW;

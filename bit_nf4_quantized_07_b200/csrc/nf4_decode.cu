@@ -50,7 +50,6 @@
 // 2st+1 (k pair "2c+8"), and X and A are read with the same permutation of k,
 // so every product still pairs equal k.
 #include <atomic>
-#include <type_traits>
 
 #include "qln_common.cuh"
 #include "qln_internal.h"
@@ -84,7 +83,7 @@ struct DfParams {
     uint16_t *Y;         // [n][rows]
     uint16_t *U_out;     // [n][r] or null
     int *status;         // device status word
-    int S, Q, nsub, nkb_max, RS, E, JT;
+    int S, Q, nsub, nsubA, nkb_max, RS, E, JT;
     int off_ring, off_slots, off_uslots, off_sb, off_su, off_ah, off_bar;  // shared-memory layout (bytes)
 };
 
@@ -129,7 +128,7 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
     // and tile row fits); 64-bit values appear only in global offsets.
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
-    const int n = p.n, r = p.r, S = p.S, nsub = p.nsub, nkbx = p.nkb_max, RS = p.RS, E = p.E;
+    const int n = p.n, r = p.r, S = p.S, nsub = p.nsub, nsubA = p.nsubA, nkbx = p.nkb_max, RS = p.RS, E = p.E;
     const int KB = p.KB, T = p.T, Q = p.Q;
     const int rank = (int)blockIdx.x % S, cl = (int)blockIdx.x / S;
     const int kb0 = KB * rank / S, nkb = KB * (rank + 1) / S - kb0;
@@ -149,9 +148,17 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
     const uint32_t slots_s = smem_u32(dsm + p.off_slots), uslots_s = smem_u32(dsm + p.off_uslots);
     const int ahs = nkbx + 1;
 
-    // Before the dependency wait only shared memory and the launch's own
-    // parameters are touched, nothing an earlier kernel on the stream can
-    // change: barriers and the decode table are ready while that kernel ends.
+    // Before the dependency wait the kernel touches shared memory, the
+    // launch's parameters and the weight (codes and block constants), never X,
+    // A, B, Y or U.  Reading the weight early is safe because the kernel ahead
+    // of this one on the stream has released it only after its own dependency
+    // wait (every kernel of this library does), so every kernel before that
+    // one has completed; and the kernels of this library that write a weight
+    // (quantize, double quantization) never release their dependents early, so
+    // if the kernel ahead wrote this weight, this one starts after it has
+    // completed.  A caller's own kernel that writes the weight must not release
+    // its dependents early either (it does not unless it executes
+    // griddepcontrol.launch_dependents).
     cl_arrive_relaxed();  // this CTA runs: peers may store into it once they have waited
     if (lane == 0) {
         for (int s = 0; s < RS; ++s) tc::mbar_init(bar_w + 8u * s, 1);
@@ -160,27 +167,35 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
     }
     {   // table: warp w writes the rows e = 16 k + w, so c[e & 15] = c[w] is a constant
         const float clo = nf4_value(warp);
-#pragma unroll 1
-        for (int k = 0; k < 16; ++k)
+#pragma unroll
+        for (int k = 0; k < 16; ++k)  // k is a compile-time index: c[k] is a literal
             *reinterpret_cast<uint32_t *>(tab + (16 * k + warp) * 256 + lane * 4) = pack_bf16x2(nf4_value(k), clo);
     }
     __syncwarp();
-    pdl_wait();  // X, A, B and the weight may all be written by the previous kernel on the stream
-    pdl_trigger();
-    if (blockIdx.x == 0 && tid == 0) *p.status = QLN_OK;
 
-    auto issue = [&](int k) {  // box k of this warp's list -> ring slot k % RS
-        if (k < nboxes && lane == 0) {
-            const int ii = k / nbox, gb = k - ii * nbox;
-            const int e = ii / cntf, u = ii - e * cntf;
-            const int tile = t0 + e * E + ts0 + L * u;
-            const int s = k % RS;
+    // The boxes of this warp's list are requested in order: box k goes to ring
+    // slot k % RS.  The cursor (epoch ie, item iu within it, box ig within the
+    // item, slot is) follows the list without divisions.
+    int ik = 0, ie = 0, iu = 0, ig = 0, is = 0;
+    auto issue_next = [&]() {
+        if (ik < nboxes && lane == 0) {
+            const int tile = t0 + ie * E + ts0 + L * iu;
             tc::fence_proxy_async_smem();  // the slot's earlier reads come before the copy
-            tc::mbar_arrive_expect_tx(bar_w + 8u * s, (uint32_t)kDfBoxBytes);
-            tc::tma_load_2d(ring_w + (uint32_t)(s * kDfBoxBytes), &tm_codes, (kb0 + sb0 + 4 * gb) * 32, tile * 16,
-                            bar_w + 8u * s);
+            tc::mbar_arrive_expect_tx(bar_w + 8u * is, (uint32_t)kDfBoxBytes);
+            tc::tma_load_2d(ring_w + (uint32_t)(is * kDfBoxBytes), &tm_codes, (kb0 + sb0 + 4 * ig) * 32, tile * 16,
+                            bar_w + 8u * is);
+        }
+        ++ik;
+        if (++is == RS) is = 0;
+        if (++ig == nbox) {
+            ig = 0;
+            if (++iu == cntf) {
+                iu = 0;
+                ++ie;
+            }
         }
     };
+
     // adapter rows B of the tiles this CTA folds in epoch e (tile ts = li * S + rank)
     auto stage_b = [&](int e) {
         const int Ee = e + 1 < nep ? E : El;
@@ -223,22 +238,27 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
         }
     };
 
-    // ---- 1. requests: the small operands first, then the code boxes ------------------
+    // ---- 1. requests: the weight (code boxes, block constants) before the
+    //         dependency wait, then X and the B rows ---------------------------------------
+#pragma unroll 1
+    for (int k = 0; k < RS; ++k) issue_next();
+    stage_ah(0);
+    pdl_wait();  // X, A, B and the workspace may be written by the previous kernel on the stream
+    pdl_trigger();
+    if (blockIdx.x == 0 && tid == 0) *p.status = QLN_OK;
     // X chunk: line (token t, block bl) at row t * nkbx + bl, second half; 16-B chunks swizzled by t & 1
 #pragma unroll 1
-    for (int i = tid; i < 8 * NT * nkbx * 8; i += kDfThreads) {
-        const int t = i / (nkbx * 8), j = i - t * (nkbx * 8);
-        uint8_t *dst = tab + (t * nkbx + (j >> 3)) * 256 + 128 + (((j & 7) ^ (t & 1)) << 4);
-        if (t < n && j < nkb * 8)
-            cp_async16(dst, p.X + (int64_t)t * p.cols + kb0 * 64 + j * 8);
-        else
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
+    for (int t = warp; t < 8 * NT; t += kDfWarps)
+#pragma unroll 1
+        for (int j = lane; j < nkbx * 8; j += 32) {
+            uint8_t *dst = tab + (t * nkbx + (j >> 3)) * 256 + 128 + (((j & 7) ^ (t & 1)) << 4);
+            if (t < n && j < nkb * 8)
+                cp_async16(dst, p.X + (int64_t)t * p.cols + kb0 * 64 + j * 8);
+            else
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
     stage_b(0);
     cp_async_commit();
-#pragma unroll 1
-    for (int k = 0; k < RS; ++k) issue(k);
-    stage_ah(0);
     cp_async_wait<0>();
     __syncthreads();  // table, X, block constants and the B rows of epoch 0 in place
 
@@ -251,13 +271,14 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
         xoff[nt] = (uint32_t)((t * nkbx + sb0) * 256 + 128 + (((2 * c) ^ (t & 1)) << 4));
     }
     // one 64-wide block: 4 MMA steps per token tile into tmp (A from the decode table
-    // or, for A tiles, straight from registers)
+    // or, for A items, straight from registers)
     auto block_mma = [&](uint32_t xb, const uint32_t (&av)[4][4], float (&tmp)[NT][4], bool zero) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             uint4 xv[NT];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) xv[nt] = df_lds128(tab + ((xoff[nt] + xb) ^ (uint32_t)(hh << 4)));
+            for (int nt = 0; nt < NT; ++nt)  // token rows past n are zero: no load
+                xv[nt] = 8 * nt + g < n ? df_lds128(tab + ((xoff[nt] + xb) ^ (uint32_t)(hh << 4))) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int sp = 0; sp < 2; ++sp) {
                 const int st = 2 * hh + sp;
@@ -276,16 +297,21 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
 #pragma unroll 1
     for (int e = 0; e < nep; ++e) {
         const int Ee = e + 1 < nep ? E : El;
-        const int nts = Ee + (e == 0 ? p.JT : 0);
+        // this warp's items: weight tiles ts0, ts0 + L, ...; then, in the first
+        // epoch, A items w, w + 16, ... (A tile jt, block sub-range sa of nsubA)
+        const int nwi = Ee > ts0 ? (Ee - ts0 + L - 1) / L : 0;
+        const int nai = e == 0 && p.JT * nsubA > warp ? (p.JT * nsubA - warp + kDfWarps - 1) / kDfWarps : 0;
         bool waited = false;
 #pragma unroll 1
-        for (int ts = ts0; ts < nts; ts += L) {
+        for (int it = 0; it < nwi + nai; ++it) {
+            const bool wt = it < nwi;
+            const int ts = ts0 + L * it;                   // weight tile of the epoch (wt)
+            const int ja = warp + kDfWarps * (it - nwi);   // A item (!wt)
             float acc[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) acc[nt][q] = 0.f;
-            const bool wt = ts < Ee;
             if (wt) {
                 // ---- a weight tile: decode and multiply, box by box, block by block ----
                 const float *ahr = sAh + (ts * 16 + g) * ahs + sb0;  // row g; row g + 8 at + 8 * ahs
@@ -328,23 +354,27 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
                         }
                     }
                     __syncwarp();  // every lane is done with this slot
-                    issue(kbx + RS);
+                    issue_next();  // box kbx + RS
                     ++kbx;
                 }
             } else {
-                // ---- an A tile: rows 16 jt .. 16 jt + 15 of A (zero past r), the same MMA ----
-                const int j0 = 16 * (ts - Ee) + g, j1 = j0 + 8;  // rows past r read as zero
-                const uint16_t *ar0 = p.A + (int64_t)(j0 < r ? j0 : 0) * p.cols + (kb0 + sb0) * 64 + 16 * c;
-                const uint16_t *ar1 = p.A + (int64_t)(j1 < r ? j1 : 0) * p.cols + (kb0 + sb0) * 64 + 16 * c;
+                // ---- an A item: rows 16 jt .. 16 jt + 15 of A (zero past r) over blocks
+                //      [ab0, ab0 + anb) of this CTA's K range, the same MMA ----
+                const int jt = ja / nsubA, sa = ja - jt * nsubA;
+                const int ab0 = nkb * sa / nsubA, anb = nkb * (sa + 1) / nsubA - ab0;
+                const int j0 = 16 * jt + g, j1 = j0 + 8;  // rows past r read as zero
+                const uint16_t *ar0 = p.A + (int64_t)(j0 < r ? j0 : 0) * p.cols + (kb0 + ab0) * 64 + 16 * c;
+                const uint16_t *ar1 = p.A + (int64_t)(j1 < r ? j1 : 0) * p.cols + (kb0 + ab0) * 64 + 16 * c;
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                const int xsh = (ab0 - sb0) * 256;  // X lines of block ab0 relative to this lane's xoff
 #pragma unroll 1
-                for (int b = 0; b < snb; ++b) {
+                for (int b = 0; b < anb; ++b) {
                     const uint4 a00 = j0 < r ? df_ldg128(ar0 + b * 64) : z, a01 = j0 < r ? df_ldg128(ar0 + b * 64 + 8) : z;
                     const uint4 a10 = j1 < r ? df_ldg128(ar1 + b * 64) : z, a11 = j1 < r ? df_ldg128(ar1 + b * 64 + 8) : z;
                     // k pairs 16c + 4 st + {0, 1} and {2, 3}
                     const uint32_t av[4][4] = {{a00.x, a10.x, a00.y, a10.y}, {a00.z, a10.z, a00.w, a10.w},
                                                {a01.x, a11.x, a01.y, a11.y}, {a01.z, a11.z, a01.w, a11.w}};
-                    block_mma((uint32_t)(b * 256), av, acc, false);
+                    block_mma((uint32_t)(xsh + b * 256), av, acc, false);
                 }
             }
             if (!waited) {
@@ -356,9 +386,9 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
                 const uint32_t a0 = slots_s + (uint32_t)(((((li * S + rank) * nsub + sub) * NT) * 32 + lane) * 16);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) cl_st4(cl_map(a0 + nt * kDfPartBytes, (uint32_t)(ts % S)), acc[nt]);
-            } else {  // to every CTA of the cluster
-                const uint32_t a0 =
-                    uslots_s + (uint32_t)((((((ts - Ee) * S + rank) * nsub + sub) * NT) * 32 + lane) * 16);
+            } else {  // to every CTA of the cluster: slot [jt][rank][sa]
+                const int jt = ja / nsubA, sa = ja - jt * nsubA;
+                const uint32_t a0 = uslots_s + (uint32_t)(((((jt * S + rank) * nsubA + sa) * NT) * 32 + lane) * 16);
 #pragma unroll 1
                 for (int q = 0; q < S; ++q)
 #pragma unroll
@@ -369,7 +399,6 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
         cp_async_wait<0>();  // this thread's B-row copies of the epoch have landed
         cl_arrive();
         cl_wait();  // every partial of the epoch has landed here
-
         // ---- 3. folds -----------------------------------------------------------------------
         if (e == 0) {  // U, in the order (rank, sub-range); every CTA keeps bf16(s U)
             const bool wu = p.U_out != nullptr && cl == 0 && rank == 0;
@@ -377,14 +406,21 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
             for (int pc = warp; pc < p.JT * NT; pc += kDfWarps) {
                 const int jt = pc / NT, nt = pc - jt * NT;
                 float f[4] = {0.f, 0.f, 0.f, 0.f};
-                const float4 *sl = reinterpret_cast<const float4 *>(dsm + p.off_uslots) + (jt * S * nsub * NT + nt) * 32 + lane;
+                const float4 *sl = reinterpret_cast<const float4 *>(dsm + p.off_uslots) + (jt * S * nsubA * NT + nt) * 32 + lane;
+                const int np = S * nsubA;
 #pragma unroll 1
-                for (int q = 0; q < S * nsub; ++q) {
-                    const float4 v = sl[q * NT * 32];
-                    f[0] = __fadd_rn(f[0], v.x);
-                    f[1] = __fadd_rn(f[1], v.y);
-                    f[2] = __fadd_rn(f[2], v.z);
-                    f[3] = __fadd_rn(f[3], v.w);
+                for (int q0 = 0; q0 < np; q0 += 4) {  // four partials in flight, added in order
+                    float4 v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) v[u] = q0 + u < np ? sl[(q0 + u) * NT * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (q0 + u < np) {
+                            f[0] = __fadd_rn(f[0], v[u].x);
+                            f[1] = __fadd_rn(f[1], v[u].y);
+                            f[2] = __fadd_rn(f[2], v[u].z);
+                            f[3] = __fadd_rn(f[3], v[u].w);
+                        }
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {  // U^T[j][t]: j = 16 jt + g (+8), t = 8 nt + 2c (+1)
@@ -406,15 +442,23 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
 #pragma unroll
                 for (int q = 0; q < 4; ++q) f[nt][q] = 0.f;
             const float4 *sl = reinterpret_cast<const float4 *>(dsm + p.off_slots) + (li * S * nsub * NT) * 32 + lane;
+            const int np = S * nsub;
 #pragma unroll 1
-            for (int q = 0; q < S * nsub; ++q) {
+            for (int q0 = 0; q0 < np; q0 += 4) {  // four partials in flight, added in order
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const float4 v = sl[(q * NT + nt) * 32];
-                    f[nt][0] = __fadd_rn(f[nt][0], v.x);
-                    f[nt][1] = __fadd_rn(f[nt][1], v.y);
-                    f[nt][2] = __fadd_rn(f[nt][2], v.z);
-                    f[nt][3] = __fadd_rn(f[nt][3], v.w);
+                    float4 v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        v[u] = q0 + u < np ? sl[((q0 + u) * NT + nt) * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (q0 + u < np) {
+                            f[nt][0] = __fadd_rn(f[nt][0], v[u].x);
+                            f[nt][1] = __fadd_rn(f[nt][1], v[u].y);
+                            f[nt][2] = __fadd_rn(f[nt][2], v[u].z);
+                            f[nt][3] = __fadd_rn(f[nt][3], v[u].w);
+                        }
                 }
             }
 #pragma unroll 1
@@ -459,7 +503,7 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
 
 // ---- host: plan and launch --------------------------------------------------------------
 struct DfLayout {
-    int S, Q, nsub, nkb_max, RS, E, JT;
+    int S, Q, nsub, nsubA, nkb_max, RS, E, JT;
     int off_ring, off_slots, off_uslots, off_sb, off_su, off_ah, off_bar;
     size_t smem;
 };
@@ -476,7 +520,7 @@ static bool df_fit(DfLayout &L, int NT, int r) {
     L.off_slots = (int)off;
     off += df_a128(own * L.S * L.nsub * part);
     L.off_uslots = (int)off;
-    off += df_a128((int64_t)L.JT * L.S * L.nsub * part);
+    off += df_a128((int64_t)L.JT * L.S * L.nsubA * part);
     L.off_sb = (int)off;
     off += df_a128(own * 16 * r * 2);
     L.off_su = (int)off;
@@ -489,8 +533,8 @@ static bool df_fit(DfLayout &L, int NT, int r) {
     return off <= (int64_t)kDfSmemMax;
 }
 
-// Plan for one cluster size S given Q clusters: sub-ranges, epoch size and
-// ring depth.  Returns false if no layout fits.
+// Plan for one cluster size S given Q clusters: sub-ranges, A sub-ranges and
+// epoch size.  Returns false if no layout fits.
 static bool df_plan_s(int64_t T, int64_t KB, int r, int NT, int S, int64_t Q, DfLayout &L) {
     L.S = S;
     L.Q = (int)Q;
@@ -499,18 +543,20 @@ static bool df_plan_s(int64_t T, int64_t KB, int r, int NT, int S, int64_t Q, Df
     if (S > KB || (int64_t)8 * NT * L.nkb_max > kDfXLines || Q < 1) return false;
     const int64_t m = (T + Q - 1) / Q;
     const int64_t nkb_min = KB / S;
+    // A items (U): at most 32, ideally enough sub-ranges of one block or more for every warp to
+    // take one; fewer when their partials do not fit
+    int nsubA0 = (int)(nkb_min < kDfWarps ? nkb_min : kDfWarps);
+    while (nsubA0 > 1 && L.JT * nsubA0 > 2 * kDfWarps) nsubA0 /= 2;
     // sub-ranges: fewest code boxes per warp (items of the first epoch spread
     // over 16 warps; a box carries 4 blocks whether or not all are used), ties
-    // to fewer sub-ranges (fewer partials to fold), among the
-    // counts whose layout fits; then the largest epoch (all tiles when
-    // possible) and the deepest ring
+    // to fewer sub-ranges (fewer partials to fold), among the counts whose
+    // layout fits; then the largest epoch, the largest A split, the deepest ring
     int64_t done = 0;  // costs already tried are below this
     for (;;) {
         int best_ns = 0;
         int64_t best_cost = -1;
         for (int ns = 1; ns <= kDfWarps && ns <= nkb_min; ns *= 2) {
-            const int64_t items = (m + L.JT) * ns;
-            const int64_t cost = ((items + kDfWarps - 1) / kDfWarps) * (((L.nkb_max + ns - 1) / ns + 3) / 4);
+            const int64_t cost = ((m * ns + kDfWarps - 1) / kDfWarps) * (((L.nkb_max + ns - 1) / ns + 3) / 4);
             if (cost >= done && (best_cost < 0 || cost < best_cost)) {
                 best_cost = cost;
                 best_ns = ns;
@@ -518,15 +564,16 @@ static bool df_plan_s(int64_t T, int64_t KB, int r, int NT, int S, int64_t Q, Df
         }
         if (best_ns == 0) return false;
         for (int ns = best_ns; ns <= kDfWarps && ns <= nkb_min; ns *= 2) {
-            const int64_t items = (m + L.JT) * ns;
-            if (((items + kDfWarps - 1) / kDfWarps) * (((L.nkb_max + ns - 1) / ns + 3) / 4) != best_cost) continue;
+            if (((m * ns + kDfWarps - 1) / kDfWarps) * (((L.nkb_max + ns - 1) / ns + 3) / 4) != best_cost) continue;
             L.nsub = ns;
             for (int64_t E = m; E >= 1; --E)
-                for (int rs = 4; rs >= 2; --rs) {
-                    L.E = (int)E;
-                    L.RS = rs;
-                    if (df_fit(L, NT, r)) return true;
-                }
+                for (int nsa = nsubA0; nsa >= 1; nsa /= 2)
+                    for (int rs = 4; rs >= 2; --rs) {
+                        L.nsubA = nsa;
+                        L.E = (int)E;
+                        L.RS = rs;
+                        if (df_fit(L, NT, r)) return true;
+                    }
         }
         done = best_cost + 1;
     }
@@ -614,6 +661,7 @@ static cudaError_t launch_df(DfParams p, const qln_nf4_weight *w, cudaStream_t s
     p.S = best.S;
     p.Q = best.Q;
     p.nsub = best.nsub;
+    p.nsubA = best.nsubA;
     p.nkb_max = best.nkb_max;
     p.RS = best.RS;
     p.E = best.E;

@@ -41,18 +41,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test with a suspend-time hint: a thread whose phase is not complete
+// is parked (it issues nothing) until the phase completes or about `hint_ns`
+// have passed, so waiting warps leave the issue slots to working ones.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: gives up after `limit_ns` of global time, or as soon as
 // *abort is set by another thread of the CTA.  Returns false on give-up.
+// Each test parks the thread for up to 20 us while the phase is incomplete.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort,
                                                   uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0u) {
-            if (abort && *abort) return false;
-            if (global_timer_ns() - t0 > limit_ns) return false;
-        }
+    for (;;) {
+        if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+        if (abort && *abort) return false;
+        if (global_timer_ns() - t0 > limit_ns) return false;
     }
 }
 
