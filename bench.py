@@ -83,6 +83,15 @@ def _workload(name):
     return {"prefill": synthetic.PREFILL, "large": synthetic.LARGE, "pr1": synthetic.PR1}[name]
 
 
+def l2_note(cfg, nsets):
+    """How the timed step relates to the 126 MB L2: the fp32 weight of one
+    input set and whether the rotating sets defeat the cache."""
+    w_mb = cfg.dout * cfg.din * 4 / 1e6
+    if w_mb > 126:
+        return f"{nsets} rotating input sets (W0 fp32 alone {w_mb:.0f} MB > 126 MB L2)"
+    return f"{nsets} rotating input sets; W0 fp32 {w_mb:.1f} MB fits in the 126 MB L2 (launch-bound layer, not L2-defeated)"
+
+
 def codec_bytes_per_param():
     """Algorithmic bytes per parameter: quantize + DQ reads fp32 W0 and writes
     codes, rhat and the group scales; dequant reads those and writes BF16."""
@@ -368,6 +377,89 @@ def measure_sweep(api, dev, use_graph=True):
             "dequant_ms": td * 1e3, "dequant_GBs": params * db / td / 1e9}
 
 
+def measure_layer(api, dev, cfg, nsets=2, reps=4):
+    """One layer's rows (quantize + DQ, dequant, forward, backward) on its own
+    inputs: `nsets` input sets of the layer's shapes and distributions
+    (seeded torch CUDA generators), each row captured as one CUDA graph of
+    `reps` calls over the rotating sets and replayed 3 times between CUDA
+    events; reported per call.  Used for the large layer (28672 x 8192,
+    4096 tokens, r = 64), whose fp32 weight (940 MB) alone is far above L2."""
+    import torch
+    numel = cfg.dout * cfg.din
+    nb = numel // 64
+    gen = torch.Generator(device=dev)
+    sets = []
+    for i in range(nsets):
+        gen.manual_seed(9000 + 10 * cfg.index + i)
+        W = torch.randn(cfg.dout, cfg.din, generator=gen, device=dev) * cfg.w_sigma
+        if cfg.outlier_rate > 0:
+            m = torch.rand(cfg.dout, cfg.din, generator=gen, device=dev) < cfg.outlier_rate
+            W = torch.where(m, W * 10.0, W)
+            del m
+        X = torch.randn(cfg.n, cfg.din, generator=gen, device=dev).to(torch.bfloat16)
+        A = (torch.randn(cfg.r, cfg.din, generator=gen, device=dev) * cfg.ab_sigma).to(torch.bfloat16)
+        B = (torch.randn(cfg.dout, cfg.r, generator=gen, device=dev) * cfg.ab_sigma).to(torch.bfloat16)
+        dY = torch.randn(cfg.n, cfg.dout, generator=gen, device=dev).to(torch.bfloat16)
+        sets.append((W.contiguous(), X, A, B, dY))
+    codes = torch.empty(numel // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(nb, dtype=torch.float32, device=dev)
+    qabs = torch.empty(nb, dtype=torch.int8, device=dev)
+    scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+    mu = torch.empty(1, dtype=torch.float32, device=dev)
+    wdq = torch.empty(cfg.dout, cfg.din, dtype=torch.bfloat16, device=dev)
+    Y = torch.empty(cfg.n, cfg.dout, dtype=torch.bfloat16, device=dev)
+    U = torch.empty(cfg.n, cfg.r, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(cfg.n, cfg.din, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(cfg.r, cfg.din, dtype=torch.float32, device=dev)
+    dB = torch.empty(cfg.dout, cfg.r, dtype=torch.float32, device=dev)
+    ws_dq = api.alloc_workspace(api.workspace_bytes(api.OP_DOUBLE_QUANT, nb), dev)
+    ws_f = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_FWD, cfg.dout, cfg.din, cfg.n, cfg.r), dev)
+    ws_b = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_BWD, cfg.dout, cfg.din, cfg.n, cfg.r), dev)
+    wq = api.NF4Weight(codes=codes, rows=cfg.dout, cols=cfg.din, absmax=absmax, qabs=qabs, dq_scale=scale, dq_mean=mu)
+    api.nf4_quantize(sets[0][0], codes, absmax)
+    api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)
+    rows = {
+        "quantize_dq": lambda i: (api.nf4_quantize(sets[i % nsets][0], codes, absmax),
+                                  api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)),
+        "dequant": lambda i: api.nf4_dequant(wq, wdq),
+        "fwd": lambda i: api.qlora_linear_fwd(wq, *sets[i % nsets][1:4], cfg.s, Y=Y, U_out=U, ws=ws_f),
+        "bwd": lambda i: api.qlora_linear_bwd(wq, *sets[i % nsets][1:4], cfg.s, sets[i % nsets][4], U=U, dX=dX,
+                                              dA=dA, dB=dB, ws=ws_b),
+    }
+    stream = torch.cuda.current_stream()
+    ms = {}
+    for k, fn in rows.items():
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for i in range(reps):
+                fn(i)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(reps):
+                fn(i)
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        del g
+        ms[k] = e0.elapsed_time(e1) / (3 * reps)
+    qb, db = codec_bytes_per_param()
+    out = {"ms": ms, "fwd_TFLOPs": cfg.fwd_flops() / (ms["fwd"] * 1e-3) / 1e12,
+           "bwd_TFLOPs": cfg.bwd_flops() / (ms["bwd"] * 1e-3) / 1e12,
+           "quantize_dq_GBs": numel * qb / (ms["quantize_dq"] * 1e-3) / 1e9,
+           "dequant_GBs": numel * db / (ms["dequant"] * 1e-3) / 1e9,
+           "timing": f"CUDA graph of {reps} calls over {nsets} input sets, 3 replays"}
+    del sets
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------------------
 # GPU leg
 # ---------------------------------------------------------------------------
@@ -625,7 +717,7 @@ def run_ours(args):
                       "global_batch": cfg.n * world, "parallelism": f"dp{world}",
                       "step": "nf4_quantize+nf4_double_quant+nf4_dequant+qlora_linear_fwd+qlora_linear_bwd"
                               "+qln_adamw_step(A,B)",
-                      "l2": "3 rotating input sets (W0 fp32 alone 180 MB > 126 MB L2)",
+                      "l2": l2_note(cfg, NSETS),
                       "timing": "python-enqueued steps" if args.no_graph else
                       "CUDA graph replay per step (one graph per input set)"},
            "gpu_launches": launches, "roofline": roof, "parts": parts, "clocks": clk.summary(),
@@ -636,6 +728,13 @@ def run_ours(args):
         parts["decode_4096x4096_r16"] = measure_decode(api, dev)
         for k, v in parts["decode_4096x4096_r16"].items():
             v["frac_hbm"] = v["GBs"] / peaks["hbm_gbs"]
+        lg = measure_layer(api, dev, synthetic.LARGE)
+        lg["fwd_frac_bf16"] = lg["fwd_TFLOPs"] / peaks["bf16_tflops"]
+        lg["bwd_frac_bf16"] = lg["bwd_TFLOPs"] / peaks["bf16_tflops"]
+        lg["quantize_dq_frac_hbm"] = lg["quantize_dq_GBs"] / peaks["hbm_gbs"]
+        lg["dequant_frac_hbm"] = lg["dequant_GBs"] / peaks["hbm_gbs"]
+        lg["roofline_traffic"] = _recorded_traffic(synthetic.LARGE.name)
+        parts["large_28672x8192_n4096_r64"] = lg
         sw = measure_sweep(api, dev, use_graph=not args.no_graph)
         sw["quantize_dq_frac_hbm"] = sw["quantize_dq_GBs"] / peaks["hbm_gbs"]
         sw["dequant_frac_hbm"] = sw["dequant_GBs"] / peaks["hbm_gbs"]

@@ -216,6 +216,19 @@ def nf4_double_quant_noalloc(absmax: torch.Tensor, qabs, dq_scale, dq_mean):
     """nf4_double_quant into caller-provided outputs, with no device workspace:
     for callers that cannot allocate device memory (see the header)."""
     nb = absmax.numel()
+    # the library writes nb codes, ceil(nb / 256) scales and one mean through
+    # raw pointers: check dtypes, sizes, layout and device here
+    ng = (nb + 255) // 256
+    for name, t, dt, need in (("absmax", absmax, torch.float32, nb), ("qabs", qabs, torch.int8, nb),
+                              ("dq_scale", dq_scale, torch.float32, ng), ("dq_mean", dq_mean, torch.float32, 1)):
+        if t.dtype != dt:
+            raise ValueError(f"{name} must be {dt}, got {t.dtype}")
+        if t.numel() < need:
+            raise ValueError(f"{name} holds {t.numel()} elements, needs {need}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.device != absmax.device:
+            raise ValueError(f"{name} is on {t.device}, absmax on {absmax.device}")
     _need_cuda(absmax, qabs, dq_scale, dq_mean)
     _check("nf4_double_quant_noalloc", lib().nf4_double_quant_noalloc(_p(absmax), nb, _p(qabs), _p(dq_scale),
                                                                       _p(dq_mean), _stream()))

@@ -44,12 +44,8 @@ def lib():
         L.oracle_nf4_nearest.argtypes = [ctypes.c_float, P]
         L.oracle_nf4_quantize.restype = None
         L.oracle_nf4_quantize.argtypes = [P, I64, P, P, P]
-        L.oracle_pairwise_sum.restype = ctypes.c_double
-        L.oracle_pairwise_sum.argtypes = [P, I64]
-        L.oracle_dq_mean.restype = ctypes.c_float
-        L.oracle_dq_mean.argtypes = [P, I64]
         L.oracle_nf4_double_quant.restype = None
-        L.oracle_nf4_double_quant.argtypes = [P, I64, P, P, P]
+        L.oracle_nf4_double_quant.argtypes = [P, I64, ctypes.c_float, P, P]
         L.oracle_dq_restore.restype = ctypes.c_float
         L.oracle_dq_restore.argtypes = [ctypes.c_int8, ctypes.c_float, ctypes.c_float]
         L.oracle_bf16_rn.restype = ctypes.c_uint16
@@ -63,7 +59,7 @@ def lib():
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
         L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         L.oracle_nf4_double_quant_e4m3.restype = None
-        L.oracle_nf4_double_quant_e4m3.argtypes = [P, I64, P, P, P]
+        L.oracle_nf4_double_quant_e4m3.argtypes = [P, I64, ctypes.c_float, P, P]
         L.oracle_dq_restore_e4m3.restype = ctypes.c_float
         L.oracle_dq_restore_e4m3.argtypes = [ctypes.c_uint8, ctypes.c_float, ctypes.c_float]
         L.oracle_nf4_dequant_fmt.restype = None
@@ -181,14 +177,58 @@ def quantize16(bits, kind: str):
     return quantize(widen16(bits, kind))
 
 
-def pairwise_sum(a) -> float:
-    a = _c(a, np.float32).reshape(-1)
-    return lib().oracle_pairwise_sum(_ptr(a), a.size)
+def exact_sum_units(a) -> int:
+    """The exact sum of binary32 values, as an integer count of 2^-149.
+
+    Every finite binary32 value is m * 2^(s - 149) with an integer m < 2^24
+    and s = max(exponent field, 1) - 1 (subnormals have s = 0), so the sum is
+    the integer sum of m * 2^s: summed exactly per exponent (numpy int64, at
+    most 2^24 per term), then shifted into one Python integer."""
+    bits = _c(a, np.float32).reshape(-1).view(np.uint32)
+    e = ((bits >> 23) & 0xFF).astype(np.int64)
+    f = (bits & 0x7FFFFF).astype(np.int64)
+    m = np.where(e > 0, f | 0x800000, f)
+    m = np.where((bits >> 31) == 1, -m, m)
+    s = np.maximum(e, 1) - 1
+    total = 0
+    for sv in np.unique(s):
+        total += int(m[s == sv].sum(dtype=np.int64)) << int(sv)
+    return total
+
+
+def nearest_f32(num: int, den: int) -> np.float32:
+    """The binary32 value nearest to (num / den) * 2^-149, ties to even.
+
+    Binary32 values below 2^-125 are the integers 0 .. 2^24 in units of
+    2^-149 and their bit pattern is that integer; above, a value with leading
+    bit p (p >= 24) keeps 24 significant bits, a quantum of 2^(p - 23) units,
+    and has exponent field p - 22 (a significand that rounds up to 2^24 carries
+    into the exponent through the same formula)."""
+    if den <= 0:
+        raise ValueError("den must be positive")
+    neg = num < 0
+    num = -num if neg else num
+    p = num // den
+    p = p.bit_length() - 1 if p > 0 else -1   # leading bit of floor(num / den)
+    shift = max(0, p - 23)
+    d = den << shift                          # quantum of 2^shift units
+    k, rem = divmod(num, d)
+    if 2 * rem > d or (2 * rem == d and (k & 1)):
+        k += 1
+    bits = k if shift == 0 else ((shift + 1) << 23) + (k - (1 << 23))
+    if bits >= 0x7F800000:
+        bits = 0x7F800000                     # beyond the largest finite value
+    return np.array([bits | (0x80000000 if neg else 0)], np.uint32).view(np.float32)[0]
 
 
 def dq_mean(absmax) -> np.float32:
+    """mu of the double quantization: the mean of the block constants
+    ("LoRA 与 QLoRA", section 2, DQ: subtract the mean mu; mu kept in 32 bits),
+    read as the binary32 value nearest to the exact mean, ties to even."""
     a = _c(absmax, np.float32).reshape(-1)
-    return np.float32(lib().oracle_dq_mean(_ptr(a), a.size))
+    if a.size < 1:
+        raise ValueError("no block constants")
+    return nearest_f32(exact_sum_units(a), a.size)
 
 
 def double_quant(absmax, fmt: str = "int8"):
@@ -203,16 +243,16 @@ def double_quant(absmax, fmt: str = "int8"):
     nb = a.size
     ng = (nb + DQ_GROUP - 1) // DQ_GROUP
     scale = np.zeros(ng, np.float32)
-    mu = np.zeros(1, np.float32)
+    mu = dq_mean(a)
     if fmt == "int8":
         qabs = np.zeros(nb, np.int8)
-        lib().oracle_nf4_double_quant(_ptr(a), nb, _ptr(qabs), _ptr(scale), _ptr(mu))
+        lib().oracle_nf4_double_quant(_ptr(a), nb, ctypes.c_float(mu), _ptr(qabs), _ptr(scale))
     elif fmt == "e4m3":
         qabs = np.zeros(nb, np.uint8)
-        lib().oracle_nf4_double_quant_e4m3(_ptr(a), nb, _ptr(qabs), _ptr(scale), _ptr(mu))
+        lib().oracle_nf4_double_quant_e4m3(_ptr(a), nb, ctypes.c_float(mu), _ptr(qabs), _ptr(scale))
     else:
         raise ValueError(fmt)
-    return qabs, scale, mu[0]
+    return qabs, scale, mu
 
 
 def e4m3_value(code: int) -> float:

@@ -141,28 +141,9 @@ void oracle_nf4_quantize(const float *w, int64_t numel, const float cb[16],
 /* O3. Double quantization of the block constants (groups of 256).          */
 /* ------------------------------------------------------------------------ */
 
-/* S = sum of a_j as a perfect binary tree in binary64: the leaves are
- * (double)a_j, zero-padded to the next power of two, and each level adds
- * adjacent pairs.  A fixed tree makes mu reproducible bit for bit. */
-double oracle_pairwise_sum(const float *a, int64_t n) {
-    if (n <= 0) return 0.0;
-    int64_t p = 1;
-    while (p < n) p <<= 1;
-    double *buf = (double *)calloc((size_t)p, sizeof(double));
-    for (int64_t i = 0; i < n; ++i) buf[i] = (double)a[i];
-    for (int64_t len = p; len > 1; len >>= 1)
-        for (int64_t i = 0; i < len / 2; ++i) buf[i] = buf[2 * i] + buf[2 * i + 1];
-    double s = buf[0];
-    free(buf);
-    return s;
-}
-
-/* mu = mean of all a_j [P1 DQ: subtract the mean mu]: binary32 of S / nb,
- * the division done in binary64. */
-float oracle_dq_mean(const float *absmax, int64_t nb) {
-    double s = oracle_pairwise_sum(absmax, nb);
-    return (float)(s / (double)nb);
-}
+/* mu, the mean of the a_j, is computed exactly by the Python front end
+ * (oracle/codec.py, dq_mean) and passed in: the binary32 value nearest to the
+ * exact mean, ties to even. */
 
 /* [P1 DQ] r_j = (a_j - mu) / b, r_j quantized to 8 bits as rhat_j,
  * restored as ahat_j = mu + b * rhat_j; mu and b kept in 32 bits.
@@ -174,10 +155,8 @@ float oracle_dq_mean(const float *absmax, int64_t nb) {
  *   b_g   = fp32(B_g / 127)
  *   rhat  = clamp(rint(fp32(d_j / b_g)), -127, 127), ties to even; 0 if b_g == 0.
  * The final group may be partial. */
-void oracle_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs,
-                             float *scale, float *mu_out) {
-    float mu = oracle_dq_mean(absmax, nb);
-    *mu_out = mu;
+void oracle_nf4_double_quant(const float *absmax, int64_t nb, float mu, int8_t *qabs,
+                             float *scale) {
     int64_t ng = (nb + 255) / 256;
     for (int64_t g = 0; g < ng; ++g) {
         int64_t j0 = g * 256, j1 = j0 + 256 < nb ? j0 + 256 : nb;
@@ -240,10 +219,8 @@ uint8_t oracle_e4m3_encode(float x) {
  *   d_j   = fp32(a_j - mu)
  *   b_g   = fp32(max_{j in g} |d_j| / 448)        (448: the largest E4M3 value)
  *   rhat  = E4M3(fp32(d_j / b_g)), nearest-even, saturating; code 0 if b_g == 0. */
-void oracle_nf4_double_quant_e4m3(const float *absmax, int64_t nb, uint8_t *qabs,
-                                  float *scale, float *mu_out) {
-    float mu = oracle_dq_mean(absmax, nb);
-    *mu_out = mu;
+void oracle_nf4_double_quant_e4m3(const float *absmax, int64_t nb, float mu, uint8_t *qabs,
+                                  float *scale) {
     int64_t ng = (nb + 255) / 256;
     for (int64_t g = 0; g < ng; ++g) {
         int64_t j0 = g * 256, j1 = j0 + 256 < nb ? j0 + 256 : nb;

@@ -178,3 +178,23 @@ def test_dequant_flat_and_format_argument_errors(L):
     bad.dq_format = 9                                                            # neither INT8 nor E4M3
     assert L.nf4_dequant(ctypes.byref(bad), out, None) == 2
     assert L.nf4_dequant_flat(ctypes.byref(bad), 64, out, None) == 2
+
+
+def test_noalloc_binding_rejects_wrong_dtypes_and_short_outputs():
+    """The binding of the allocation-free double quantization checks what the
+    library will write through raw pointers before calling it."""
+    import pytest
+    import torch
+    from bit_nf4_quantized_07_b200 import api
+    nb = 1000
+    ok = dict(absmax=torch.zeros(nb), qabs=torch.zeros(nb, dtype=torch.int8),
+              dq_scale=torch.zeros(4), dq_mean=torch.zeros(1))
+    bad = [dict(ok, absmax=torch.zeros(nb, dtype=torch.float64)),
+           dict(ok, qabs=torch.zeros(nb, dtype=torch.uint8)),
+           dict(ok, qabs=torch.zeros(nb - 1, dtype=torch.int8)),
+           dict(ok, dq_scale=torch.zeros(3)),
+           dict(ok, dq_mean=torch.zeros(0)),
+           dict(ok, dq_scale=torch.zeros(8)[::2])]
+    for kw in bad:
+        with pytest.raises(ValueError):
+            api.nf4_double_quant_noalloc(**kw)

@@ -48,28 +48,55 @@ def test_bits_per_param_closed_forms_against_actual_byte_counts():
     assert round(saving_gb) == p["saving_65b_gb"]
 
 
-def test_mean_within_one_ulp_of_exact_rational_mean():
-    for seed, nb in ((31, 4096), (32, 1000), (33, 1), (34, 70001)):
+def test_mean_is_the_nearest_binary32_to_the_exact_mean():
+    """mu is the mean of the block constants kept in 32 bits: the binary32
+    value nearest to the exact rational mean, ties to even.  Checked against
+    an independent exact sum (Python fractions of every value) and a rounding
+    of that rational by bisection over the binary32 grid."""
+    def nearest_by_search(x: Fraction) -> np.float32:
+        f = np.float32(float(x))  # within one ulp of x
+        best = None
+        for cand in (np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))):
+            d = abs(Fraction(float(cand)) - x)
+            key = (d, int(np.array([cand], np.float32).view(np.uint32)[0]) & 1)
+            if best is None or key < best[0]:
+                best = (key, cand)
+        return best[1]
+    for seed, nb in ((31, 4096), (32, 1000), (33, 1), (34, 70001), (36, 3)):
         a = np.abs(synthetic.normal_f32(nb, 0.02, seed))
-        mu = codec.dq_mean(a)
         exact = sum((Fraction(float(x)) for x in a), Fraction(0)) / nb
-        ulp = np.spacing(np.float32(abs(float(exact))))
-        assert abs(Fraction(float(mu)) - exact) <= Fraction(float(ulp))
+        assert codec.dq_mean(a) == nearest_by_search(exact)
 
 
-def test_pairwise_tree_sum():
-    # integers: every partial sum exact, so any tree gives the exact sum
-    a = np.arange(1, 1001, dtype=np.float32)
-    assert codec.pairwise_sum(a) == 500500.0
-    # a pair-order probe: 2^24 and the ones are not associative in fp32, but
-    # the binary64 tree adds them exactly
-    a = np.array([2.0 ** 24, 1.0, 1.0, 1.0, 1.0], np.float32)
-    assert codec.pairwise_sum(a) == 2.0 ** 24 + 4
-    # against an exact reference within binary64 pairwise-summation error
-    g = synthetic.normal_f32(12345, 1.0, 35)
-    s = codec.pairwise_sum(g)
-    exact = math.fsum(float(x) for x in g)
-    assert abs(s - exact) <= 14 * np.finfo(np.float64).eps * float(np.sum(np.abs(g.astype(np.float64))))
+def test_mean_closed_forms_and_ties():
+    f32 = np.float32
+    u = 2.0 ** -23
+    cases = [
+        ([0.25] * 5, 0.25),                              # a constant
+        ([1.0, 1.0 + u], 1.0),                           # exact midpoint, even neighbour below
+        ([1.0 + u, 1.0 + 2 * u], 1.0 + 2 * u),           # exact midpoint, even neighbour above
+        ([2.0 ** -149, 0.0], 0.0),                       # half of the smallest subnormal: tie to 0
+        ([2.0 ** -149, 2.0 ** -149, 0.0], 2.0 ** -149),  # two thirds of it: rounds up
+        ([-1.0, 3.0], 1.0),                              # signs
+        ([float(np.finfo(np.float32).max)] * 2, float(np.finfo(np.float32).max)),  # the exact sum overflows fp32
+        ([0.1] * 1000, float(f32(0.1))),                 # a repeated binary32 value
+    ]
+    for vals, want in cases:
+        assert codec.dq_mean(np.array(vals, f32)) == f32(want), vals
+
+
+def test_binary32_rounding_of_exact_rationals_matches_numpy_casts():
+    """nearest_f32 rounds an exact rational; for rationals that are binary64
+    values, numpy's float64 -> float32 cast is that correct rounding."""
+    rng = np.random.Generator(np.random.PCG64(37))
+    x = np.concatenate([rng.standard_normal(2000) * 10.0 ** rng.integers(-40, 38, 2000),
+                        rng.standard_normal(200) * 2.0 ** -140,  # subnormal range
+                        (np.float32(rng.standard_normal(200)).astype(np.float64) +
+                         np.spacing(np.float32(1.0)) / 2)])      # near binary32 midpoints
+    for v in x:
+        fr = Fraction(float(v)) * 2 ** 149
+        got = codec.nearest_f32(fr.numerator, fr.denominator)
+        assert got == np.float32(v), v
 
 
 def test_dq_error_bound_extremes_and_range():
