@@ -1,7 +1,8 @@
 """Benchmark of the QLoRA-linear hot path on B200.
 
 One step = one pass of the whole path over one batch of the layer:
-  nf4_quantize (fp32 W0 -> NF4 codes + absmax) -> nf4_double_quant ->
+  nf4_quantize_dq (fp32 W0 -> NF4 codes + absmax, then the double
+  quantization of the constants, in one call) ->
   nf4_dequant (materialised BF16 W', the standalone decode) ->
   qlora_linear_fwd (U = X A^T, fused NF4 GEMM + adapter) ->
   qlora_linear_bwd (G = dY B, fused dX GEMM, dA, dB).
@@ -337,8 +338,7 @@ def measure_sweep(api, dev, use_graph=True):
 
     def quant_pass():
         for (W, c, a, q, sc, mu) in mats:
-            api.nf4_quantize(W, c, a)
-            api.nf4_double_quant(a, q, sc, mu, ws=ws)
+            api.nf4_quantize_dq(W, c, a, q, sc, mu, ws=ws)
 
     def deq_pass():
         for w in wq:
@@ -416,11 +416,9 @@ def measure_layer(api, dev, cfg, nsets=2, reps=4):
     ws_f = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_FWD, cfg.dout, cfg.din, cfg.n, cfg.r), dev)
     ws_b = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_BWD, cfg.dout, cfg.din, cfg.n, cfg.r), dev)
     wq = api.NF4Weight(codes=codes, rows=cfg.dout, cols=cfg.din, absmax=absmax, qabs=qabs, dq_scale=scale, dq_mean=mu)
-    api.nf4_quantize(sets[0][0], codes, absmax)
-    api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)
+    api.nf4_quantize_dq(sets[0][0], codes, absmax, qabs, scale, mu, ws=ws_dq)
     rows = {
-        "quantize_dq": lambda i: (api.nf4_quantize(sets[i % nsets][0], codes, absmax),
-                                  api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)),
+        "quantize_dq": lambda i: api.nf4_quantize_dq(sets[i % nsets][0], codes, absmax, qabs, scale, mu, ws=ws_dq),
         "dequant": lambda i: api.nf4_dequant(wq, wdq),
         "fwd": lambda i: api.qlora_linear_fwd(wq, *sets[i % nsets][1:4], cfg.s, Y=Y, U_out=U, ws=ws_f),
         "bwd": lambda i: api.qlora_linear_bwd(wq, *sets[i % nsets][1:4], cfg.s, sets[i % nsets][4], U=U, dX=dX,
@@ -535,8 +533,7 @@ def run_ours(args):
 
     def step_body(i):
         W, X, A, B, dYs = sets[i % NSETS]
-        api.nf4_quantize(W, codes, absmax)
-        api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)
+        api.nf4_quantize_dq(W, codes, absmax, qabs, scale, mu, ws=ws_dq)
         api.nf4_dequant(wq, wdq)
         api.qlora_linear_fwd(wq, X, A, B, cfg.s, Y=Y, U_out=U, ws=ws_f)
         api.qlora_linear_bwd(wq, X, A, B, cfg.s, dYs, U=U, dX=dX, dA=dA, dB=dB, ws=ws_b)
@@ -549,8 +546,7 @@ def run_ours(args):
 
     # Rows of the step, for the per-row times.
     rows = {
-        "quantize_dq": lambda i: (api.nf4_quantize(sets[i % NSETS][0], codes, absmax),
-                                  api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)),
+        "quantize_dq": lambda i: api.nf4_quantize_dq(sets[i % NSETS][0], codes, absmax, qabs, scale, mu, ws=ws_dq),
         "quantize": lambda i: api.nf4_quantize(sets[i % NSETS][0], codes, absmax),
         "double_quant": lambda i: api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq),
         "dequant": lambda i: api.nf4_dequant(wq, wdq),
@@ -659,8 +655,7 @@ def run_ours(args):
     def e2e_step():
         for d, h in ((dW, hW), (dXi, hX), (dAi, hA), (dBi, hB), (ddY, hdY)):
             d.copy_(h, non_blocking=True)
-        api.nf4_quantize(dW, codes, absmax)
-        api.nf4_double_quant(absmax, qabs, scale, mu, ws=ws_dq)
+        api.nf4_quantize_dq(dW, codes, absmax, qabs, scale, mu, ws=ws_dq)
         api.nf4_dequant(wq, wdq)
         api.qlora_linear_fwd(wq, dXi, dAi, dBi, cfg.s, Y=Y, U_out=U, ws=ws_f)
         api.qlora_linear_bwd(wq, dXi, dAi, dBi, cfg.s, ddY, U=U, dX=dX, dA=dA, dB=dB, ws=ws_b)
@@ -715,7 +710,7 @@ def run_ours(args):
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
            "config": {"workload": cfg.name, "dout": cfg.dout, "din": cfg.din, "n": cfg.n, "r": cfg.r, "s": cfg.s,
                       "global_batch": cfg.n * world, "parallelism": f"dp{world}",
-                      "step": "nf4_quantize+nf4_double_quant+nf4_dequant+qlora_linear_fwd+qlora_linear_bwd"
+                      "step": "nf4_quantize_dq+nf4_dequant+qlora_linear_fwd+qlora_linear_bwd"
                               "+qln_adamw_step(A,B)",
                       "l2": l2_note(cfg, NSETS),
                       "timing": "python-enqueued steps" if args.no_graph else

@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "QLN_OK", 1: "QLN_ERR_NULL", 2: "QLN_ERR_SHAPE", 3: "QLN_ERR_
 OP_DOUBLE_QUANT, OP_LINEAR_FWD, OP_LINEAR_BWD = 1, 2, 3
 
 #: Every symbol include/qlora_nf4.h declares.
-EXPORTS = ("nf4_quantize", "nf4_quantize_ex", "nf4_double_quant", "nf4_double_quant_ex", "nf4_double_quant_noalloc",
+EXPORTS = ("nf4_quantize", "nf4_quantize_ex", "nf4_quantize_dq", "nf4_double_quant", "nf4_double_quant_ex", "nf4_double_quant_noalloc",
            "nf4_dequant",
            "nf4_dequant_flat", "qlora_linear_fwd", "qlora_linear_bwd", "qln_workspace_bytes", "qln_codebook",
            "qln_status_str", "qln_version", "qln_launch_count", "qln_adamw_step")
@@ -68,6 +68,7 @@ def lib():
         sig = {
             "nf4_quantize": ([P, I64, P, P, P], I32),
             "nf4_quantize_ex": ([P, I32, I64, P, P, P], I32),
+            "nf4_quantize_dq": ([P, I32, I64, I32, P, P, P, P, P, P, SZ, P], I32),
             "nf4_double_quant": ([P, I64, P, P, P, P, SZ, P], I32),
             "nf4_double_quant_ex": ([P, I64, I32, P, P, P, P, SZ, P], I32),
             "nf4_double_quant_noalloc": ([P, I64, P, P, P, P], I32),
@@ -186,6 +187,34 @@ def nf4_quantize(W: torch.Tensor, codes: Optional[torch.Tensor] = None, absmax: 
     return codes, absmax
 
 
+def nf4_quantize_dq(W: torch.Tensor, codes=None, absmax=None, qabs=None, dq_scale=None, dq_mean=None, ws=None,
+                    fmt: str = "int8"):
+    """W (fp32/bf16/fp16) -> (codes, absmax, qabs, dq_scale, dq_mean): nf4_quantize
+    then nf4_double_quant in one call (nf4_quantize_dq), the same bits."""
+    if W.dtype not in _DTYPES:
+        raise ValueError(f"unsupported weight dtype {W.dtype}")
+    n = W.numel()
+    nb = (n + 63) // 64
+    dev = W.device
+    if codes is None:
+        codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev)
+    if absmax is None:
+        absmax = torch.empty(nb, dtype=torch.float32, device=dev)
+    if qabs is None:
+        qabs = torch.empty(nb, dtype=torch.int8 if fmt == "int8" else torch.uint8, device=dev)
+    if dq_scale is None:
+        dq_scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+    if dq_mean is None:
+        dq_mean = torch.empty(1, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = alloc_workspace(workspace_bytes(OP_DOUBLE_QUANT, nb), dev)
+    _need_cuda(W, codes, absmax, qabs, dq_scale, dq_mean, ws)
+    _check("nf4_quantize_dq", lib().nf4_quantize_dq(_p(W), _DTYPES[W.dtype], n, DQ_FORMATS[fmt], _p(codes),
+                                                    _p(absmax), _p(qabs), _p(dq_scale), _p(dq_mean), _p(ws),
+                                                    ws.numel(), _stream()))
+    return codes, absmax, qabs, dq_scale, dq_mean
+
+
 def nf4_double_quant(absmax: torch.Tensor, qabs=None, dq_scale=None, dq_mean=None, ws=None, fmt: str = "int8"):
     """fp32 absmax [nb] -> (qabs [nb], dq_scale fp32 [ceil(nb/256)], dq_mean fp32 [1]).
 
@@ -236,14 +265,15 @@ def nf4_double_quant_noalloc(absmax: torch.Tensor, qabs, dq_scale, dq_mean):
 
 
 def quantize_weight(W: torch.Tensor, double_quant: bool = True, ws=None, dq_format: str = "int8") -> NF4Weight:
-    """nf4_quantize (+ nf4_double_quant in the given 8-bit format) of a
-    [rows][cols] weight (fp32, bf16 or fp16)."""
+    """nf4_quantize_dq (or nf4_quantize alone without double quantization)
+    of a [rows][cols] weight (fp32, bf16 or fp16)."""
     rows, cols = W.shape
+    if double_quant:
+        codes, absmax, qabs, scale, mean = nf4_quantize_dq(W, ws=ws, fmt=dq_format)
+        return NF4Weight(codes=codes, rows=rows, cols=cols, absmax=absmax, qabs=qabs, dq_scale=scale, dq_mean=mean,
+                         dq_format=dq_format)
     codes, absmax = nf4_quantize(W)
     w = NF4Weight(codes=codes, rows=rows, cols=cols, absmax=absmax)
-    if double_quant:
-        w.qabs, w.dq_scale, w.dq_mean = nf4_double_quant(absmax, ws=ws, fmt=dq_format)
-        w.dq_format = dq_format
     return w
 
 

@@ -177,6 +177,25 @@ qln_status nf4_double_quant_ex(const float *absmax, int64_t nb, int32_t dq_forma
                                                      (cudaStream_t)stream, sms));
 }
 
+qln_status nf4_quantize_dq(const void *W, int32_t dtype, int64_t numel, int32_t dq_format, uint8_t *codes,
+                           float *absmax, void *qabs_v, float *dq_scale, float *dq_mean, void *ws, size_t ws_bytes,
+                           void *stream) {
+    int8_t *qabs = static_cast<int8_t *>(qabs_v);
+    if (!W || !codes || !absmax || !qabs || !dq_scale || !dq_mean || !ws) return QLN_ERR_NULL;
+    if (numel <= 0 || (numel + 63) / 64 > qln::dq_max_blocks()) return QLN_ERR_SHAPE;
+    if (dtype != QLN_DTYPE_F32 && dtype != QLN_DTYPE_BF16 && dtype != QLN_DTYPE_F16) return QLN_ERR_SHAPE;
+    if (dq_format != QLN_DQ_INT8 && dq_format != QLN_DQ_E4M3) return QLN_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(absmax, 16) || !aligned(qabs, 4) ||
+        !aligned(dq_scale, 4) || !aligned(dq_mean, 4) || !aligned(ws, 256))
+        return QLN_ERR_ALIGN;
+    if (ws_bytes < qln::dq_workspace_bytes((numel + 63) / 64)) return QLN_ERR_WORKSPACE;
+    int sms = 0;
+    qln_status s = check_device(&sms);
+    if (s != QLN_OK) return s;
+    return from_cuda(qln::launch_nf4_quantize_dq(W, dtype, numel, codes, absmax, qabs, dq_scale, dq_mean, ws,
+                                                    dq_format == QLN_DQ_E4M3, (cudaStream_t)stream, sms));
+}
+
 qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale, float *dq_mean,
                             void *ws, size_t ws_bytes, void *stream) {
     return nf4_double_quant_ex(absmax, nb, QLN_DQ_INT8, qabs, dq_scale, dq_mean, ws, ws_bytes, stream);
@@ -191,7 +210,7 @@ qln_status nf4_double_quant_noalloc(const float *absmax, int64_t nb, int8_t *qab
     int sms = 0;
     qln_status s = check_device(&sms);
     if (s != QLN_OK) return s;
-    return from_cuda(qln::launch_nf4_double_quant_static(absmax, nb, qabs, dq_scale, dq_mean, (cudaStream_t)stream));
+    return from_cuda(qln::launch_nf4_double_quant_static(absmax, nb, qabs, dq_scale, dq_mean, (cudaStream_t)stream, sms));
 }
 
 qln_status nf4_dequant(const qln_nf4_weight *w, uint16_t *out, void *stream) {

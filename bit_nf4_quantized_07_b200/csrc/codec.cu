@@ -7,7 +7,9 @@
 // "LoRA 与 QLoRA" section QLoRA 2 (a_j = max|W_j| per 64 weights,
 // r_j = (a_j - mu)/b, 8-bit rhat_j, ahat_j = mu + b rhat_j).
 #include <atomic>
+#include <mutex>
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 
 #include "qln_common.cuh"
@@ -267,6 +269,283 @@ template <> struct QzIn<F16In> {
     }
 };
 
+// ===========================================================================
+// The DQ mean mu: the binary32 value nearest to the exact mean of the block
+// constants, ties to even ("LoRA 与 QLoRA", section 2: subtract the mean mu;
+// mu is kept in 32 bits).
+//
+// Exact sums.  Every finite binary32 value is an integer number of units of
+// 2^-149: |a| = m * 2^s units with m < 2^24 and s = max(exponent field, 1) - 1
+// in [0, 253].  A sum is held as kXLimbs signed 64-bit limbs, limb k weighing
+// 2^(32 k) units.  A thread keeps a run of values that fall on the same limb
+// pair in one 64-bit word (at most 64 values of < 2^55 each), and a run is
+// added to the limbs as a low part (< 2^32) on limb k and a high part on limb
+// k + 1.  Integer addition is associative, so the result does not depend on the
+// order in which threads, warps or CTAs add their parts, and no limb can
+// overflow for fewer than 2^30 values.
+// ===========================================================================
+constexpr int kXLimbs = 10;  // 320 bits: a value reaches bit 277; the rest holds carries and the sign
+constexpr int64_t kMeanMaxBlocks = (int64_t)1 << 25;  // nb limit (numel 2^31); the limbs stay exact to 2^30
+
+struct XRun {
+    long long acc = 0;  // sum of the run, in units of 2^(32 k)
+    int k = -1;         // limb of the run (-1: empty)
+    int cnt = 0;
+};
+
+__device__ __forceinline__ void xsum_flush_lane(XRun &x, unsigned long long *lim) {
+    if (x.k >= 0 && x.acc != 0) {
+        atomicAdd(&lim[x.k], (unsigned long long)(x.acc & 0xffffffffll));
+        atomicAdd(&lim[x.k + 1], (unsigned long long)(x.acc >> 32));
+    }
+    x.acc = 0;
+    x.k = -1;
+    x.cnt = 0;
+}
+
+// Adds one binary32 value (finite) to this thread's run; a value on another
+// limb pair (rare: the constants of one weight are close in magnitude) first
+// sends the run to the shared limbs.
+__device__ __forceinline__ void xsum_add(XRun &x, float v, unsigned long long *lim) {
+    const uint32_t b = __float_as_uint(v);
+    const int e = (int)((b >> 23) & 0xffu);
+    const uint32_t m = (b & 0x7fffffu) | (e ? 0x800000u : 0u);
+    if (m == 0) return;
+    const int s = (e > 1 ? e : 1) - 1;
+    const int k = s >> 5;
+    if (k != x.k || x.cnt == 64) {
+        xsum_flush_lane(x, lim);
+        x.k = k;
+    }
+    const long long t = (long long)m << (s & 31);
+    x.acc += (b >> 31) ? -t : t;
+    ++x.cnt;
+}
+
+// A warp's runs into the shared limbs: one pair of atomics per warp when every
+// lane's run sits on the same limb pair (the usual case), else one per lane.
+__device__ __forceinline__ void xsum_flush_warp(XRun &x, unsigned long long *lim) {
+    const int kk = x.acc != 0 ? x.k : -1;
+    const int k0 = (int)__reduce_max_sync(0xffffffffu, (unsigned)(kk + 1)) - 1;
+    if (__all_sync(0xffffffffu, kk == -1 || kk == k0)) {
+        long long lo = kk >= 0 ? (x.acc & 0xffffffffll) : 0, hi = kk >= 0 ? (x.acc >> 32) : 0;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            lo += __shfl_xor_sync(0xffffffffu, lo, o);
+            hi += __shfl_xor_sync(0xffffffffu, hi, o);
+        }
+        if ((threadIdx.x & 31) == 0 && k0 >= 0) {
+            atomicAdd(&lim[k0], (unsigned long long)lo);
+            atomicAdd(&lim[k0 + 1], (unsigned long long)hi);
+        }
+        x.acc = 0;
+        x.k = -1;
+        x.cnt = 0;
+    } else {
+        xsum_flush_lane(x, lim);
+    }
+}
+
+// mu = the binary32 value nearest to (limbs / nb) units, ties to even, by one
+// thread.  The limbs are carried into 32-bit digits d (two's complement over
+// the digits for a negative sum) and the magnitude S is cut to its top 64
+// bits, S = T 2^sh + R with T >= 2^63 when sh > 0 (and R < 2^sh), or T = S and
+// sh = 0.  Then S / nb = (T div nb) 2^sh + (rem 2^sh + R) / nb: the quotient
+// q = T div nb has at least 39 bits when sh > 0 (nb < 2^25), and the exact
+// mean has bits below q's last exactly when rem or R is nonzero -- enough for
+// 24 significant bits, the guard bit and the sticky bit, from one 64-bit
+// division.
+__device__ float xsum_mean(const unsigned long long (&limb)[kXLimbs], uint32_t nb) {
+    uint32_t d[kXLimbs];
+    long long carry = 0;
+#pragma unroll
+    for (int k = 0; k < kXLimbs; ++k) {
+        const long long v = (long long)limb[k] + carry;
+        d[k] = (uint32_t)v;
+        carry = (v - (long long)(uint32_t)v) >> 32;
+    }
+    const bool neg = carry < 0;
+    if (neg) {  // magnitude of a negative two's complement number
+        uint32_t c = 1;
+#pragma unroll
+        for (int k = 0; k < kXLimbs; ++k) {
+            const uint64_t t = (uint64_t)(~d[k]) + c;
+            d[k] = (uint32_t)t;
+            c = (uint32_t)(t >> 32);
+        }
+    }
+    int t = 0;  // top nonzero digit (0 for a zero sum)
+#pragma unroll
+    for (int k = 1; k < kXLimbs; ++k)
+        if (d[k] != 0) t = k;
+    uint64_t T;
+    int sh = 0;
+    bool R = false;  // a nonzero bit of S below T
+    if (t < 2) {
+        T = ((uint64_t)d[1] << 32) | d[0];
+    } else {
+        uint32_t d2 = 0, d1 = 0, d0 = 0;
+#pragma unroll
+        for (int k = 2; k < kXLimbs; ++k) {
+            if (k == t) { d2 = d[k]; d1 = d[k - 1]; d0 = d[k - 2]; }
+            if (k < t && d[k - 2] != 0) R = true;  // digits below t - 2
+        }
+        const int z = __clz(d2);  // d2 != 0
+        const uint64_t top = ((uint64_t)d2 << 32) | d1;
+        T = z ? (top << z) | (d0 >> (32 - z)) : top;  // 64 bits from bit 32 t + 31 - z down
+        if (z ? (d0 << z) != 0u : d0 != 0u) R = true;
+        sh = 32 * (t - 2) + 32 - z;
+    }
+    const uint64_t q = T / nb;
+    const uint64_t rem = T - q * nb;
+    const int lb = q ? 63 - __clzll((long long)q) : -1;
+    uint32_t bits;
+    if (sh + lb <= 23) {  // below 2^-125 (then sh == 0): the value in units is the pattern itself
+        uint32_t k = (uint32_t)q;
+        if (2 * rem > nb || (2 * rem == nb && (k & 1u))) ++k;
+        bits = k;
+    } else {
+        const int rs = lb - 23;  // >= 1: q's bits below rs are rounded off
+        const uint32_t sig = (uint32_t)(q >> rs) & 0xffffffu;
+        const uint64_t below = q & ((1ull << rs) - 1);
+        const uint64_t half = 1ull << (rs - 1);
+        const bool guard = (below & half) != 0;
+        const bool sticky = (below & (half - 1)) != 0 || rem != 0 || R;
+        uint32_t m = sig;
+        if (guard && (sticky || (m & 1u))) ++m;
+        const uint64_t b64 = ((uint64_t)(sh + rs + 1) << 23) + m - (1u << 23);
+        bits = b64 >= 0x7f800000ull ? 0x7f800000u : (uint32_t)b64;
+    }
+    return __uint_as_float(bits | (neg ? 0x80000000u : 0u));
+}
+
+// The limbs read by lanes 0..kXLimbs-1 of the calling warp (one coalesced
+// request) and mu formed by lane 0; every lane of the warp must call it.
+__device__ __forceinline__ float xsum_mean_warp(const unsigned long long *glim, uint32_t nb) {
+    const int lane = threadIdx.x & 31;
+    const unsigned long long mine = lane < kXLimbs ? __ldcg(glim + lane) : 0ull;
+    unsigned long long L[kXLimbs];
+#pragma unroll
+    for (int k = 0; k < kXLimbs; ++k) L[k] = __shfl_sync(0xffffffffu, mine, k);
+    return lane == 0 ? xsum_mean(L, nb) : 0.f;
+}
+
+// The DQ scratch (256 bytes): a status word, a generation word, an arrival
+// counter and two banks of limbs.  A call reads the generation g at its start
+// and sums into bank g % 2, which is zero; the last CTA of the call's summing
+// kernel to arrive puts the counter back to zero, zeroes the other bank and
+// then advances the generation, so the next call finds its bank zeroed and
+// nothing has to be cleared after the last reader.
+struct DqScratch {
+    int *status;  // null: none (the allocation-free entry point)
+    unsigned *gen;
+    int *arrive;
+    unsigned long long *bank[2];  // [kXLimbs] each
+};
+constexpr int kDqStatusOffset = 0, kDqGenOffset = 16, kDqArriveOffset = 32, kDqBank0Offset = 64, kDqBank1Offset = 160;
+constexpr size_t kDqScratchBytes = 256;
+static_assert(kDqBank0Offset + 8 * kXLimbs <= kDqBank1Offset && kDqBank1Offset + 8 * kXLimbs <= (int)kDqScratchBytes,
+              "limb banks inside the scratch");
+
+__device__ __forceinline__ DqScratch dq_scratch(unsigned char *ws, bool with_status) {
+    DqScratch d;
+    d.status = with_status ? reinterpret_cast<int *>(ws + kDqStatusOffset) : nullptr;
+    d.gen = reinterpret_cast<unsigned *>(ws + kDqGenOffset);
+    d.arrive = reinterpret_cast<int *>(ws + kDqArriveOffset);
+    d.bank[0] = reinterpret_cast<unsigned long long *>(ws + kDqBank0Offset);
+    d.bank[1] = reinterpret_cast<unsigned long long *>(ws + kDqBank1Offset);
+    return d;
+}
+
+// The generation, read by thread 0 and shared with the CTA (every thread calls).
+__device__ __forceinline__ unsigned dq_read_gen(const DqScratch &sc, unsigned *gen_s) {
+    if (threadIdx.x == 0) *gen_s = __ldcg(sc.gen);
+    __syncthreads();
+    return *gen_s;
+}
+
+// Thread 0, after the CTA's limbs are in bank g % 2: count this CTA in; the
+// last of G to arrive resets the counter, zeroes the other bank and publishes
+// generation g + 1 (a release, after everything it has seen).  Returns whether
+// this CTA was the last.
+__device__ __forceinline__ bool dq_arrive(const DqScratch &sc, unsigned g, int G) {
+    __threadfence();
+    if (atomicAdd(sc.arrive, 1) != G - 1) return false;
+    *sc.arrive = 0;
+    unsigned long long *other = sc.bank[(g + 1) & 1];
+#pragma unroll
+    for (int k = 0; k < kXLimbs; ++k) other[k] = 0ull;
+    __threadfence();
+    atomicExch(sc.gen, g + 1);
+    return true;
+}
+
+// 8 consecutive constants starting at j (zeros past nb).
+__device__ __forceinline__ void load8_const(float (&v)[8], const float *__restrict__ a, int64_t j, int64_t nb) {
+    if (j + 8 <= nb) {
+        const float4 x = __ldg(reinterpret_cast<const float4 *>(a + j));
+        const float4 y = __ldg(reinterpret_cast<const float4 *>(a + j + 4));
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+        v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = (j + i < nb) ? a[j + i] : 0.f;
+    }
+}
+
+// This CTA's constants into its shared limbs, then into the scratch limbs.
+// Every thread of the CTA calls it; on return the CTA's part is published.
+// One group of 256 block constants, one warp, 8 consecutive constants per
+// lane (e, starting at j0): d = fp32(a - mu), b = fp32(max|d| / 127 or 448),
+// rhat = clamp(rint(fp32(d / b)), -127, 127) or E4M3(fp32(d / b)); 0 if b == 0.
+__device__ __forceinline__ void dq_quantize_group(const float (&e)[8], int64_t j0, int64_t nb, float mu, bool e4m3,
+                                                  int lane, int64_t g, int8_t *__restrict__ qabs,
+                                                  float *__restrict__ scale) {
+    float d[8], m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        d[i] = __fsub_rn(e[i], mu);
+        if (j0 + i < nb) m = fmaxf(m, fabsf(d[i]));
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float b = __fdiv_rn(m, e4m3 ? 448.0f : 127.0f);  // 448: the largest E4M3 value
+    if (lane == 0) scale[g] = b;
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t r = 0;
+        if (b != 0.f) {
+            const float x = __fdiv_rn(d[i], b);
+            r = e4m3 ? (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3)  // nearest-even, saturating
+                     : (uint32_t)((int)fminf(fmaxf(rintf(x), -127.f), 127.f) & 0xff);
+        }
+        w[i >> 2] |= (r & 0xffu) << (8 * (i & 3));
+    }
+    if (j0 + 8 <= nb) {
+        *reinterpret_cast<uint32_t *>(qabs + j0) = w[0];
+        *reinterpret_cast<uint32_t *>(qabs + j0 + 4) = w[1];
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (j0 + i < nb) qabs[j0 + i] = (int8_t)((w[i >> 2] >> (8 * (i & 3))) & 0xff);
+    }
+}
+
+// Grid-wide barrier helpers: an acquiring load of a counter, the global timer.
+constexpr uint64_t kDqfWaitNs = 2000000000ull;
+
+__device__ __forceinline__ unsigned dqf_ld_acquire_u32(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint64_t dqf_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 constexpr int kQzWarps = 24;       // two CTAs of 24 warps per SM
 constexpr int kQzCtasPerSm = 2;
 constexpr int kQzStages = 3;       // chunks per warp ring
@@ -283,21 +562,18 @@ constexpr int kQzLutBytes = 256 * 128;                                    // 256
 // raises no absmax and gets code 7, which is what a ragged tail stores); a
 // lane's last partial code word is written byte by byte.  Idx is 32-bit
 // whenever every element offset stays below 2^31.
+
 template <typename T, typename Idx>
 __global__ void __launch_bounds__(kQzThreads, kQzCtasPerSm) nf4_quantize_kernel(const T *__restrict__ W, Idx numel,
                                                                                 uint8_t *__restrict__ codes,
-                                                                                float *__restrict__ absmax,
-                                                                                bool release_early) {
+                                                                                float *__restrict__ absmax) {
     constexpr int kB = QzIn<T>::kBytes;
     extern __shared__ __align__(16) unsigned char qz_smem[];
     for (int i = threadIdx.x; i < kQzLutBytes / 4; i += kQzThreads)  // bucket i/32, lane i%32
         reinterpret_cast<uint32_t *>(qz_smem)[i] = kSnapTable.e[i >> 5];
     __syncthreads();
     pdl_wait();  // W may come from the previous kernel; codes/absmax may still be read by it
-    // This kernel writes a weight (codes, absmax), and a forward may read its
-    // weight before its own dependency wait; so the next kernel is released
-    // early only when it is known to wait first.
-    if (release_early) pdl_trigger();
+    pdl_trigger();
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -373,6 +649,8 @@ __global__ void __launch_bounds__(kQzThreads, kQzCtasPerSm) nf4_quantize_kernel(
     cp_async_wait<0>();
 }
 
+// Launch of the quantize kernel: a persistent grid of up to two CTAs per SM,
+// as a programmatic dependent.
 template <typename T, typename Idx>
 static cudaError_t launch_quantize_t(const T *W, int64_t numel, uint8_t *codes, float *absmax, cudaStream_t st,
                                      int num_sms) {
@@ -381,11 +659,10 @@ static cudaError_t launch_quantize_t(const T *W, int64_t numel, uint8_t *codes, 
     if (grid > (int64_t)kQzCtasPerSm * num_sms) grid = (int64_t)kQzCtasPerSm * num_sms;
     if (grid < 1) grid = 1;
     const int smem = kQzLutBytes + kQzWarps * kQzStages * 256 * QzIn<T>::kBytes;
-    cudaError_t e =
-        cudaFuncSetAttribute(nf4_quantize_kernel<T, Idx>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kern = nf4_quantize_kernel<T, Idx>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(nf4_quantize_kernel<T, Idx>, dim3((unsigned)grid), dim3(kQzThreads), (size_t)smem, st, W,
-                      (Idx)numel, codes, absmax, false);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kQzThreads), (size_t)smem, st, W, (Idx)numel, codes, absmax);
 }
 
 template <typename T>
@@ -407,330 +684,191 @@ cudaError_t launch_nf4_quantize(const void *W, int dtype, int64_t numel, uint8_t
     }
 }
 
-// ===========================================================================
-// K2: partial sums for mu.  CTA c sums the block constants a[C c, C (c+1)) as
-// a perfect binary tree in binary64 (zero-padded), C = 2048 * NG: thread t
-// folds its 8 * NG consecutive leaves (8 at a time, the 8-leaf sums merged
-// like a binary counter, which is the tree order), a warp xor-butterfly adds
-// lane pairs level by level (addition is commutative, so both lanes of a pair
-// hold the same node), and the 8 warp roots are folded pairwise.  The result
-// is exactly the aligned subtree of the whole-tensor tree.  C grows with nb so
-// that there are at most kMaxPartials partial sums.
-// ===========================================================================
-constexpr int kMeanThreads = 256;
-constexpr int kMaxPartials = 1024;
-constexpr int64_t kMeanMaxBlocks = (int64_t)1 << 25;  // nb limit: C <= 32768
-
-__device__ __forceinline__ double tree8(const float (&v)[8]) {
-    const double s01 = __dadd_rn((double)v[0], (double)v[1]), s23 = __dadd_rn((double)v[2], (double)v[3]);
-    const double s45 = __dadd_rn((double)v[4], (double)v[5]), s67 = __dadd_rn((double)v[6], (double)v[7]);
-    return __dadd_rn(__dadd_rn(s01, s23), __dadd_rn(s45, s67));
-}
-
-// 8 consecutive constants starting at j (zeros past nb).
-__device__ __forceinline__ void load8_const(float (&v)[8], const float *__restrict__ a, int64_t j, int64_t nb) {
-    if (j + 8 <= nb) {
-        const float4 x = __ldg(reinterpret_cast<const float4 *>(a + j));
-        const float4 y = __ldg(reinterpret_cast<const float4 *>(a + j + 4));
-        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-        v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
-    } else {
+template <int P>
+__device__ __forceinline__ void dq_add_cta(const float (&e)[P][8], unsigned long long *slim,
+                                           unsigned long long *glim) {
+    XRun x;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = (j + i < nb) ? a[j + i] : 0.f;
+    for (int i = 0; i < P; ++i)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) xsum_add(x, e[i][u], slim);
+    xsum_flush_warp(x, slim);
+    __syncthreads();
+    if (threadIdx.x < kXLimbs && slim[threadIdx.x] != 0ull) atomicAdd(&glim[threadIdx.x], slim[threadIdx.x]);
+}
+
+constexpr int kDqThreads = 256;
+constexpr int kDqGroupsPerCta = kDqThreads / 32;  // one group of 256 constants per warp
+
+// ===========================================================================
+// K2: the exact sum.  Each CTA adds the constants of 8 groups per pass (8 per
+// lane) into its shared limbs and then, with one reduction per nonzero limb,
+// into the call's bank of the scratch; the last CTA to arrive advances the
+// generation.  Nothing waits: K3 reads the bank only after this grid has
+// completed.
+// ===========================================================================
+__global__ void __launch_bounds__(kDqThreads) dq_sum_kernel(const float *__restrict__ a, int64_t nb,
+                                                            unsigned char *ws, bool with_status) {
+    __shared__ unsigned long long slim[kXLimbs];
+    __shared__ unsigned gen_s;
+    if (threadIdx.x < kXLimbs) slim[threadIdx.x] = 0ull;
+    __syncthreads();
+    pdl_wait();  // the constants come from the previous kernel (the quantize)
+    pdl_trigger();
+    const DqScratch sc = dq_scratch(ws, with_status);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && sc.status) *sc.status = QLN_OK;
+    const unsigned g0 = dq_read_gen(sc, &gen_s);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
+    XRun x;
+    for (int64_t g = (int64_t)blockIdx.x * kDqGroupsPerCta + warp; g < ng; g += (int64_t)gridDim.x * kDqGroupsPerCta) {
+        float e[8];
+        load8_const(e, a, g * kDqGroup + 8 * lane, nb);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) xsum_add(x, e[u], slim);
     }
+    xsum_flush_warp(x, slim);
+    __syncthreads();
+    if (threadIdx.x < kXLimbs && slim[threadIdx.x] != 0ull) atomicAdd(&sc.bank[g0 & 1][threadIdx.x], slim[threadIdx.x]);
+    __syncthreads();
+    if (threadIdx.x == 0) dq_arrive(sc, g0, (int)gridDim.x);
 }
 
-__device__ __forceinline__ double warp_butterfly_sum(double s, int levels) {
-    for (int l = 0; l < levels; ++l) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 1 << l));
-    return s;
-}
-
-template <int NG>
-__global__ void __launch_bounds__(kMeanThreads) dq_partial_kernel(const float *__restrict__ a, int64_t nb,
-                                                                  double *__restrict__ partial) {
-    __shared__ double warp_root[kMeanThreads / 32];
+// ===========================================================================
+// K3: the group quantization.  mu is either read (mu_in) or formed here from
+// the bank K2 summed into: warp 0 of every CTA reads the limbs and forms mu
+// while the other warps load their first groups, and CTA 0 writes it out.  The
+// bank is zeroed by the next call's K2 (or single launch), not here.  A warp takes groups warp, warp + 8 gridDim, ... with the next group's
+// constants requested before the current one is quantized.
+// ===========================================================================
+__global__ void __launch_bounds__(kDqThreads) dq_quant_kernel(const float *__restrict__ a, int64_t nb,
+                                                              int8_t *__restrict__ qabs, float *__restrict__ scale,
+                                                              const float *__restrict__ mu_in,
+                                                              float *__restrict__ mu_out, unsigned char *scratch,
+                                                              bool e4m3) {
+    __shared__ float mu_s;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
+    const int64_t gstep = (int64_t)gridDim.x * kDqGroupsPerCta;
+    int64_t g = (int64_t)blockIdx.x * kDqGroupsPerCta + warp;
     pdl_wait();
     pdl_trigger();
-    const int64_t base = ((int64_t)blockIdx.x * kMeanThreads + threadIdx.x) * (8 * NG);
-    float v[NG][8];
-#pragma unroll
-    for (int g = 0; g < NG; ++g) load8_const(v[g], a, base + 8 * g, nb);  // all loads in flight at once
-    double level[5];  // level[k]: a pending subtree of 8 * 2^k leaves (binary counter over g)
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-        double s = tree8(v[g]);
-        int k = 0;
-#pragma unroll
-        for (int t = g; t & 1; t >>= 1, ++k) s = __dadd_rn(level[k], s);
-        level[k] = s;
-    }
-    constexpr int top = NG == 1 ? 0 : NG == 2 ? 1 : NG == 4 ? 2 : NG == 8 ? 3 : 4;
-    const double s = warp_butterfly_sum(level[top], 5);
-    if ((threadIdx.x & 31) == 0) warp_root[threadIdx.x >> 5] = s;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const double w01 = __dadd_rn(warp_root[0], warp_root[1]), w23 = __dadd_rn(warp_root[2], warp_root[3]);
-        const double w45 = __dadd_rn(warp_root[4], warp_root[5]), w67 = __dadd_rn(warp_root[6], warp_root[7]);
-        partial[blockIdx.x] = __dadd_rn(__dadd_rn(w01, w23), __dadd_rn(w45, w67));
-    }
-}
-
-// One group of 256 block constants, one warp, 8 consecutive constants per
-// lane (e, starting at j0): d = fp32(a - mu), b = fp32(max|d| / 127 or 448),
-// rhat = clamp(rint(fp32(d / b)), -127, 127) or E4M3(fp32(d / b)); 0 if b == 0.
-__device__ __forceinline__ void dq_quantize_group(const float (&e)[8], int64_t j0, int64_t nb, float mu, bool e4m3,
-                                                  int lane, int64_t g, int8_t *__restrict__ qabs,
-                                                  float *__restrict__ scale) {
-    float d[8], m = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        d[i] = __fsub_rn(e[i], mu);
-        if (j0 + i < nb) m = fmaxf(m, fabsf(d[i]));
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const float b = __fdiv_rn(m, e4m3 ? 448.0f : 127.0f);  // 448: the largest E4M3 value
-    if (lane == 0) scale[g] = b;
-    uint32_t w[2] = {0u, 0u};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        uint32_t r = 0;
-        if (b != 0.f) {
-            const float x = __fdiv_rn(d[i], b);
-            r = e4m3 ? (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3)  // nearest-even, saturating
-                     : (uint32_t)((int)fminf(fmaxf(rintf(x), -127.f), 127.f) & 0xff);
-        }
-        w[i >> 2] |= (r & 0xffu) << (8 * (i & 3));
-    }
-    if (j0 + 8 <= nb) {
-        *reinterpret_cast<uint32_t *>(qabs + j0) = w[0];
-        *reinterpret_cast<uint32_t *>(qabs + j0 + 4) = w[1];
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (j0 + i < nb) qabs[j0 + i] = (int8_t)((w[i >> 2] >> (8 * (i & 3))) & 0xff);
-    }
-}
-
-// ===========================================================================
-// K3: each warp quantizes one group of 256 constants: d = fp32(a - mu),
-// b = fp32(max|d| / 127), rhat = clamp(rint(fp32(d / b)), -127, 127).  Every
-// CTA first folds the np K2 partials (zero-padded to P = a power of two >= 8)
-// into S and mu = fp32(S / nb) -- the top of the same tree, so mu is
-// bit-exact: warp w folds the aligned slice [w P/8, (w+1) P/8) (lane-local
-// pairs, then a butterfly) and one thread folds the 8 slice sums.  The
-// group's constants are requested before the fold.
-// ===========================================================================
-constexpr int kDqThreads = 256;
-
-__global__ void __launch_bounds__(kDqThreads) dq_quant_kernel(const float *__restrict__ a, int64_t nb,
-                                                              const double *__restrict__ partial, int np,
-                                                              int P, int8_t *__restrict__ qabs,
-                                                              float *__restrict__ scale, float *__restrict__ mu_out,
-                                                              bool e4m3) {
-    __shared__ double slice[kDqThreads / 32];
-    __shared__ float mu_s;
-    pdl_wait();
-    // writes the DQ constants of a weight: no early release (see the quantize kernel)
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int64_t g = (int64_t)blockIdx.x * (kDqThreads / 32) + warp;
-    const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
-    const int64_t j0 = g * kDqGroup + 8 * lane;  // this lane's 8 consecutive constants
     float e[8];
-    load8_const(e, a, g < ng ? j0 : nb, nb);
-
-    {   // the partial sums: L leaves per warp, c per lane (P <= 1024, so c <= 4)
-        const int L = P / 8;
-        const int c = L >= 32 ? L / 32 : 1;
-        const int first = warp * L + lane * c;
-        double s = 0.0;
-        if (lane * c < L) {
-            double t[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) t[i] = (i < c && first + i < np) ? __ldcg(partial + first + i) : 0.0;
-            s = c == 1 ? t[0] : c == 2 ? __dadd_rn(t[0], t[1]) : __dadd_rn(__dadd_rn(t[0], t[1]), __dadd_rn(t[2], t[3]));
+    load8_const(e, a, g < ng ? g * kDqGroup + 8 * lane : nb, nb);
+    const DqScratch sc = dq_scratch(scratch, false);
+    if (warp == 0) {
+        if (scratch) {  // K2 advanced the generation: its bank is the other one
+            const float mu = xsum_mean_warp(sc.bank[(__ldcg(sc.gen) + 1) & 1], (uint32_t)nb);
+            if (lane == 0) {
+                mu_s = mu;
+                if (blockIdx.x == 0) *mu_out = mu;
+            }
+        } else if (lane == 0) {
+            mu_s = __ldcg(mu_in);
         }
-        int levels = 0;
-        for (int span = L / c; span > 1 && levels < 5; span >>= 1) ++levels;
-        s = warp_butterfly_sum(s, levels);
-        if (lane == 0) slice[warp] = s;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const double w01 = __dadd_rn(slice[0], slice[1]), w23 = __dadd_rn(slice[2], slice[3]);
-        const double w45 = __dadd_rn(slice[4], slice[5]), w67 = __dadd_rn(slice[6], slice[7]);
-        const double S = __dadd_rn(__dadd_rn(w01, w23), __dadd_rn(w45, w67));
-        const float mu = __double2float_rn(__ddiv_rn(S, (double)nb));
-        mu_s = mu;
-        if (blockIdx.x == 0) *mu_out = mu;
     }
     __syncthreads();
     const float mu = mu_s;
-    if (g >= ng) return;
-    dq_quantize_group(e, j0, nb, mu, e4m3, lane, g, qabs, scale);
+    for (; g < ng; g += gstep) {
+        float nx[8];
+        load8_const(nx, a, g + gstep < ng ? (g + gstep) * kDqGroup + 8 * lane : nb, nb);
+        dq_quantize_group(e, g * kDqGroup + 8 * lane, nb, mu, e4m3, lane, g, qabs, scale);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) e[u] = nx[u];
+    }
+}
+
+// K3's grid: one group per warp up to the CTAs the device holds at once (a
+// few per SM), then more groups per warp.
+static int64_t dq_quant_grid(int64_t nb, int num_sms) {
+    const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
+    int64_t grid = (ng + kDqGroupsPerCta - 1) / kDqGroupsPerCta;
+    if (grid > 4LL * num_sms) grid = 4LL * num_sms;
+    return grid < 1 ? 1 : grid;
 }
 
 // ===========================================================================
-// Fused double quantization (the workspace entry point): one launch that
-// forms the mean, waits on a grid-wide barrier and quantizes.
-//  1. CTA c owns the 8 * GPW groups [8 GPW c, 8 GPW (c + 1)) -- an aligned
-//     subtree of 2048 GPW block constants.  Each warp keeps its GPW groups'
-//     constants in registers, sums each group as a binary64 perfect tree (8
-//     leaves per lane, then a butterfly), folds its groups and the CTA folds
-//     its 8 warps, both pairwise: the CTA's partial is exactly that subtree of
-//     the whole-tensor tree.  It is published in the workspace.
-//  2. Barrier: the CTA counts itself in (release) and waits, bounded by
-//     kDqfWaitNs, until all G CTAs have (acquire).  G never exceeds the CTAs
-//     the device holds at once, so every CTA is resident.
-//  3. Every CTA folds the G partials (zero-padded to P, the top of the same
-//     tree: mu is bit-exact), then quantizes its groups from registers.
-// The workspace header holds the status word (offset 0), the arrival counter
-// (64) and the departure counter (128); the last CTA to leave puts both
-// counters back to zero, so every call starts from and leaves a zeroed header.
+// Single-launch double quantization (the workspace entry point, when the grid
+// fits on the device): CTA c owns P groups per warp, keeps them in registers,
+// adds them into the call's bank of limbs, and waits on a grid-wide barrier
+// (bounded by kDqfWaitNs) until every CTA has: the last to arrive advances the
+// generation, which the others poll.  Then each CTA reads the limbs, forms mu
+// itself (every CTA gets the same value) and quantizes its groups.  The launch
+// is cooperative, so every CTA is resident whatever else runs on the device.
 // ===========================================================================
-constexpr int kDqfArriveOffset = 64;
-constexpr int kDqfLeaveOffset = 128;
-constexpr uint64_t kDqfWaitNs = 2000000000ull;
-
-__device__ __forceinline__ int dqf_ld_acquire(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ uint64_t dqf_timer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-template <int GPW>
-__global__ void __launch_bounds__(kDqThreads) dq_fused_kernel(const float *__restrict__ a, int64_t nb,
+template <int P>
+__global__ void __launch_bounds__(kDqThreads, P == 1 ? 6 : 4) dq_fused_kernel(const float *__restrict__ a, int64_t nb,
                                                               int8_t *__restrict__ qabs, float *__restrict__ scale,
                                                               float *__restrict__ mu_out, unsigned char *ws, int G,
-                                                              int P, bool e4m3) {
-    __shared__ double wsum[kDqThreads / 32];
+                                                              bool e4m3) {
+    __shared__ unsigned long long slim[kXLimbs];
     __shared__ float mu_s;
     __shared__ int ok_s;
-    int *status = reinterpret_cast<int *>(ws);
-    int *arrive = reinterpret_cast<int *>(ws + kDqfArriveOffset);
-    int *leave = reinterpret_cast<int *>(ws + kDqfLeaveOffset);
-    double *partial = reinterpret_cast<double *>(ws + 256);
+    __shared__ unsigned gen_s;
+    if (threadIdx.x < kXLimbs) slim[threadIdx.x] = 0ull;
+    __syncthreads();
     pdl_wait();  // the constants come from the previous kernel (the quantize)
-    // writes the DQ constants of a weight: no early release (see the quantize kernel)
+    pdl_trigger();
+    const DqScratch sc = dq_scratch(ws, true);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
-    const int64_t g0 = ((int64_t)blockIdx.x * (kDqThreads / 32) + warp) * GPW;
-    if (blockIdx.x == 0 && threadIdx.x == 0) *status = QLN_OK;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *sc.status = QLN_OK;
+    const unsigned g0 = dq_read_gen(sc, &gen_s);
+    unsigned long long *bank = sc.bank[g0 & 1];
 
-    // ---- 1. this CTA's subtree of the mean -----------------------------------
-    float e[GPW][8];
-    double gs[GPW];
+    // groups c*8P + warp + 8p, p < P: all P loads in flight at once
+    float e[P][8];
 #pragma unroll
-    for (int i = 0; i < GPW; ++i) {
-        const int64_t j0 = (g0 + i) * kDqGroup + 8 * lane;
-        load8_const(e[i], a, (g0 + i) < ng ? j0 : nb, nb);
-        gs[i] = warp_butterfly_sum(tree8(e[i]), 5);
+    for (int q = 0; q < P; ++q) {
+        const int64_t g = ((int64_t)blockIdx.x * P + q) * kDqGroupsPerCta + warp;
+        load8_const(e[q], a, g < ng ? g * kDqGroup + 8 * lane : nb, nb);
     }
-#pragma unroll
-    for (int len = GPW; len > 1; len >>= 1)
-#pragma unroll
-        for (int i = 0; i < len / 2; ++i) gs[i] = __dadd_rn(gs[2 * i], gs[2 * i + 1]);
-    if (lane == 0) wsum[warp] = gs[0];
+    dq_add_cta<P>(e, slim, bank);
     __syncthreads();
-    if (threadIdx.x == 0) {
-        const double w01 = __dadd_rn(wsum[0], wsum[1]), w23 = __dadd_rn(wsum[2], wsum[3]);
-        const double w45 = __dadd_rn(wsum[4], wsum[5]), w67 = __dadd_rn(wsum[6], wsum[7]);
-        __stcg(partial + blockIdx.x, __dadd_rn(__dadd_rn(w01, w23), __dadd_rn(w45, w67)));
-        __threadfence();
-        atomicAdd(arrive, 1);
-        // ---- 2. grid barrier, bounded -------------------------------------------
-        bool ok = dqf_ld_acquire(arrive) >= G;
+    if (threadIdx.x == 0) {  // the grid barrier: the generation moves on when the last CTA arrives
+        bool ok = dq_arrive(sc, g0, G) || dqf_ld_acquire_u32(sc.gen) != g0;
         if (!ok) {
             const uint64_t t0 = dqf_timer_ns();
             for (uint32_t it = 0; !ok; ++it) {
-                ok = dqf_ld_acquire(arrive) >= G;
+                ok = dqf_ld_acquire_u32(sc.gen) != g0;
                 if (!ok && (it & 63u) == 63u && dqf_timer_ns() - t0 > kDqfWaitNs) break;
             }
         }
-        if (!ok) atomicExch(status, (int)QLN_ERR_TIMEOUT);
+        if (!ok) atomicExch(sc.status, (int)QLN_ERR_TIMEOUT);
         ok_s = ok;
     }
     __syncthreads();
     const bool ok = ok_s != 0;
-
-    // ---- 3. mu from the G partials, then the groups ----------------------------
-    if (ok) {
-        const int L = P / 8;  // leaves per warp slice; P <= 2048, so c <= 8
-        const int c = L >= 32 ? L / 32 : 1;
-        const int first = warp * L + lane * c;
-        double s = 0.0;
-        if (lane * c < L) {
-            double t[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) t[i] = (i < c && first + i < G) ? __ldcg(partial + first + i) : 0.0;
-#pragma unroll
-            for (int len = 8; len > 1; len >>= 1)
-#pragma unroll
-                for (int i = 0; i < len / 2; ++i) t[i] = __dadd_rn(t[2 * i], t[2 * i + 1]);
-            // leaves past c are zero, so the 8-leaf tree equals the c-leaf one
-            s = t[0];
-        }
-        int levels = 0;
-        for (int span = L / c; span > 1 && levels < 5; span >>= 1) ++levels;
-        s = warp_butterfly_sum(s, levels);
-        __syncthreads();  // wsum is reused
-        if (lane == 0) wsum[warp] = s;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            const double w01 = __dadd_rn(wsum[0], wsum[1]), w23 = __dadd_rn(wsum[2], wsum[3]);
-            const double w45 = __dadd_rn(wsum[4], wsum[5]), w67 = __dadd_rn(wsum[6], wsum[7]);
-            const double S = __dadd_rn(__dadd_rn(w01, w23), __dadd_rn(w45, w67));
-            const float mu = __double2float_rn(__ddiv_rn(S, (double)nb));
+    if (ok && warp == 0) {
+        const float mu = xsum_mean_warp(bank, (uint32_t)nb);
+        if (lane == 0) {
             mu_s = mu;
             if (blockIdx.x == 0) *mu_out = mu;
         }
-        __syncthreads();
-        const float mu = mu_s;
+    }
+    __syncthreads();
+    if (ok) {
 #pragma unroll
-        for (int i = 0; i < GPW; ++i)
-            if (g0 + i < ng) dq_quantize_group(e[i], (g0 + i) * kDqGroup + 8 * lane, nb, mu, e4m3, lane, g0 + i, qabs,
-                                               scale);
+        for (int q = 0; q < P; ++q) {
+            const int64_t g = ((int64_t)blockIdx.x * P + q) * kDqGroupsPerCta + warp;
+            if (g < ng) dq_quantize_group(e[q], g * kDqGroup + 8 * lane, nb, mu_s, e4m3, lane, g, qabs, scale);
+        }
     }
-    // ---- leave: the last CTA out zeroes the counters for the next call --------
-    if (threadIdx.x == 0 && ok && atomicAdd(leave, 1) == G - 1) {
-        *arrive = 0;
-        *leave = 0;
-    }
-}
-
-// Leaves per K2 CTA: 2048 * NG with NG the smallest power of two (<= 16) that
-// keeps the partial count within kMaxPartials.
-static int dq_groups_per_thread(int64_t nb) {
-    int ng = 1;
-    while (ng < 16 && (nb + 2048LL * ng - 1) / (2048LL * ng) > kMaxPartials) ng <<= 1;
-    return ng;
-}
-
-static int64_t dq_partial_count(int64_t nb) {
-    const int64_t C = 2048LL * dq_groups_per_thread(nb);
-    return (nb + C - 1) / C;
 }
 
 size_t dq_workspace_bytes(int64_t nb) {
-    const int64_t fused = ((nb + kDqGroup - 1) / kDqGroup + 7) / 8;  // one partial per CTA of the fused kernel
-    const int64_t np = dq_partial_count(nb) > fused ? dq_partial_count(nb) : fused;
-    return (size_t)(256 + ((np * 8 + 255) / 256) * 256);
+    (void)nb;
+    return kDqScratchBytes;
 }
 
-// CTAs of the fused kernel the device holds at once (cached per variant).
-template <int GPW>
+// CTAs of the fused kernel (P groups per warp) that a cooperative launch can
+// hold; the per-SM figure is cached (one device type per process).
+template <int P>
 static int dq_fused_capacity(int num_sms) {
     static std::atomic<int> cached{0};
     int per_sm = cached.load(std::memory_order_relaxed);
     if (per_sm == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dq_fused_kernel<GPW>, kDqThreads, 0) !=
-            cudaSuccess) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dq_fused_kernel<P>, kDqThreads, 0) != cudaSuccess) {
             cudaGetLastError();
             return 0;
         }
@@ -739,104 +877,161 @@ static int dq_fused_capacity(int num_sms) {
     return per_sm * num_sms;
 }
 
-// The fused kernel when its grid fits on the device at once; false when it
-// does not (then the two-kernel path runs).
-template <int GPW>
+template <int P>
+static cudaError_t launch_dq_fused(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu, void *ws,
+                                   bool e4m3, cudaStream_t st, int G) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)G);
+    cfg.blockDim = dim3(kDqThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    // A driver that refuses a cooperative launch with programmatic serialization
+    // gets a plain cooperative launch (remembered per process).
+    static std::atomic<int> pdl_refused{0};
+    cfg.numAttrs = pdl_refused.load(std::memory_order_relaxed) ? 1 : 2;
+    note_launch();
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, dq_fused_kernel<P>, absmax, nb, qabs, scale, mu, w, G, e4m3);
+    if (err != cudaSuccess && cfg.numAttrs == 2) {
+        cudaGetLastError();
+        pdl_refused.store(1, std::memory_order_relaxed);
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelEx(&cfg, dq_fused_kernel<P>, absmax, nb, qabs, scale, mu, w, G, e4m3);
+    }
+    return err;
+}
+
+// The fused kernel, launched cooperatively (every CTA resident) and as a
+// programmatic dependent, with the fewest groups per warp (1, 2 or 4) whose
+// grid fits on the device; false when even 4 do not fit.
 static bool try_dq_fused(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu, void *ws, bool e4m3,
                          cudaStream_t st, int num_sms, cudaError_t *err) {
     const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
-    const int64_t G = (ng + 8 * GPW - 1) / (8 * GPW);
-    if (G > dq_fused_capacity<GPW>(num_sms)) return false;
-    int P = 8;
-    while (P < G) P <<= 1;
-    if (P > 2048) return false;
-    *err = launch_pdl(dq_fused_kernel<GPW>, dim3((unsigned)G), dim3(kDqThreads), 0, st, absmax, nb, qabs, scale, mu,
-                      static_cast<unsigned char *>(ws), (int)G, P, e4m3);
+    auto grid = [&](int P) { return (ng + (int64_t)P * kDqGroupsPerCta - 1) / ((int64_t)P * kDqGroupsPerCta); };
+    if (grid(1) <= dq_fused_capacity<1>(num_sms)) {
+        *err = launch_dq_fused<1>(absmax, nb, qabs, scale, mu, ws, e4m3, st, (int)grid(1));
+    } else if (grid(2) <= dq_fused_capacity<2>(num_sms)) {
+        *err = launch_dq_fused<2>(absmax, nb, qabs, scale, mu, ws, e4m3, st, (int)grid(2));
+    } else if (grid(4) <= dq_fused_capacity<4>(num_sms)) {
+        *err = launch_dq_fused<4>(absmax, nb, qabs, scale, mu, ws, e4m3, st, (int)grid(4));
+    } else {
+        return false;
+    }
     return true;
 }
 
 int64_t dq_max_blocks() { return kMeanMaxBlocks; }
 
-// K2 then K3, each launched as a programmatic dependent of the kernel before it.
-static cudaError_t launch_dq_pair(const float *absmax, int64_t nb, double *partial, int8_t *qabs, float *scale,
-                                  float *mu, bool e4m3, cudaStream_t st) {
-    const int NG = dq_groups_per_thread(nb);
-    const int np = (int)dq_partial_count(nb);
-    int P = 8;
-    while (P < np) P <<= 1;
-    cudaError_t e;
-    const dim3 g2((unsigned)np), b2(kMeanThreads);
-    switch (NG) {
-        case 1: e = launch_pdl(dq_partial_kernel<1>, g2, b2, 0, st, absmax, nb, partial); break;
-        case 2: e = launch_pdl(dq_partial_kernel<2>, g2, b2, 0, st, absmax, nb, partial); break;
-        case 4: e = launch_pdl(dq_partial_kernel<4>, g2, b2, 0, st, absmax, nb, partial); break;
-        case 8: e = launch_pdl(dq_partial_kernel<8>, g2, b2, 0, st, absmax, nb, partial); break;
-        default: e = launch_pdl(dq_partial_kernel<16>, g2, b2, 0, st, absmax, nb, partial); break;
-    }
-    if (e != cudaSuccess) return e;
+// K2 then K3 (mu from the limbs), each launched as a programmatic dependent of
+// the kernel before it.
+static cudaError_t launch_dq_pair(const float *absmax, int64_t nb, unsigned char *scratch, bool with_status,
+                                  int8_t *qabs, float *scale, float *mu, bool e4m3, cudaStream_t st, int num_sms) {
     const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
-    const int64_t grid = (ng + (kDqThreads / 32) - 1) / (kDqThreads / 32);
-    return launch_pdl(dq_quant_kernel, dim3((unsigned)grid), dim3(kDqThreads), 0, st, absmax, nb,
-                      (const double *)partial, np, P, qabs, scale, mu, e4m3);
+    int64_t g2 = (ng + kDqGroupsPerCta - 1) / kDqGroupsPerCta;
+    if (g2 > 4LL * num_sms) g2 = 4LL * num_sms;  // a few passes per CTA for very large weights
+    cudaError_t e = launch_pdl(dq_sum_kernel, dim3((unsigned)g2), dim3(kDqThreads), 0, st, absmax, nb, scratch,
+                               with_status);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(dq_quant_kernel, dim3((unsigned)dq_quant_grid(nb, num_sms)), dim3(kDqThreads), 0, st, absmax,
+                      nb, qabs, scale, (const float *)nullptr, mu, scratch, e4m3);
 }
 
 cudaError_t launch_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,
                                     void *ws, bool e4m3, cudaStream_t st, int num_sms) {
     cudaError_t e = cudaSuccess;
-    // Measured on B200 (CUDA graphs, after the quantize): the single launch with
-    // one group per warp saves ~1.7 us on an 11008 x 4096 weight and is within
-    // 0.2 us of the two kernels on 4096 x 4096; more groups per warp serialise
-    // each warp's work (8 per warp: 12.9 us against 4.9 us), so weights too
-    // large for one group per warp take the two kernels.
-    if (try_dq_fused<1>(absmax, nb, qabs, scale, mu, ws, e4m3, st, num_sms, &e)) return e;
-    double *partial = reinterpret_cast<double *>(reinterpret_cast<char *>(ws) + 256);
-    return launch_dq_pair(absmax, nb, partial, qabs, scale, mu, e4m3, st);
+    if (try_dq_fused(absmax, nb, qabs, scale, mu, ws, e4m3, st, num_sms, &e)) return e;
+    return launch_dq_pair(absmax, nb, static_cast<unsigned char *>(ws), true, qabs, scale, mu, e4m3, st, num_sms);
+}
+
+// The quantize, then the double quantization of its block constants (the
+// single cooperative launch where it fits), each a programmatic dependent of
+// the kernel before it: the combined entry point computes exactly what the two
+// entry points compute.
+cudaError_t launch_nf4_quantize_dq(const void *W, int dtype, int64_t numel, uint8_t *codes, float *absmax,
+                                   int8_t *qabs, float *scale, float *mu, void *ws, bool e4m3, cudaStream_t st,
+                                   int num_sms) {
+    cudaError_t e = launch_nf4_quantize(W, dtype, numel, codes, absmax, st, num_sms);
+    if (e != cudaSuccess) return e;
+    return launch_nf4_double_quant(absmax, (numel + 63) / 64, qabs, scale, mu, ws, e4m3, st, num_sms);
 }
 
 // ===========================================================================
-// Allocation-free double quantization.  The only scratch K2/K3 need is the
-// binary64 partial sums of mu (at most kMaxPartials of them).  This variant
-// keeps them in a fixed, file-scope device array instead of a caller
-// workspace, so a caller that cannot allocate device memory can still run the
-// path.  The array is 8 KB; the entry point accepts nb up to 1024 * 8192 =
-// 8,388,608 blocks (536,870,912 weights); every GPU that loads the library
-// holds it until the process exits.  Each call overwrites every partial it
-// reads before reading it, so nothing has to be cleared between calls; two
+// Allocation-free double quantization.  The only scratch the two-kernel path
+// needs is the generation word, the arrival counter and the banks of limbs;
+// this variant keeps them in a fixed, file-scope device array instead of a
+// caller workspace, so a caller that cannot allocate device memory can still
+// run the path.  The array is kDqScratchBytes (256 bytes); every GPU that loads
+// the library holds it until the process exits.  Each call leaves the bank the
+// next call sums into zeroed, so nothing has to be cleared between calls; two
 // calls that overlap on the GPU (different streams, no ordering) share the
-// array and race.
+// array and race.  There is no status word (no workspace to hold it).
 // ===========================================================================
-constexpr int kStaticPartials = kMaxPartials;
-static __device__ __align__(256) double g_dq_static_partials[kStaticPartials];
-static std::atomic<double *> g_dq_static_ptr[64];
+static __device__ __align__(256) unsigned char g_dq_static_scratch[kDqScratchBytes];
 
-int64_t dq_static_max_blocks() { return (int64_t)1024 * 8192; }
+int64_t dq_static_max_blocks() { return kMeanMaxBlocks; }
 
-// Device address of the array on the current device.  In host code the
-// symbol names a host-side stand-in, so the address is looked up once per
-// device (with that device current) and cached.
-static cudaError_t dq_static_partials(double **out) {
+// Device address of the array for the current device and context.  In host
+// code the symbol names a host-side stand-in, so the address is looked up
+// (with the device current) and cached per device together with the context
+// it was looked up in: a context torn down and made again may load the module
+// elsewhere, so a new context means a new lookup.
+struct DqStaticSlot {
+    std::mutex mu;
+    void *ctx = nullptr;
+    unsigned char *ptr = nullptr;
+};
+static DqStaticSlot g_dq_static_slot[64];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+static CtxGetCurrentFn ctx_get_current_fn() {
+    static std::atomic<CtxGetCurrentFn> fn{nullptr};
+    CtxGetCurrentFn f = fn.load(std::memory_order_acquire);
+    if (!f) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) {
+            f = reinterpret_cast<CtxGetCurrentFn>(p);
+            fn.store(f, std::memory_order_release);
+        }
+    }
+    return f;
+}
+
+static cudaError_t dq_static_scratch(unsigned char **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    double *p = g_dq_static_ptr[dev].load(std::memory_order_acquire);
-    if (!p) {
+    CtxGetCurrentFn getctx = ctx_get_current_fn();
+    if (!getctx) return cudaErrorDeviceUninitialized;
+    CUcontext ctx = nullptr;
+    if (getctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+    DqStaticSlot &slot = g_dq_static_slot[dev];
+    std::lock_guard<std::mutex> lock(slot.mu);
+    if (slot.ptr == nullptr || ctx == nullptr || slot.ctx != (void *)ctx) {
         void *addr = nullptr;
-        e = cudaGetSymbolAddress(&addr, g_dq_static_partials);
+        e = cudaGetSymbolAddress(&addr, g_dq_static_scratch);  // makes the device's context current if needed
         if (e != cudaSuccess) return e;
-        p = static_cast<double *>(addr);
-        g_dq_static_ptr[dev].store(p, std::memory_order_release);
+        if (getctx(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+        slot.ptr = static_cast<unsigned char *>(addr);
+        slot.ctx = (void *)ctx;
     }
-    *out = p;
+    *out = slot.ptr;
     return cudaSuccess;
 }
 
 cudaError_t launch_nf4_double_quant_static(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,
-                                           cudaStream_t st) {
-    double *partial = nullptr;
-    cudaError_t e = dq_static_partials(&partial);
+                                           cudaStream_t st, int num_sms) {
+    unsigned char *scratch = nullptr;
+    cudaError_t e = dq_static_scratch(&scratch);
     if (e != cudaSuccess) return e;
-    return launch_dq_pair(absmax, nb, partial, qabs, scale, mu, false, st);
+    return launch_dq_pair(absmax, nb, scratch, false, qabs, scale, mu, false, st, num_sms);
 }
 
 // ===========================================================================

@@ -148,17 +148,9 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
     const uint32_t slots_s = smem_u32(dsm + p.off_slots), uslots_s = smem_u32(dsm + p.off_uslots);
     const int ahs = nkbx + 1;
 
-    // Before the dependency wait the kernel touches shared memory, the
-    // launch's parameters and the weight (codes and block constants), never X,
-    // A, B, Y or U.  Reading the weight early is safe because the kernel ahead
-    // of this one on the stream has released it only after its own dependency
-    // wait (every kernel of this library does), so every kernel before that
-    // one has completed; and the kernels of this library that write a weight
-    // (quantize, double quantization) never release their dependents early, so
-    // if the kernel ahead wrote this weight, this one starts after it has
-    // completed.  A caller's own kernel that writes the weight must not release
-    // its dependents early either (it does not unless it executes
-    // griddepcontrol.launch_dependents).
+    // Before the dependency wait only shared memory and the launch's own
+    // parameters are touched, nothing an earlier kernel on the stream can
+    // change: barriers and the decode table are ready while that kernel ends.
     cl_arrive_relaxed();  // this CTA runs: peers may store into it once they have waited
     if (lane == 0) {
         for (int s = 0; s < RS; ++s) tc::mbar_init(bar_w + 8u * s, 1);
@@ -238,14 +230,14 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
         }
     };
 
-    // ---- 1. requests: the weight (code boxes, block constants) before the
-    //         dependency wait, then X and the B rows ---------------------------------------
+    // ---- 1. requests: the code boxes first (the longest latency), then the block
+    //         constants, X and the B rows --------------------------------------------------
+    pdl_wait();  // the weight, X, A, B and the workspace may be written by the previous kernel
+    pdl_trigger();
+    if (blockIdx.x == 0 && tid == 0) *p.status = QLN_OK;
 #pragma unroll 1
     for (int k = 0; k < RS; ++k) issue_next();
     stage_ah(0);
-    pdl_wait();  // X, A, B and the workspace may be written by the previous kernel on the stream
-    pdl_trigger();
-    if (blockIdx.x == 0 && tid == 0) *p.status = QLN_OK;
     // X chunk: line (token t, block bl) at row t * nkbx + bl, second half; 16-B chunks swizzled by t & 1
 #pragma unroll 1
     for (int t = warp; t < 8 * NT; t += kDfWarps)

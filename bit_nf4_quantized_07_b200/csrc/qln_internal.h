@@ -40,6 +40,9 @@ cudaError_t launch_nf4_quantize(const void *W, int dtype, int64_t numel, uint8_t
                                 cudaStream_t st, int num_sms);
 cudaError_t launch_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,
                                     void *ws, bool e4m3, cudaStream_t st, int num_sms);
+cudaError_t launch_nf4_quantize_dq(const void *W, int dtype, int64_t numel, uint8_t *codes, float *absmax,
+                                   int8_t *qabs, float *scale, float *mu, void *ws, bool e4m3, cudaStream_t st,
+                                   int num_sms);
 cudaError_t launch_nf4_dequant(const qln_nf4_weight *w, uint16_t *out, cudaStream_t st, int num_sms);
 cudaError_t launch_adamw(float *p, const float *g, float *m, float *v, uint16_t *p_bf16, int64_t n, float lr,
                          float b1, float b2, float eps, float wd, const int64_t *step, int flags, cudaStream_t st,
@@ -49,7 +52,7 @@ cudaError_t launch_nf4_dequant_flat(const qln_nf4_weight *w, int64_t numel, uint
 size_t dq_workspace_bytes(int64_t nb);
 // allocation-free variant: scratch in a file-scope device array (codec.cu)
 cudaError_t launch_nf4_double_quant_static(const float *absmax, int64_t nb, int8_t *qabs, float *scale, float *mu,
-                                           cudaStream_t st);
+                                           cudaStream_t st, int num_sms);
 int64_t dq_static_max_blocks();
 int64_t dq_max_blocks();
 

@@ -41,15 +41,22 @@
  *   NULL pointers (QLN_ERR_NULL), bad sizes (QLN_ERR_SHAPE), pointers not
  *   16-byte aligned (QLN_ERR_ALIGN), workspace too small (QLN_ERR_WORKSPACE),
  *   current device not sm_100 (QLN_ERR_ARCH).  A failed launch returns
- *   QLN_ERR_CUDA (cudaGetLastError).  Kernels that wait on on-chip barriers
- *   give up after a bounded number of polls and write QLN_ERR_TIMEOUT into the
- *   int32 status word at byte offset 0 of the workspace; read it after the
- *   stream has synchronised (0 = QLN_OK).  Each workspace call clears it.
- * - Bytes 4..255 of a workspace hold counters (the decode-sized forward,
- *   n <= 32; the single-launch double quantization's grid barrier).
- *   Zero-fill a workspace once before its first use; every call
- *   leaves the counters at zero again (also across CUDA graph replays).  After
- *   a call that reported QLN_ERR_TIMEOUT, zero the first 256 bytes again.
+ *   QLN_ERR_CUDA (cudaGetLastError).  Kernels that wait (on TMA barriers, on
+ *   a thread-block cluster, on the grid-wide barrier of the single-launch
+ *   double quantization) give up after a bounded time and write
+ *   QLN_ERR_TIMEOUT into the int32 status word at byte offset 0 of the
+ *   workspace; read it after the stream has synchronised (0 = QLN_OK).  Each
+ *   workspace call clears it.
+ * - Bytes 4..255 of a double-quantization workspace hold a generation word,
+ *   a counter and two banks for the exact sum of mu.  Zero-fill a workspace
+ *   once before its first use and leave it to the library afterwards: each
+ *   call sums into the bank the generation selects, zeroes the other one and
+ *   advances the generation, so every call finds what it needs zeroed (also
+ *   across CUDA graph replays).  After a call that reported QLN_ERR_TIMEOUT,
+ *   zero the first 256 bytes again.  The linear forward and backward keep no state in the
+ *   workspace between calls.
+ * - No entry point creates streams or events or synchronises the host: each
+ *   enqueues its kernels on the caller's stream, in order, and returns.
  */
 #ifndef QLORA_NF4_H
 #define QLORA_NF4_H
@@ -151,23 +158,24 @@ QLN_API qln_status nf4_quantize_ex(const void *W, int32_t dtype, int64_t numel, 
  * jjjymmm.cn "Double Quantization" (blocks of 256 constants).
  *   absmax   [nb] fp32 in;  qabs [nb] int8 out;  dq_scale [ceil(nb/256)] fp32
  *   out;  dq_mean [1] fp32 out.
- * mu = fp32(S / nb), S the binary64 sum of all a_j over a fixed perfect binary
- * tree (leaves zero-padded to a power of two), so mu is reproducible bit for
- * bit.  Per group g: d_j = fp32(a_j - mu), b_g = fp32(max|d_j| / 127),
+ * mu = the binary32 value nearest to the exact mean (1/nb) sum_j a_j, ties
+ * to even: the sum is formed exactly in integer arithmetic, so mu does not
+ * depend on the order of summation, the grid or the device.  Per group g:
+ * d_j = fp32(a_j - mu), b_g = fp32(max|d_j| / 127),
  * rhat_j = clamp(rint(fp32(d_j / b_g)), -127, 127) (ties to even), 0 when
  * b_g == 0.  The last group may be partial.
  *   ws / ws_bytes: device scratch of at least
- *   qln_workspace_bytes(QLN_OP_DOUBLE_QUANT, nb, 0, 0, 0) bytes, 256-byte
- *   aligned.  Its first 256 bytes are a header: a status word at offset 0
- *   (QLN_OK, or QLN_ERR_TIMEOUT when a bounded device wait gave up) and
- *   counters of the single-launch path's grid barrier.  Zero the header once
- *   before the first call; every call leaves it zeroed again (zero it anew
- *   after a QLN_ERR_TIMEOUT).  The rest is scratch.
- * Weights of up to about 116 M parameters take a single launch whose CTAs
- * meet at a grid-wide barrier; its grid is sized so that the whole device
- * holds it at once.  A kernel on another stream that keeps SMs busy only
- * delays it, and a wait longer than 2 s ends with QLN_ERR_TIMEOUT in the
- * status word instead of a hang.
+ *   qln_workspace_bytes(QLN_OP_DOUBLE_QUANT, nb, 0, 0, 0) (= 256) bytes,
+ *   256-byte aligned: a status word at offset 0 (QLN_OK, or QLN_ERR_TIMEOUT
+ *   when a bounded device wait gave up), the counters of the single-launch
+ *   path's grid barrier and the exact sum.  Zero it once before the first
+ *   call and then leave it to the library (zero it anew after a
+ *   QLN_ERR_TIMEOUT).
+ * Weights of up to about 310 M parameters take a single cooperative launch
+ * whose CTAs meet at a grid-wide barrier: every CTA is resident at once, so a
+ * kernel on another stream can only delay it, and a wait longer than 2 s
+ * ends with QLN_ERR_TIMEOUT in the status word instead of a hang.  Larger
+ * weights take two launches that do not wait on one another.
  * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE if nb <= 0 or nb > 2^25 (numel above
  * 2^31); QLN_ERR_WORKSPACE; QLN_ERR_ALIGN if absmax is not 16-byte aligned or
  * ws is not 256-byte aligned.
@@ -192,25 +200,51 @@ QLN_API qln_status nf4_double_quant_ex(const float *absmax, int64_t nb, int32_t 
                                        float *dq_scale, float *dq_mean, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * nf4_quantize_dq -- nf4_quantize_ex followed by nf4_double_quant_ex, as one
+ * call with the same bits.  Defined by the two passages those entry points
+ * cite: "LoRA 与 QLoRA" section QLoRA (blockwise NF4 with absmax, then the
+ * double quantization of the block constants).
+ *   W [numel] of dtype in; codes [ceil(numel/2)], absmax [nb], qabs [nb],
+ *   dq_scale [ceil(nb/256)], dq_mean [1] out, nb = ceil(numel/64); dq_format
+ *   QLN_DQ_INT8 or QLN_DQ_E4M3 (as nf4_double_quant_ex).
+ * The two steps are enqueued back to back, the second as a programmatic
+ * dependent of the first, with the double quantization's launch shapes (its
+ * single cooperative launch where that fits).  W must be finite (mu of
+ * non-finite constants is not defined).
+ *   ws / ws_bytes: a double-quantization workspace (qln_workspace_bytes
+ *   QLN_OP_DOUBLE_QUANT, 256 bytes), zeroed once before the first call and
+ *   then left to the library; byte 0 is the status word.
+ * Errors: QLN_ERR_NULL; QLN_ERR_SHAPE (numel <= 0 or above 2^31, unknown
+ * dtype or format); QLN_ERR_ALIGN (W, codes, absmax 16-byte; ws 256-byte);
+ * QLN_ERR_WORKSPACE; QLN_ERR_ARCH.
+ */
+QLN_API qln_status nf4_quantize_dq(const void *W, int32_t dtype, int64_t numel, int32_t dq_format, uint8_t *codes,
+                                   float *absmax, void *qabs, float *dq_scale, float *dq_mean, void *ws,
+                                   size_t ws_bytes, void *stream);
+
+/*
  * nf4_double_quant_noalloc -- nf4_double_quant without a caller workspace.
  * The pages describe nothing like it: it exists for callers that cannot
  * allocate device memory at the point where they quantize -- for example a
  * runtime that reserves all device memory up front in its own pool and
  * forbids further cudaMalloc, or a plugin that only receives tensors from a
  * host framework and has no allocator of its own.  It computes exactly what
- * nf4_double_quant computes (same kernels, same bits) and allocates nothing:
+ * nf4_double_quant computes (the same bits) and allocates nothing:
  * it calls no cudaMalloc, cudaFree or other allocating routine.
- *   Scratch: an 8 KB array of binary64 partial sums at file scope in the
- *   library, present on every GPU that loads it until the process exits.
- *   Limit: nb <= 8,388,608 block constants (weights <= 536,870,912); larger
- *   nb returns QLN_ERR_SHAPE before anything is launched.
- *   Set-up: the first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture on that device.
- *   Sharing: every call uses the same array.  Each call rewrites all of it
- *   that it reads, so nothing carries over, but calls that overlap on the GPU
- *   (e.g. on two unordered streams) race on it and must be serialised by the
- *   caller.
+ *   Scratch: a 256-byte array at file scope in the library (a generation
+ *   word, a counter and the exact sum of mu), present on every GPU that loads it
+ *   until the process exits.  It always takes the two-launch path, whose
+ *   kernels never wait on one another.
+ *   Limit: nb <= 2^25 block constants, as nf4_double_quant; larger nb returns
+ *   QLN_ERR_SHAPE before anything is launched.
+ *   Set-up: the first call in a CUDA context looks up the array's device
+ *   address (cudaGetSymbolAddress, with that device current) and caches it
+ *   with the context; make that first call before any stream capture in that
+ *   context.
+ *   Sharing: every call uses the same array; each leaves the part the next
+ *   call sums into zeroed, so nothing carries over from call to call.  Calls
+ *   that overlap on the GPU (e.g. on two unordered streams) race on it and
+ *   must be serialised by the caller.
  * Arguments and outputs as nf4_double_quant.  Errors: QLN_ERR_NULL,
  * QLN_ERR_SHAPE, QLN_ERR_ALIGN, QLN_ERR_ARCH, QLN_ERR_CUDA.
  */

@@ -58,8 +58,11 @@ def test_version_and_status_strings(L):
 
 
 def test_workspace_sizes(L):
-    assert api.workspace_bytes(api.OP_DOUBLE_QUANT, 4096) >= 256 + 8
-    assert api.workspace_bytes(api.OP_DOUBLE_QUANT, 3670016) >= 256 + 8 * (3670016 // 8192)
+    # double quantization: a 256-byte header (status, barrier counters, the
+    # exact sum of mu) whatever nb is
+    assert api.workspace_bytes(api.OP_DOUBLE_QUANT, 4096) == 256
+    assert api.workspace_bytes(api.OP_DOUBLE_QUANT, 1 << 25) == 256
+    assert api.workspace_bytes(api.OP_DOUBLE_QUANT, 0) == 0
     f = api.workspace_bytes(api.OP_LINEAR_FWD, 11008, 4096, 2048, 16)
     assert f >= 256 + 2 * 2048 * 16 * 2
     b = api.workspace_bytes(api.OP_LINEAR_BWD, 11008, 4096, 2048, 16)
@@ -98,6 +101,23 @@ def test_double_quant_argument_errors(L):
     assert L.nf4_double_quant(A16, (1 << 25) + 1, A16, A16, A16, ws, 1 << 40, None) == 2
     assert L.nf4_double_quant(A16, 100, A16, A16, A16, P(0x20010), need, None) == 3
     assert L.nf4_double_quant(A16, 100, A16, A16, A16, ws, need - 1, None) == 4
+
+
+def test_quantize_dq_argument_errors(L):
+    ws = P(0x20000)
+    q = lambda **k: L.nf4_quantize_dq(k.get("W", A16), k.get("dtype", 0), k.get("numel", 4096), k.get("fmt", 0),
+                                      A16, k.get("absmax", A16), A16, A16, A16, k.get("ws", ws),
+                                      k.get("wsb", 256), None)
+    assert q(W=None) == 1
+    assert q(ws=None) == 1
+    assert q(numel=0) == 2
+    assert q(numel=(1 << 31) + 1) == 2
+    assert q(dtype=7) == 2
+    assert q(fmt=2) == 2
+    assert q(W=A4) == 3
+    assert q(absmax=A4) == 3            # 16-byte: the group pass reads 8 constants at a time
+    assert q(ws=P(0x20010)) == 3
+    assert q(wsb=255) == 4
 
 
 def test_dequant_argument_errors(L):

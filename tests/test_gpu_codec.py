@@ -25,6 +25,15 @@ def _gpu_codec(w: np.ndarray):
             mu.cpu().numpy()[0], dev_bf16_bits(deq).reshape(-1), dev_bf16_bits(deq_plain).reshape(-1))
 
 
+def _scratch_at_rest(ws):
+    """The DQ scratch between calls: status 0, arrival counter 0 and the bank of
+    limbs the next call sums into (bank gen % 2) all zero."""
+    w = ws[:256].view(torch.int32).cpu().numpy()
+    gen = int(w[4])                                   # generation word at byte 16
+    bank = w[16:36] if gen % 2 == 0 else w[40:60]     # banks at bytes 64 and 160, 80 bytes each
+    return w[0] == 0 and w[8] == 0 and not bank.any()
+
+
 def _check_all(w):
     n = w.size
     g = _gpu_codec(w)
@@ -228,9 +237,10 @@ def test_e4m3_double_quant_and_dequant_bit_exact(shape, seed):
 
 @pytest.mark.parametrize("fmt", ["int8", "e4m3"])
 def test_single_launch_dq_repeats_replays_and_leaves_header_zeroed(fmt):
-    """The single-launch double quantization (grid barrier on counters in the
-    workspace header): back-to-back calls and CUDA graph replays on one
-    workspace give the oracle's bits, and every call leaves the header at zero."""
+    """The single-launch double quantization (grid barrier on counters and the
+    exact sum in the workspace header): back-to-back calls, a call on another
+    stream and CUDA graph replays on one workspace give the oracle's bits, and
+    every call leaves the scratch ready for the next one."""
     w = synthetic.normal_f32((11008 // 4, 4096), 0.02, 61)
     codes, absmax = api.nf4_quantize(torch.from_numpy(w).cuda())
     nb = absmax.numel()
@@ -245,7 +255,7 @@ def test_single_launch_dq_repeats_replays_and_leaves_header_zeroed(fmt):
     assert np.array_equal(q.cpu().numpy().view(np.uint8), q_ref.view(np.uint8))
     assert np.array_equal(b.cpu().numpy().view(np.uint32), b_ref.view(np.uint32))
     assert np.float32(mu.item()).view(np.uint32) == np.float32(mu_ref).view(np.uint32)
-    assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0
+    assert _scratch_at_rest(ws)
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
@@ -261,20 +271,21 @@ def test_single_launch_dq_repeats_replays_and_leaves_header_zeroed(fmt):
         graph.replay()
     torch.cuda.synchronize()
     assert np.array_equal(q.cpu().numpy().view(np.uint8), q_ref.view(np.uint8))
-    assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0
+    assert _scratch_at_rest(ws)
 
 
 def test_single_launch_dq_barrier_runs_out_and_reports_timeout():
     """Failure detection without a GPU fault: an arrival counter that can
-    never reach the grid size makes every CTA's bounded barrier wait (2 s) run
-    out; the kernel records QLN_ERR_TIMEOUT and finishes.  With the header
-    zeroed again the next call is exact."""
+    never count the last CTA in leaves the generation where it is, so every
+    CTA's bounded barrier wait (2 s) runs out; the kernel records
+    QLN_ERR_TIMEOUT and finishes.  With the header zeroed again the next call
+    is exact."""
     import time
     w = synthetic.normal_f32((1024, 4096), 0.02, 62)
     codes, absmax = api.nf4_quantize(torch.from_numpy(w).cuda())
     nb = absmax.numel()
     ws = api.alloc_workspace(api.workspace_bytes(api.OP_DOUBLE_QUANT, nb))
-    ws[64:68].view(torch.int32).fill_(-(1 << 30))  # the barrier's arrival counter
+    ws[32:36].view(torch.int32).fill_(-(1 << 30))  # the barrier's arrival counter: no CTA is ever last
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     api.nf4_double_quant(absmax, ws=ws)
@@ -287,3 +298,152 @@ def test_single_launch_dq_barrier_runs_out_and_reports_timeout():
     assert api.device_status(ws) == 0
     q_ref, b_ref, mu_ref = codec.double_quant(codec.quantize(w)[1])
     assert np.array_equal(q.cpu().numpy(), q_ref) and np.float32(mu.item()) == np.float32(mu_ref)
+
+
+def _spread_constants(nb, seed):
+    """Block constants spanning subnormals to 1e30 (and some negative ones,
+    which the entry point accepts): the exact sum's runs fall on different
+    limbs inside one warp and the sum changes sign along the way."""
+    rng = np.random.default_rng(seed)
+    a = (rng.random(nb) * 10.0 ** rng.integers(-44, 31, nb)).astype(np.float32)
+    a[rng.integers(0, nb, max(1, nb // 50))] *= -1
+    a[rng.integers(0, nb, 8)] = np.float32(1.4e-45)
+    return a
+
+
+@pytest.mark.parametrize("nb", [1, 255, 257, 70001, 2000003, 3670016, 6000001])
+@pytest.mark.parametrize("kind", ["normal", "spread"])
+def test_double_quant_every_launch_shape_matches_oracle(nb, kind):
+    """Direct double quantization of block constants against the oracle, at
+    sizes that take each launch shape on a 148-SM B200: one group per warp
+    (nb <= 1.8 M), two (<= 2.4 M), four (<= 4.8 M) in the single cooperative
+    launch, and the two-launch path beyond.  mu must be the oracle's bits."""
+    a = (np.abs(synthetic.normal_f32(nb, 0.02, 70 + nb % 97)) if kind == "normal"
+         else _spread_constants(nb, 71 + nb % 89))
+    q, b, mu = api.nf4_double_quant(torch.from_numpy(a).cuda())
+    torch.cuda.synchronize()
+    q_ref, b_ref, mu_ref = codec.double_quant(a)
+    assert np.float32(mu.item()).view(np.uint32) == np.float32(mu_ref).view(np.uint32), (mu.item(), mu_ref)
+    assert np.array_equal(b.cpu().numpy().view(np.uint32), b_ref.view(np.uint32)), "dq scale"
+    assert np.array_equal(q.cpu().numpy(), q_ref), f"{np.sum(q.cpu().numpy() != q_ref)} dq codes differ"
+
+
+@pytest.mark.parametrize("numel,dtype,fmt,seed", [
+    (64, torch.float32, "int8", 80), (4096 * 4096, torch.float32, "int8", 81), (1000 * 192 + 37, torch.float32, "int8", 82),
+    (11008 * 512, torch.bfloat16, "int8", 83), (333333, torch.float16, "e4m3", 84), (5 * 16384 + 1, torch.bfloat16, "e4m3", 85)])
+def test_quantize_dq_one_call_matches_oracle(numel, dtype, fmt, seed):
+    """nf4_quantize_dq (quantize with the exact sum formed on the way, then the
+    group quantization) against the oracle's quantize + double_quant of the
+    same weights, ragged tails and every input dtype included; repeated calls
+    on one workspace give the same bits and leave its scratch ready for the
+    next call."""
+    w = synthetic.normal_f32(numel, 0.02, seed)
+    Wc = torch.from_numpy(w).to(dtype)          # rounded to the input dtype on the host
+    w_exact = Wc.float().numpy()                # the values the kernel sees (widening is exact)
+    Wd = Wc.cuda()
+    ws = api.alloc_workspace(api.workspace_bytes(api.OP_DOUBLE_QUANT, (numel + 63) // 64))
+    out = api.nf4_quantize_dq(Wd, ws=ws, fmt=fmt)
+    again = api.nf4_quantize_dq(Wd, ws=ws, fmt=fmt)
+    torch.cuda.synchronize()
+    codes, absmax, q, b, mu = [t.cpu().numpy() for t in out]
+    c_ref, a_ref = codec.quantize(w_exact)
+    q_ref, b_ref, mu_ref = codec.double_quant(a_ref, fmt=fmt)
+    assert np.array_equal(codes, c_ref), f"{np.sum(codes != c_ref)} code bytes differ"
+    assert np.array_equal(absmax.view(np.uint32), a_ref.view(np.uint32))
+    assert np.float32(mu[0]).view(np.uint32) == np.float32(mu_ref).view(np.uint32), (mu[0], mu_ref)
+    assert np.array_equal(b.view(np.uint32), b_ref.view(np.uint32)), "dq scale"
+    assert np.array_equal(q.view(np.uint8), q_ref.view(np.uint8)), "dq codes"
+    for x, y in zip(out, again):
+        assert torch.equal(x, y)
+    assert api.device_status(ws) == 0
+    assert _scratch_at_rest(ws)
+
+
+def test_single_launch_dqs_near_the_size_limit_on_two_unordered_streams():
+    """Two single-launch double quantizations, each with a grid of about 3/4 of
+    what the device holds at once (four groups per warp, 4.5 M constants), on
+    two streams with no order between them.  The cooperative launch keeps each
+    grid's CTAs resident together, so both grid barriers complete: status
+    QLN_OK and the oracle's bits for both."""
+    nb = 4_500_000
+    a_np = [np.abs(synthetic.normal_f32(nb, 0.02, 90 + k)) for k in range(2)]
+    a = [torch.from_numpy(x).cuda() for x in a_np]
+    ws = [api.alloc_workspace(api.workspace_bytes(api.OP_DOUBLE_QUANT, nb)) for _ in range(2)]
+    outs = [(torch.empty(nb, dtype=torch.int8, device="cuda"), torch.empty((nb + 255) // 256, device="cuda"),
+             torch.empty(1, device="cuda")) for _ in range(2)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for k in range(2):
+            with torch.cuda.stream(streams[k]):
+                api.nf4_double_quant(a[k], *outs[k], ws=ws[k])
+    torch.cuda.synchronize()
+    for k in range(2):
+        assert api.device_status(ws[k]) == 0, api.status_str(api.device_status(ws[k]))
+        q_ref, b_ref, mu_ref = codec.double_quant(a_np[k])
+        q, b, mu = (t.cpu().numpy() for t in outs[k])
+        assert np.float32(mu[0]).view(np.uint32) == np.float32(mu_ref).view(np.uint32)
+        assert np.array_equal(b.view(np.uint32), b_ref.view(np.uint32))
+        assert np.array_equal(q, q_ref)
+        assert _scratch_at_rest(ws[k])
+
+
+def test_quantize_dq_constants_spanning_many_binades():
+    """nf4_quantize_dq on weights whose blocks are scaled by 10^-30 .. 10^30:
+    the block constants a warp sums fall on different limbs of the exact sum,
+    which takes the lane-by-lane path; mu, scales and codes still match the
+    oracle bit for bit."""
+    rng = np.random.default_rng(95)
+    nblk = 300_001
+    w = (rng.standard_normal((nblk, 64)) * 10.0 ** rng.integers(-30, 31, (nblk, 1))).astype(np.float32)
+    Wd = torch.from_numpy(w).cuda()
+    out = api.nf4_quantize_dq(Wd)
+    torch.cuda.synchronize()
+    codes, absmax, q, b, mu = [t.cpu().numpy() for t in out]
+    c_ref, a_ref = codec.quantize(w)
+    q_ref, b_ref, mu_ref = codec.double_quant(a_ref)
+    assert np.array_equal(absmax.view(np.uint32), a_ref.view(np.uint32))
+    assert np.array_equal(codes, c_ref)
+    assert np.float32(mu[0]).view(np.uint32) == np.float32(mu_ref).view(np.uint32), (mu[0], mu_ref)
+    assert np.array_equal(b.view(np.uint32), b_ref.view(np.uint32))
+    assert np.array_equal(q, q_ref)
+
+
+def test_int8_dq_rint_ties_worked_by_hand():
+    """The hand-worked tie group (mu = 200, b = 1, quotients +-{127, 2.5, 3.5,
+    0.5, 1.5}) through the device double quantization, alone and as part of a
+    larger array whose extra constants are all equal to mu."""
+    d = np.array([127, -127, 2.5, -2.5, 3.5, -3.5, 0.5, -0.5, 1.5, -1.5], np.float64)
+    a = (200.0 + d).astype(np.float32)
+    for arr in (a, np.concatenate([a, np.full(1000, 200.0, np.float32)])):
+        q, b, mu = api.nf4_double_quant(torch.from_numpy(arr).cuda())
+        torch.cuda.synchronize()
+        assert mu.item() == 200.0 and b[0].item() == 1.0
+        assert q[:10].cpu().tolist() == [127, -127, 2, -2, 4, -4, 0, 0, 2, -2]
+
+
+@pytest.mark.parametrize("n", [1, 128])
+def test_dq_restore_order_worked_by_hand(n):
+    """ahat = fp32(mu + fp32(b rhat)) with b = 1 + 2^-23, rhat = 3, mu = -3 is
+    2^-21 (an FMA would give 3 2^-23), worked by hand.  A 128 x 64 weight whose
+    codes all hold the book's 1.0: nf4_dequant gives bf16(2^-21) everywhere,
+    and the fused forward with one-hot token rows and B = 0 returns that
+    weight, through the decode-sized kernel (n = 1) and the tensor-core GEMM
+    (n = 128)."""
+    rows, cols = 128, 64
+    nb = rows * cols // 64
+    codes = torch.full((rows * cols // 2,), 0xFF, dtype=torch.uint8, device="cuda")
+    qabs = torch.full((nb,), 3, dtype=torch.int8, device="cuda")
+    scale = torch.tensor([1.0 + 2.0 ** -23], dtype=torch.float32, device="cuda")
+    mu = torch.tensor([-3.0], dtype=torch.float32, device="cuda")
+    absmax = torch.zeros(nb, dtype=torch.float32, device="cuda")
+    wq = api.NF4Weight(codes=codes, rows=rows, cols=cols, absmax=absmax, qabs=qabs, dq_scale=scale, dq_mean=mu)
+    deq = api.nf4_dequant(wq)
+    X = torch.zeros(n, cols, dtype=torch.bfloat16, device="cuda")
+    X[torch.arange(n), torch.arange(n) % cols] = 1.0
+    A = torch.zeros(16, cols, dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros(rows, 16, dtype=torch.bfloat16, device="cuda")
+    Y, _ = api.qlora_linear_fwd(wq, X, A, B, 1.0)
+    torch.cuda.synchronize()
+    assert np.all(dev_bf16_bits(deq) == 0x3500)
+    assert np.all(dev_bf16_bits(Y) == 0x3500)

@@ -344,3 +344,36 @@ def test_backwards_on_two_unordered_streams_and_in_a_graph():
         _compare("dX", f64(dev_bf16_bits(alone[i][0])), dXr)
         _compare("dA", alone[i][1].double().cpu().numpy(), dAr)
         _compare("dB", alone[i][2].double().cpu().numpy(), dBr)
+
+
+ADAPTER_CASES = [synthetic.DECODE[4],                                               # the decode-sized kernel
+                 synthetic.custom("adapter_tc_1024x2048_n512_r16", 1024, 2048, 512, 16, s=2.0, index=48)]  # tcgen05
+
+
+@pytest.mark.parametrize("cfg", ADAPTER_CASES, ids=lambda c: c.name)
+def test_adapter_terms_alone(cfg):
+    """The adapter term on its own ("LoRA 与 QLoRA", section LoRA: y = W0 x +
+    s B(A x)): Y(B) - Y(B = 0) against the oracle's s U B^T, and dX(B) - dX(B = 0)
+    against s G A with G = dY B, each normwise against its own magnitude.  B is
+    drawn with sigma 0.5 (25 to 50 times the workload's) so the adapter term is
+    about as large as the frozen-weight term.  Tolerance: the 2e-2 target plus the two bf16
+    roundings of the outputs being subtracted (half an ulp each, at most 2^-9
+    of the larger output), relative to the adapter term's magnitude."""
+    w, X, A, _, dY = workload(cfg)
+    B = synthetic.to_bf16_bits(synthetic.normal_f32((cfg.dout, cfg.r), 0.5, 4800 + cfg.index))
+    wq = _gpu_weight(w)
+    Xd, Ad, Bd, dYd = bf16_to_dev(X), bf16_to_dev(A), bf16_to_dev(B), bf16_to_dev(dY)
+    B0 = torch.zeros_like(Bd)
+    Y1, U1 = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s)
+    Y0, _ = api.qlora_linear_fwd(wq, Xd, Ad, B0, cfg.s)
+    dX1, _, _ = api.qlora_linear_bwd(wq, Xd, Ad, Bd, cfg.s, dYd, U=U1)
+    dX0, _, _ = api.qlora_linear_bwd(wq, Xd, Ad, B0, cfg.s, dYd, U=U1)
+    torch.cuda.synchronize()
+    Xf, Af, Bf, dYf = f64(X), f64(A), f64(B), f64(dY)
+    for name, (t1, t0), ref in (("Y adapter", (Y1, Y0), cfg.s * (Xf @ Af.T) @ Bf.T),
+                                ("dX adapter", (dX1, dX0), cfg.s * (dYf @ Bf) @ Af)):
+        a1, a0 = f64(dev_bf16_bits(t1)), f64(dev_bf16_bits(t0))
+        scale = np.max(np.abs(ref))
+        tol = TOL + 2.0 ** -9 * (np.max(np.abs(a1)) + np.max(np.abs(a0))) / scale
+        assert scale > 0.5 * np.max(np.abs(a0)), (name, "adapter term too small to test")
+        _compare(name, a1 - a0, ref, tol=tol)

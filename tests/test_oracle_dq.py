@@ -126,6 +126,41 @@ def test_dq_degenerate_groups():
     assert mu == 0 and np.all(qabs == 0)
 
 
+def test_int8_dq_rint_ties_worked_by_hand():
+    """A group whose quotients are exact halves ("LoRA 与 QLoRA" section 2:
+    r_j = (a_j - mu) / b rounded to 8 bits), worked by hand.  The constants are
+    mu +- {127, 2.5, 3.5, 0.5, 1.5} with mu = 200: the exact mean is 200, so
+    d_j = a_j - 200 exactly, max|d| = 127 gives b = 127 / 127 = 1 exactly, and
+    r_j = d_j.  Ties go to the even integer: 2.5 -> 2, 3.5 -> 4, 0.5 -> 0,
+    1.5 -> 2 (and the negatives likewise).  Rounding half away from zero
+    (3, 4, 1, 2) or truncation (2, 3, 0, 1) fails here."""
+    d = np.array([127, -127, 2.5, -2.5, 3.5, -3.5, 0.5, -0.5, 1.5, -1.5], np.float64)
+    a = (200.0 + d).astype(np.float32)
+    assert np.array_equal(a.astype(np.float64) - 200.0, d)       # the constants are exact
+    qabs, scale, mu = codec.double_quant(a)
+    assert mu == np.float32(200.0) and scale.tolist() == [1.0]
+    assert qabs.tolist() == [127, -127, 2, -2, 4, -4, 0, 0, 2, -2]
+
+
+def test_dq_restore_order_worked_by_hand():
+    """ahat = mu + b rhat ("LoRA 与 QLoRA" section 2), in the written order:
+    the product rounded to fp32 first, then the sum.  Worked by hand with
+    b = 1 + 2^-23, rhat = 3, mu = -3: b rhat = 3 + 3 2^-23 lies halfway
+    between the fp32 neighbours 3 + 2^-22 and 3 + 2^-21 (the spacing near 3 is
+    2^-22) and rounds to the even one, 3 + 2^-21; adding mu = -3 is then exact,
+    ahat = 2^-21.  A fused multiply-add rounds once, to 3 2^-23."""
+    b = np.float32(1.0 + 2.0 ** -23)
+    assert float(b) == 1.0 + 2.0 ** -23
+    got = codec.dq_restore(np.array([3], np.int8), np.array([b], np.float32), np.float32(-3.0))
+    assert float(got[0]) == 2.0 ** -21
+    fma = float(np.float32(float(b) * 3.0 + (-3.0)))              # one rounding of the exact value
+    assert fma == 3 * 2.0 ** -23 and fma != float(got[0])
+    # and the doubleDequant of a block whose codes all hold the book's 1.0 (code 15)
+    codes = np.full(32, 0xFF, np.uint8)
+    bf = codec.dequant(codes, 64, qabs=np.array([3], np.int8), scale=np.array([b], np.float32), mu=np.float32(-3.0))
+    assert np.all(bf == 0x3500)                                   # bf16 bits of 2^-21
+
+
 def test_bf16_rounding_against_torch():
     g = np.random.Generator(np.random.PCG64(37))
     x = (g.standard_normal(200000) * 10.0 ** g.integers(-30, 30, 200000)).astype(np.float32)
