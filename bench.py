@@ -312,8 +312,10 @@ def measure_decode(api, dev, copies=64, reps=5):
 def measure_sweep(api, dev, use_graph=True):
     """Quantize + DQ and dequant of every linear of a 32-layer d=4096,
     ffn=11008 decoder (6.48 B parameters, generated on the device), one pass
-    each, CUDA events around each pass.  Each pass is a CUDA graph of all 224
-    matrices' calls (use_graph=False: enqueued from Python)."""
+    each, CUDA events around each pass.  Quantize + DQ is one
+    nf4_quantize_dq_batch call over all 224 matrices; dequant is one
+    nf4_dequant call per matrix.  Each pass is a CUDA graph (use_graph=False:
+    enqueued from Python)."""
     import torch
     from bit_nf4_quantized_07_b200 import synthetic
     gen = torch.Generator(device=dev)
@@ -328,17 +330,16 @@ def measure_sweep(api, dev, use_graph=True):
                          torch.empty(nb, dtype=torch.int8, device=dev),
                          torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev),
                          torch.empty(1, dtype=torch.float32, device=dev)))
-    maxnb = max(m[2].numel() for m in mats)
-    ws = api.alloc_workspace(api.workspace_bytes(api.OP_DOUBLE_QUANT, maxnb), dev)
+    ws = api.alloc_workspace(api.workspace_bytes(api.OP_QUANTIZE_DQ_BATCH, len(mats)), dev)
+    jobs = [(W, c, a, q, sc, mu, "int8") for (W, c, a, q, sc, mu) in mats]
     outbuf = {}
     for W, *_ in mats:
         outbuf.setdefault(tuple(W.shape), torch.empty(W.shape, dtype=torch.bfloat16, device=dev))
     wq = [api.NF4Weight(codes=c, rows=W.shape[0], cols=W.shape[1], absmax=a, qabs=q, dq_scale=sc, dq_mean=mu)
           for (W, c, a, q, sc, mu) in mats]
 
-    def quant_pass():
-        for (W, c, a, q, sc, mu) in mats:
-            api.nf4_quantize_dq(W, c, a, q, sc, mu, ws=ws)
+    def quant_pass():  # the whole model in one call
+        api.nf4_quantize_dq_batch(jobs, ws=ws)
 
     def deq_pass():
         for w in wq:
@@ -371,7 +372,7 @@ def measure_sweep(api, dev, use_graph=True):
     params = synthetic.sweep_params()
     qb, db = codec_bytes_per_param()
     tq, td = e[0].elapsed_time(e[1]) * 1e-3, e[1].elapsed_time(e[2]) * 1e-3
-    del mats, wq, outbuf
+    del mats, jobs, wq, outbuf
     torch.cuda.empty_cache()
     return {"params": params, "quantize_dq_ms": tq * 1e3, "quantize_dq_GBs": params * qb / tq / 1e9,
             "dequant_ms": td * 1e3, "dequant_GBs": params * db / td / 1e9}

@@ -22,10 +22,10 @@ LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
 QLN_OK = 0
 STATUS_NAMES = {0: "QLN_OK", 1: "QLN_ERR_NULL", 2: "QLN_ERR_SHAPE", 3: "QLN_ERR_ALIGN", 4: "QLN_ERR_WORKSPACE",
                 5: "QLN_ERR_ARCH", 6: "QLN_ERR_CUDA", 7: "QLN_ERR_TIMEOUT", 8: "QLN_ERR_INTERNAL"}
-OP_DOUBLE_QUANT, OP_LINEAR_FWD, OP_LINEAR_BWD = 1, 2, 3
+OP_DOUBLE_QUANT, OP_LINEAR_FWD, OP_LINEAR_BWD, OP_QUANTIZE_DQ_BATCH = 1, 2, 3, 4
 
 #: Every symbol include/qlora_nf4.h declares.
-EXPORTS = ("nf4_quantize", "nf4_quantize_ex", "nf4_quantize_dq", "nf4_double_quant", "nf4_double_quant_ex", "nf4_double_quant_noalloc",
+EXPORTS = ("nf4_quantize", "nf4_quantize_ex", "nf4_quantize_dq", "nf4_quantize_dq_batch", "nf4_double_quant", "nf4_double_quant_ex", "nf4_double_quant_noalloc",
            "nf4_dequant",
            "nf4_dequant_flat", "qlora_linear_fwd", "qlora_linear_bwd", "qln_workspace_bytes", "qln_codebook",
            "qln_status_str", "qln_version", "qln_launch_count", "qln_adamw_step")
@@ -45,6 +45,12 @@ class CAdamWConfig(ctypes.Structure):
 
 
 ADAMW_PAGE_IN, ADAMW_PAGE_OUT = 1, 2
+
+
+class CQuantJob(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("numel", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("dq_format", ctypes.c_int32), ("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p),
+                ("qabs", ctypes.c_void_p), ("dq_scale", ctypes.c_void_p), ("dq_mean", ctypes.c_void_p)]
 
 
 class CNF4Weight(ctypes.Structure):
@@ -69,6 +75,7 @@ def lib():
             "nf4_quantize": ([P, I64, P, P, P], I32),
             "nf4_quantize_ex": ([P, I32, I64, P, P, P], I32),
             "nf4_quantize_dq": ([P, I32, I64, I32, P, P, P, P, P, P, SZ, P], I32),
+            "nf4_quantize_dq_batch": ([P, I32, P, SZ, P], I32),
             "nf4_double_quant": ([P, I64, P, P, P, P, SZ, P], I32),
             "nf4_double_quant_ex": ([P, I64, I32, P, P, P, P, SZ, P], I32),
             "nf4_double_quant_noalloc": ([P, I64, P, P, P, P], I32),
@@ -213,6 +220,31 @@ def nf4_quantize_dq(W: torch.Tensor, codes=None, absmax=None, qabs=None, dq_scal
                                                     _p(absmax), _p(qabs), _p(dq_scale), _p(dq_mean), _p(ws),
                                                     ws.numel(), _stream()))
     return codes, absmax, qabs, dq_scale, dq_mean
+
+
+def nf4_quantize_dq_batch(jobs, ws=None):
+    """nf4_quantize_dq of several weights in one call (nf4_quantize_dq_batch).
+
+    jobs: a sequence of (W, codes, absmax, qabs, dq_scale, dq_mean, fmt)
+    tuples with the outputs allocated as nf4_quantize_dq would."""
+    jobs = list(jobs)
+    arr = (CQuantJob * len(jobs))()
+    dev = jobs[0][0].device if jobs else None
+    for i, (W, codes, absmax, qabs, dq_scale, dq_mean, fmt) in enumerate(jobs):
+        if W.dtype not in _DTYPES:
+            raise ValueError(f"unsupported weight dtype {W.dtype}")
+        _need_cuda(W, codes, absmax, qabs, dq_scale, dq_mean)
+        n = W.numel()
+        nb = (n + 63) // 64
+        if (codes.numel() < (n + 1) // 2 or absmax.numel() < nb or qabs.numel() < nb
+                or dq_scale.numel() < (nb + 255) // 256 or dq_mean.numel() < 1):
+            raise ValueError(f"job {i}: an output is too small")
+        arr[i] = CQuantJob(_p(W), n, _DTYPES[W.dtype], DQ_FORMATS[fmt], _p(codes), _p(absmax), _p(qabs),
+                           _p(dq_scale), _p(dq_mean))
+    if ws is None:
+        ws = alloc_workspace(workspace_bytes(OP_QUANTIZE_DQ_BATCH, len(jobs)), dev)
+    _need_cuda(ws)
+    _check("nf4_quantize_dq_batch", lib().nf4_quantize_dq_batch(arr, len(jobs), _p(ws), ws.numel(), _stream()))
 
 
 def nf4_double_quant(absmax: torch.Tensor, qabs=None, dq_scale=None, dq_mean=None, ws=None, fmt: str = "int8"):

@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <vector>
 
 #include "qln_common.cuh"
 #include "qln_internal.h"
@@ -18,6 +19,7 @@ namespace {
 using qln::note_launch;
 
 constexpr int kMaxDevices = 64;
+constexpr int32_t kMaxBatchJobs = 1 << 20;  // jobs per nf4_quantize_dq_batch call
 int g_arch_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
 int g_num_sms[kMaxDevices];
 
@@ -196,6 +198,38 @@ qln_status nf4_quantize_dq(const void *W, int32_t dtype, int64_t numel, int32_t 
                                                     dq_format == QLN_DQ_E4M3, (cudaStream_t)stream, sms));
 }
 
+static qln_status check_quant_job(const qln_quant_job &j) {
+    if (!j.W || !j.codes || !j.absmax || !j.qabs || !j.dq_scale || !j.dq_mean) return QLN_ERR_NULL;
+    if (j.numel <= 0 || (j.numel + 63) / 64 > qln::dq_max_blocks()) return QLN_ERR_SHAPE;
+    if (j.dtype != QLN_DTYPE_F32 && j.dtype != QLN_DTYPE_BF16 && j.dtype != QLN_DTYPE_F16) return QLN_ERR_SHAPE;
+    if (j.dq_format != QLN_DQ_INT8 && j.dq_format != QLN_DQ_E4M3) return QLN_ERR_SHAPE;
+    if (!aligned(j.W, 16) || !aligned(j.codes, 16) || !aligned(j.absmax, 16) || !aligned(j.qabs, 4) ||
+        !aligned(j.dq_scale, 4) || !aligned(j.dq_mean, 4))
+        return QLN_ERR_ALIGN;
+    return QLN_OK;
+}
+
+qln_status nf4_quantize_dq_batch(const qln_quant_job *jobs, int32_t njobs, void *ws, size_t ws_bytes, void *stream) {
+    if (!jobs || !ws) return QLN_ERR_NULL;
+    if (njobs < 1 || njobs > kMaxBatchJobs) return QLN_ERR_SHAPE;
+    if (!aligned(ws, 256)) return QLN_ERR_ALIGN;
+    for (int32_t i = 0; i < njobs; ++i) {
+        const qln_status s = check_quant_job(jobs[i]);
+        if (s != QLN_OK) return s;
+    }
+    if (ws_bytes < qln::kDqBatchScratchBytes * (size_t)njobs) return QLN_ERR_WORKSPACE;
+    int sms = 0;
+    qln_status s = check_device(&sms);
+    if (s != QLN_OK) return s;
+    std::vector<qln::QuantJob> q((size_t)njobs);
+    for (int32_t i = 0; i < njobs; ++i) {
+        const qln_quant_job &j = jobs[i];
+        q[(size_t)i] = qln::QuantJob{j.W, j.dtype, j.numel, j.codes, j.absmax, static_cast<int8_t *>(j.qabs),
+                                     j.dq_scale, j.dq_mean, j.dq_format == QLN_DQ_E4M3};
+    }
+    return from_cuda(qln::launch_nf4_quantize_dq_batch(q.data(), njobs, ws, (cudaStream_t)stream, sms));
+}
+
 qln_status nf4_double_quant(const float *absmax, int64_t nb, int8_t *qabs, float *dq_scale, float *dq_mean,
                             void *ws, size_t ws_bytes, void *stream) {
     return nf4_double_quant_ex(absmax, nb, QLN_DQ_INT8, qabs, dq_scale, dq_mean, ws, ws_bytes, stream);
@@ -348,6 +382,8 @@ size_t qln_workspace_bytes(int32_t op, int64_t rows, int64_t cols, int64_t n, in
             return (rows > 0 && cols > 0 && n > 0 && r > 0) ? fwd_layout(rows, cols, n, r).total : 0;
         case QLN_OP_LINEAR_BWD:
             return (rows > 0 && cols > 0 && n > 0 && r > 0) ? bwd_layout(rows, cols, n, r).total : 0;
+        case QLN_OP_QUANTIZE_DQ_BATCH:
+            return (rows > 0 && rows <= kMaxBatchJobs) ? qln::kDqBatchScratchBytes * (size_t)rows : 0;
         default:
             return 0;
     }

@@ -6,8 +6,10 @@
 // "Double Quantization" and "QLoRA" (doubleDequant: constants first);
 // "LoRA 与 QLoRA" section QLoRA 2 (a_j = max|W_j| per 64 weights,
 // r_j = (a_j - mu)/b, 8-bit rhat_j, ahat_j = mu + b rhat_j).
+#include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -480,16 +482,18 @@ __device__ __forceinline__ bool dq_arrive(const DqScratch &sc, unsigned g, int G
     return true;
 }
 
-// 8 consecutive constants starting at j (zeros past nb).
-__device__ __forceinline__ void load8_const(float (&v)[8], const float *__restrict__ a, int64_t j, int64_t nb) {
+// 8 consecutive constants starting at j (zeros past nb), read through L2: they
+// come from the previous kernel, which may still have been running when this
+// one started (programmatic dependent launch).
+__device__ __forceinline__ void load8_const(float (&v)[8], const float *a, int64_t j, int64_t nb) {
     if (j + 8 <= nb) {
-        const float4 x = __ldg(reinterpret_cast<const float4 *>(a + j));
-        const float4 y = __ldg(reinterpret_cast<const float4 *>(a + j + 4));
+        const float4 x = __ldcg(reinterpret_cast<const float4 *>(a + j));
+        const float4 y = __ldcg(reinterpret_cast<const float4 *>(a + j + 4));
         v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
         v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
     } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = (j + i < nb) ? a[j + i] : 0.f;
+        for (int i = 0; i < 8; ++i) v[i] = (j + i < nb) ? __ldcg(a + j + i) : 0.f;
     }
 }
 
@@ -546,6 +550,78 @@ __device__ __forceinline__ uint64_t dqf_timer_ns() {
     return t;
 }
 
+// ===========================================================================
+// Deferred double quantization (the batch entry point).  A quantize kernel of
+// job i can also carry, before its own chunks, two pieces of the double
+// quantization of earlier jobs whose block constants are complete because
+// their quantize has finished:
+//  * the exact sum of job i-1's constants into that job's scratch bank (the
+//    last CTA to arrive advances the generation, as K2 does), and
+//  * the group quantization of job i-2, with mu formed from its bank (as K3).
+// Every kernel still waits for the one before it, so nothing runs concurrently
+// with anything it depends on; the double quantization's latency simply hides
+// behind the next weight's stream.
+// ===========================================================================
+struct DqPhases {
+    const float *s_absmax;  // sum phase: null for none
+    int64_t s_nb;
+    unsigned char *s_ws;
+    const float *g_absmax;  // group phase: null for none
+    int64_t g_nb;
+    unsigned char *g_ws;
+    int8_t *g_qabs;
+    float *g_scale;
+    float *g_mu;
+    int g_e4m3;
+    int *status;  // cleared by CTA 0 when not null
+};
+
+// Both phases with the whole grid (any block size that is a multiple of 32);
+// every thread of every CTA calls it.  slim: kXLimbs words of shared memory.
+__device__ __noinline__ void dq_run_phases(const DqPhases &ph, unsigned long long *slim, float *mu_s,
+                                           unsigned *gen_s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    if (ph.status && blockIdx.x == 0 && threadIdx.x == 0) *ph.status = QLN_OK;
+    const DqScratch gs = dq_scratch(ph.g_ws, false);
+    if (ph.g_absmax && warp == 0) {  // mu of job i-2: its sum advanced the generation
+        const float mu = xsum_mean_warp(gs.bank[(__ldcg(gs.gen) + 1) & 1], (uint32_t)ph.g_nb);
+        if (lane == 0) {
+            *mu_s = mu;
+            if (blockIdx.x == 0) *ph.g_mu = mu;
+        }
+    }
+    if (ph.s_absmax) {  // the exact sum of job i-1, 8 consecutive constants per thread and pass
+        const DqScratch ss = dq_scratch(ph.s_ws, false);
+        if (threadIdx.x < kXLimbs) slim[threadIdx.x] = 0ull;
+        const unsigned g0 = dq_read_gen(ss, gen_s);  // includes a __syncthreads
+        XRun x;
+        const int64_t step = (int64_t)gridDim.x * blockDim.x * 8;
+        for (int64_t j = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; j < ph.s_nb; j += step) {
+            float v[8];
+            load8_const(v, ph.s_absmax, j, ph.s_nb);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) xsum_add(x, v[u], slim);
+        }
+        xsum_flush_warp(x, slim);
+        __syncthreads();
+        if (threadIdx.x < kXLimbs && slim[threadIdx.x] != 0ull)
+            atomicAdd(&ss.bank[g0 & 1][threadIdx.x], slim[threadIdx.x]);
+        __syncthreads();
+        if (threadIdx.x == 0) dq_arrive(ss, g0, (int)gridDim.x);
+    }
+    __syncthreads();  // mu is in shared memory
+    if (ph.g_absmax) {
+        const float mu = *mu_s;
+        const int64_t ng = (ph.g_nb + kDqGroup - 1) / kDqGroup;
+        for (int64_t g = (int64_t)blockIdx.x * nw + warp; g < ng; g += (int64_t)gridDim.x * nw) {
+            float e[8];
+            load8_const(e, ph.g_absmax, g * kDqGroup + 8 * lane, ph.g_nb);
+            dq_quantize_group(e, g * kDqGroup + 8 * lane, ph.g_nb, mu, ph.g_e4m3 != 0, lane, g, ph.g_qabs,
+                              ph.g_scale);
+        }
+    }
+}
+
 constexpr int kQzWarps = 24;       // two CTAs of 24 warps per SM
 constexpr int kQzCtasPerSm = 2;
 constexpr int kQzStages = 3;       // chunks per warp ring
@@ -563,7 +639,16 @@ constexpr int kQzLutBytes = 256 * 128;                                    // 256
 // lane's last partial code word is written byte by byte.  Idx is 32-bit
 // whenever every element offset stays below 2^31.
 
-template <typename T, typename Idx>
+//
+// kLateWait (the batch entry point, second weight on, buffers of all jobs
+// disjoint): the kernel reads only the caller's weight, which was complete
+// before the batch's first launch passed its wait, and writes only its own
+// outputs, which nothing else in the batch touches; so it releases its
+// dependents and starts at once, filling the SMs the previous weight's
+// kernels leave, and waits for its predecessor only at its end -- its
+// completion then still implies that everything before it in the stream has
+// completed.
+template <typename T, typename Idx, bool kLateWait>
 __global__ void __launch_bounds__(kQzThreads, kQzCtasPerSm) nf4_quantize_kernel(const T *__restrict__ W, Idx numel,
                                                                                 uint8_t *__restrict__ codes,
                                                                                 float *__restrict__ absmax) {
@@ -572,7 +657,7 @@ __global__ void __launch_bounds__(kQzThreads, kQzCtasPerSm) nf4_quantize_kernel(
     for (int i = threadIdx.x; i < kQzLutBytes / 4; i += kQzThreads)  // bucket i/32, lane i%32
         reinterpret_cast<uint32_t *>(qz_smem)[i] = kSnapTable.e[i >> 5];
     __syncthreads();
-    pdl_wait();  // W may come from the previous kernel; codes/absmax may still be read by it
+    if (!kLateWait) pdl_wait();  // W may come from the previous kernel; codes/absmax may still be read by it
     pdl_trigger();
 
     const int lane = threadIdx.x & 31;
@@ -647,11 +732,12 @@ __global__ void __launch_bounds__(kQzThreads, kQzCtasPerSm) nf4_quantize_kernel(
         slot = (slot + 1 == kQzStages) ? 0 : slot + 1;
     }
     cp_async_wait<0>();
+    if (kLateWait) pdl_wait();
 }
 
 // Launch of the quantize kernel: a persistent grid of up to two CTAs per SM,
 // as a programmatic dependent.
-template <typename T, typename Idx>
+template <typename T, typename Idx, bool kLateWait>
 static cudaError_t launch_quantize_t(const T *W, int64_t numel, uint8_t *codes, float *absmax, cudaStream_t st,
                                      int num_sms) {
     const int64_t nchunks = ((numel + 63) / 64 + 3) / 4;
@@ -659,29 +745,35 @@ static cudaError_t launch_quantize_t(const T *W, int64_t numel, uint8_t *codes, 
     if (grid > (int64_t)kQzCtasPerSm * num_sms) grid = (int64_t)kQzCtasPerSm * num_sms;
     if (grid < 1) grid = 1;
     const int smem = kQzLutBytes + kQzWarps * kQzStages * 256 * QzIn<T>::kBytes;
-    auto kern = nf4_quantize_kernel<T, Idx>;
+    auto kern = nf4_quantize_kernel<T, Idx, kLateWait>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3((unsigned)grid), dim3(kQzThreads), (size_t)smem, st, W, (Idx)numel, codes, absmax);
 }
 
-template <typename T>
+template <typename T, bool kLateWait>
 static cudaError_t launch_quantize_any(const void *W, int64_t numel, uint8_t *codes, float *absmax, cudaStream_t st,
                                        int num_sms) {
     const T *w = static_cast<const T *>(W);
     // 32-bit indices while every element offset (and a chunk look-ahead per warp) stays below 2^31
     if (numel + (int64_t)256 * (kQzStages + 1) * kQzCtasPerSm * num_sms * kQzWarps < ((int64_t)1 << 31))
-        return launch_quantize_t<T, uint32_t>(w, numel, codes, absmax, st, num_sms);
-    return launch_quantize_t<T, int64_t>(w, numel, codes, absmax, st, num_sms);
+        return launch_quantize_t<T, uint32_t, kLateWait>(w, numel, codes, absmax, st, num_sms);
+    return launch_quantize_t<T, int64_t, kLateWait>(w, numel, codes, absmax, st, num_sms);
+}
+
+template <bool kLateWait>
+static cudaError_t launch_quantize_dtype(const void *W, int dtype, int64_t numel, uint8_t *codes, float *absmax,
+                                         cudaStream_t st, int num_sms) {
+    switch (dtype) {
+        case QLN_DTYPE_BF16: return launch_quantize_any<Bf16In, kLateWait>(W, numel, codes, absmax, st, num_sms);
+        case QLN_DTYPE_F16: return launch_quantize_any<F16In, kLateWait>(W, numel, codes, absmax, st, num_sms);
+        default: return launch_quantize_any<float, kLateWait>(W, numel, codes, absmax, st, num_sms);
+    }
 }
 
 cudaError_t launch_nf4_quantize(const void *W, int dtype, int64_t numel, uint8_t *codes, float *absmax,
                                 cudaStream_t st, int num_sms) {
-    switch (dtype) {
-        case QLN_DTYPE_BF16: return launch_quantize_any<Bf16In>(W, numel, codes, absmax, st, num_sms);
-        case QLN_DTYPE_F16: return launch_quantize_any<F16In>(W, numel, codes, absmax, st, num_sms);
-        default: return launch_quantize_any<float>(W, numel, codes, absmax, st, num_sms);
-    }
+    return launch_quantize_dtype<false>(W, dtype, numel, codes, absmax, st, num_sms);
 }
 
 template <int P>
@@ -958,6 +1050,130 @@ cudaError_t launch_nf4_quantize_dq(const void *W, int dtype, int64_t numel, uint
     cudaError_t e = launch_nf4_quantize(W, dtype, numel, codes, absmax, st, num_sms);
     if (e != cudaSuccess) return e;
     return launch_nf4_double_quant(absmax, (numel + 63) / 64, qabs, scale, mu, ws, e4m3, st, num_sms);
+}
+
+static_assert(kDqScratchBytes == kDqBatchScratchBytes, "one DQ scratch per batch job");
+
+// The deferred double quantization of a batch, one small CTA per SM: 128
+// threads of at most 32 registers fit beside the two quantize CTAs of an SM
+// (the registers those leave free), so it runs alongside the quantize
+// kernels.  It always waits for its predecessor before touching memory;
+// kEarlyRelease lets the next weight's quantize start before that wait (only
+// for a batch whose buffers are disjoint, see kLateWait).
+constexpr int kPhThreads = 128;
+template <bool kEarlyRelease>
+__global__ void __launch_bounds__(kPhThreads, 16) dq_phase_kernel(DqPhases ph) {
+    __shared__ unsigned long long slim[kXLimbs];
+    __shared__ float mu_s;
+    __shared__ unsigned gen_s;
+    if (kEarlyRelease) pdl_trigger();
+    pdl_wait();
+    if (!kEarlyRelease) pdl_trigger();
+    dq_run_phases(ph, slim, &mu_s, &gen_s);
+}
+
+namespace {
+struct ByteRange {
+    uintptr_t lo, hi;  // [lo, hi)
+    int job;           // -1: the workspace
+    bool write;
+};
+
+// True when no range written by one job (or the workspace) overlaps any range
+// of another job: then the quantize kernels of different weights and the
+// deferred double quantization may run at the same time.
+bool batch_disjoint(const QuantJob *jobs, int njobs, const void *ws) {
+    std::vector<ByteRange> r;
+    r.reserve((size_t)njobs * 6 + 1);
+    auto add = [&](const void *p, size_t n, int job, bool write) {
+        if (n) r.push_back({(uintptr_t)p, (uintptr_t)p + n, job, write});
+    };
+    for (int i = 0; i < njobs; ++i) {
+        const QuantJob &q = jobs[i];
+        const size_t nb = (size_t)((q.numel + 63) / 64);
+        add(q.W, (size_t)q.numel * (q.dtype == QLN_DTYPE_F32 ? 4 : 2), i, false);
+        add(q.codes, (size_t)((q.numel + 1) / 2), i, true);
+        add(q.absmax, nb * 4, i, true);
+        add(q.qabs, nb, i, true);
+        add(q.scale, ((nb + kDqGroup - 1) / kDqGroup) * 4, i, true);
+        add(q.mu, 4, i, true);
+    }
+    add(ws, kDqScratchBytes * (size_t)njobs, -1, true);
+    std::sort(r.begin(), r.end(), [](const ByteRange &a, const ByteRange &b) { return a.lo < b.lo; });
+    // sweep: every range against the earlier ranges still open
+    std::vector<size_t> open;
+    for (size_t k = 0; k < r.size(); ++k) {
+        size_t keep = 0;
+        for (size_t t = 0; t < open.size(); ++t) {
+            const ByteRange &o = r[open[t]];
+            if (o.hi <= r[k].lo) continue;  // closed
+            open[keep++] = open[t];
+            if (o.job != r[k].job && (o.write || r[k].write)) return false;
+        }
+        open.resize(keep);
+        open.push_back(k);
+    }
+    return true;
+}
+}  // namespace
+
+// Batch: quantize(0); then for i >= 1 the phase launch (sum of weight i-1,
+// groups of weight i-2) followed by quantize(i); then the two tail phase
+// launches (sum of n-1 and groups of n-2; groups of n-1).  Every phase launch
+// waits for the quantize before it, whose completion implies that of all
+// earlier launches (a late-waiting quantize waits at its end), so each phase
+// reads only completed constants and sums.  With disjoint buffers the
+// quantize kernels start early (see kLateWait); otherwise every launch waits
+// at its start as usual.  Job i's scratch is ws + 256 i; the first phase
+// launch clears the status word at ws + 0.
+cudaError_t launch_nf4_quantize_dq_batch(const QuantJob *jobs, int njobs, void *ws, cudaStream_t st, int num_sms) {
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    auto scratch = [&](int i) { return w + kDqScratchBytes * (size_t)i; };
+    auto nb_of = [&](int i) { return (jobs[i].numel + 63) / 64; };
+    bool status_cleared = false;
+    auto phases = [&](int s_job, int g_job) {  // -1: none
+        DqPhases ph{};
+        if (s_job >= 0) {
+            ph.s_absmax = jobs[s_job].absmax;
+            ph.s_nb = nb_of(s_job);
+            ph.s_ws = scratch(s_job);
+        }
+        if (g_job >= 0) {
+            ph.g_absmax = jobs[g_job].absmax;
+            ph.g_nb = nb_of(g_job);
+            ph.g_ws = scratch(g_job);
+            ph.g_qabs = jobs[g_job].qabs;
+            ph.g_scale = jobs[g_job].scale;
+            ph.g_mu = jobs[g_job].mu;
+            ph.g_e4m3 = jobs[g_job].e4m3 ? 1 : 0;
+        }
+        if (!status_cleared) {
+            ph.status = reinterpret_cast<int *>(w);
+            status_cleared = true;
+        }
+        return ph;
+    };
+    const bool overlap = batch_disjoint(jobs, njobs, ws);
+    cudaError_t e = launch_quantize_dtype<false>(jobs[0].W, jobs[0].dtype, jobs[0].numel, jobs[0].codes,
+                                                 jobs[0].absmax, st, num_sms);
+    if (e != cudaSuccess) return e;
+    for (int i = 1; i < njobs; ++i) {
+        const QuantJob &q = jobs[i];
+        if (overlap) {
+            e = launch_pdl(dq_phase_kernel<true>, dim3(num_sms), dim3(kPhThreads), 0, st, phases(i - 1, i - 2));
+            if (e == cudaSuccess)
+                e = launch_quantize_dtype<true>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
+        } else {
+            e = launch_pdl(dq_phase_kernel<false>, dim3(num_sms), dim3(kPhThreads), 0, st, phases(i - 1, i - 2));
+            if (e == cudaSuccess)
+                e = launch_quantize_dtype<false>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
+        }
+        if (e != cudaSuccess) return e;
+    }
+    const int tail_grid = 4 * num_sms;
+    e = launch_pdl(dq_phase_kernel<false>, dim3(tail_grid), dim3(kPhThreads), 0, st, phases(njobs - 1, njobs - 2));
+    if (e != cudaSuccess) return e;
+    return launch_pdl(dq_phase_kernel<false>, dim3(tail_grid), dim3(kPhThreads), 0, st, phases(-1, njobs - 1));
 }
 
 // ===========================================================================

@@ -1,5 +1,7 @@
 // Fused NF4 doubleDequant + GEMM on the register-level mma.sync tensor path.
-// Serves token counts too small to fill a tcgen05 tile (decode-shaped calls).
+// Serves the token counts between the decode-sized forward (n <= 32) and the
+// tcgen05 GEMM (n >= 64), i.e. 32 < n < 64, and any shape the decode-sized
+// kernel does not take; and the dX GEMM for n < 64.
 //
 // Method: "LoRA 与 QLoRA" section QLoRA 1 (4-bit weight -> dequant -> BF16
 // -> GEMM); jjjymmm.cn "QLoRA" (doubleDequant: constants first, then the

@@ -43,6 +43,20 @@ cudaError_t launch_nf4_double_quant(const float *absmax, int64_t nb, int8_t *qab
 cudaError_t launch_nf4_quantize_dq(const void *W, int dtype, int64_t numel, uint8_t *codes, float *absmax,
                                    int8_t *qabs, float *scale, float *mu, void *ws, bool e4m3, cudaStream_t st,
                                    int num_sms);
+// One weight of a quantize + double quantization batch (validated by the caller).
+struct QuantJob {
+    const void *W;
+    int dtype;
+    int64_t numel;
+    uint8_t *codes;
+    float *absmax;
+    int8_t *qabs;
+    float *scale;
+    float *mu;
+    bool e4m3;
+};
+cudaError_t launch_nf4_quantize_dq_batch(const QuantJob *jobs, int njobs, void *ws, cudaStream_t st, int num_sms);
+constexpr size_t kDqBatchScratchBytes = 256;  // per job
 cudaError_t launch_nf4_dequant(const qln_nf4_weight *w, uint16_t *out, cudaStream_t st, int num_sms);
 cudaError_t launch_adamw(float *p, const float *g, float *m, float *v, uint16_t *p_bf16, int64_t n, float lr,
                          float b1, float b2, float eps, float wd, const int64_t *step, int flags, cudaStream_t st,

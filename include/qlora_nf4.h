@@ -93,7 +93,7 @@ enum { QLN_DQ_INT8 = 0, QLN_DQ_E4M3 = 1 };
 enum { QLN_DTYPE_F32 = 0, QLN_DTYPE_BF16 = 1, QLN_DTYPE_F16 = 2 };
 
 /* Workspace-sized operations (qln_workspace_bytes `op`). */
-enum { QLN_OP_DOUBLE_QUANT = 1, QLN_OP_LINEAR_FWD = 2, QLN_OP_LINEAR_BWD = 3 };
+enum { QLN_OP_DOUBLE_QUANT = 1, QLN_OP_LINEAR_FWD = 2, QLN_OP_LINEAR_BWD = 3, QLN_OP_QUANTIZE_DQ_BATCH = 4 };
 
 /* An NF4 weight as stored by nf4_quantize (+ nf4_double_quant).  All pointers
  * are device pointers owned by the caller.  With qabs != NULL the weight is
@@ -221,6 +221,45 @@ QLN_API qln_status nf4_double_quant_ex(const float *absmax, int64_t nb, int32_t 
 QLN_API qln_status nf4_quantize_dq(const void *W, int32_t dtype, int64_t numel, int32_t dq_format, uint8_t *codes,
                                    float *absmax, void *qabs, float *dq_scale, float *dq_mean, void *ws,
                                    size_t ws_bytes, void *stream);
+
+/* One weight of nf4_quantize_dq_batch: the arguments of nf4_quantize_dq. */
+typedef struct {
+    const void *W;     /* [numel] weights of dtype, 16-byte aligned */
+    int64_t numel;     /* 1 .. 2^31 */
+    int32_t dtype;     /* QLN_DTYPE_F32, _BF16 or _F16 */
+    int32_t dq_format; /* QLN_DQ_INT8 or QLN_DQ_E4M3 */
+    uint8_t *codes;    /* [ceil(numel/2)] out, 16-byte aligned */
+    float *absmax;     /* [nb] out, nb = ceil(numel/64), 16-byte aligned */
+    void *qabs;        /* [nb] out (int8 or E4M3 codes) */
+    float *dq_scale;   /* [ceil(nb/256)] out */
+    float *dq_mean;    /* [1] out */
+} qln_quant_job;
+
+/*
+ * nf4_quantize_dq_batch -- nf4_quantize_dq of njobs weights in one call, the
+ * same bits as calling it for each job in order.  This is how a whole model is
+ * quantized for QLoRA ("LoRA 与 QLoRA" section QLoRA: every frozen weight
+ * stored as NF4 with double-quantized constants).
+ * The double quantization of weight i, whose latency is mostly waiting (an
+ * exact sum over all constants, then the groups), is not run after weight i:
+ * the sum of weight i's constants runs at the start of weight i+1's quantize
+ * launch and the group quantization at the start of weight i+2's, while those
+ * launches' first weight chunks are in flight; two small launches finish the
+ * last two weights.  Launches still run one after the other in stream order,
+ * each reading only what earlier launches completed, so the jobs' buffers may
+ * be laid out in any way that separate nf4_quantize_dq calls allow.
+ *   ws / ws_bytes: qln_workspace_bytes(QLN_OP_QUANTIZE_DQ_BATCH, njobs, 0, 0,
+ *   0) = 256 * njobs bytes, 256-byte aligned, zeroed once before the first
+ *   call and then left to the library (job i uses bytes 256 i .. 256 i + 255
+ *   as its double-quantization scratch); byte 0 holds QLN_OK afterwards (no
+ *   launch of this call waits on anything).
+ * Errors: QLN_ERR_NULL (jobs, ws, or a job pointer); QLN_ERR_SHAPE (njobs < 1
+ * or above 2^20, or a job's sizes, dtype or format); QLN_ERR_ALIGN;
+ * QLN_ERR_WORKSPACE; QLN_ERR_ARCH.  Every job is checked before anything is
+ * launched.
+ */
+QLN_API qln_status nf4_quantize_dq_batch(const qln_quant_job *jobs, int32_t njobs, void *ws, size_t ws_bytes,
+                                         void *stream);
 
 /*
  * nf4_double_quant_noalloc -- nf4_double_quant without a caller workspace.
@@ -367,7 +406,8 @@ QLN_API qln_status qln_adamw_step(float *param, const float *grad, float *m, flo
                                   void *stream);
 
 /* Device workspace, in bytes, that `op` needs for these sizes (nb for
- * QLN_OP_DOUBLE_QUANT is passed as `rows`).  Returns 0 for an unknown op. */
+ * QLN_OP_DOUBLE_QUANT and the job count for QLN_OP_QUANTIZE_DQ_BATCH are
+ * passed as `rows`).  Returns 0 for an unknown op. */
 QLN_API size_t qln_workspace_bytes(int32_t op, int64_t rows, int64_t cols, int64_t n, int32_t r);
 
 /* The 16 NF4 values (fp32, ascending) the kernels snap to and decode with. */

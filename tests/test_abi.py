@@ -120,6 +120,29 @@ def test_quantize_dq_argument_errors(L):
     assert q(wsb=255) == 4
 
 
+def test_quantize_dq_batch_argument_errors(L):
+    ws = P(0x20000)
+    good = dict(W=0x10000, numel=4096, dtype=0, dq_format=0, codes=0x10000, absmax=0x10000, qabs=0x10000,
+                dq_scale=0x10000, dq_mean=0x10000)
+
+    def call(n=2, wsb=512, ws_=ws, **bad):
+        arr = (api.CQuantJob * 2)(api.CQuantJob(**good), api.CQuantJob(**dict(good, **bad)))
+        return L.nf4_quantize_dq_batch(arr, n, ws_, wsb, None)
+    assert L.nf4_quantize_dq_batch(None, 1, ws, 256, None) == 1
+    assert call(ws_=None) == 1
+    assert call(W=None) == 1                  # the second job is checked too
+    assert call(n=0) == 2
+    assert call(n=(1 << 20) + 1, wsb=1 << 40) == 2
+    assert call(numel=0) == 2
+    assert call(dtype=9) == 2
+    assert call(dq_format=5) == 2
+    assert call(absmax=0x10004) == 3
+    assert call(ws_=P(0x20010)) == 3
+    assert call(wsb=511) == 4
+    assert api.workspace_bytes(api.OP_QUANTIZE_DQ_BATCH, 224) == 224 * 256
+    assert api.workspace_bytes(api.OP_QUANTIZE_DQ_BATCH, 0) == 0
+
+
 def test_dequant_argument_errors(L):
     out = A16
     assert L.nf4_dequant(None, out, None) == 1

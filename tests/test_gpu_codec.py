@@ -447,3 +447,68 @@ def test_dq_restore_order_worked_by_hand(n):
     torch.cuda.synchronize()
     assert np.all(dev_bf16_bits(deq) == 0x3500)
     assert np.all(dev_bf16_bits(Y) == 0x3500)
+
+
+BATCH_SHAPES = [(64 * 1000 + 37, torch.float32, "int8"), (4096 * 1024, torch.bfloat16, "int8"),
+                (333_333, torch.float16, "e4m3"), (64, torch.float32, "int8"), (11008 * 256, torch.float32, "int8")]
+
+
+@pytest.mark.parametrize("njobs", [1, 2, 3, 5])
+def test_quantize_dq_batch_matches_oracle_per_job(njobs):
+    """nf4_quantize_dq_batch: every job's codes, constants, DQ codes, scales and
+    mu equal the oracle's quantize + double_quant of that job (the sum of job i
+    runs inside job i+1's launch and its groups inside job i+2's, the last two
+    in the tail launches).  A second call on the same workspace gives the same
+    bits, and the scratch of every job is ready for the next call."""
+    shapes = [BATCH_SHAPES[k % len(BATCH_SHAPES)] for k in range(njobs)]
+    jobs, host = [], []
+    for k, (numel, dtype, fmt) in enumerate(shapes):
+        w = synthetic.normal_f32(numel, 0.02 * (k + 1), 120 + k)
+        Wc = torch.from_numpy(w).to(dtype)
+        host.append((Wc.float().numpy(), fmt))
+        nb = (numel + 63) // 64
+        jobs.append((Wc.cuda(), torch.empty((numel + 1) // 2, dtype=torch.uint8, device="cuda"),
+                     torch.empty(nb, device="cuda"),
+                     torch.empty(nb, dtype=torch.int8 if fmt == "int8" else torch.uint8, device="cuda"),
+                     torch.empty((nb + 255) // 256, device="cuda"), torch.empty(1, device="cuda"), fmt))
+    ws = api.alloc_workspace(api.workspace_bytes(api.OP_QUANTIZE_DQ_BATCH, njobs))
+    api.nf4_quantize_dq_batch(jobs, ws=ws)
+    torch.cuda.synchronize()
+    first = [[t.clone() for t in j[1:6]] for j in jobs]
+    api.nf4_quantize_dq_batch(jobs, ws=ws)
+    torch.cuda.synchronize()
+    assert api.device_status(ws) == 0
+    for k, ((w_exact, fmt), j) in enumerate(zip(host, jobs)):
+        for a, b in zip(first[k], j[1:6]):
+            assert torch.equal(a, b), f"job {k}: second call differs"
+        assert _scratch_at_rest(ws[256 * k:256 * (k + 1)])
+        codes, absmax, q, b, mu = [t.cpu().numpy() for t in j[1:6]]
+        c_ref, a_ref = codec.quantize(w_exact)
+        q_ref, b_ref, mu_ref = codec.double_quant(a_ref, fmt=fmt)
+        assert np.array_equal(codes, c_ref), f"job {k}: codes"
+        assert np.array_equal(absmax.view(np.uint32), a_ref.view(np.uint32)), f"job {k}: absmax"
+        assert np.float32(mu[0]).view(np.uint32) == np.float32(mu_ref).view(np.uint32), f"job {k}: mu"
+        assert np.array_equal(b.view(np.uint32), b_ref.view(np.uint32)), f"job {k}: dq scale"
+        assert np.array_equal(q.view(np.uint8), q_ref.view(np.uint8)), f"job {k}: dq codes"
+
+
+def test_quantize_dq_batch_with_shared_outputs_runs_in_order():
+    """Jobs whose outputs overlap (the second weight written into the first
+    one's buffers) take the ordered schedule: the result is that of the second
+    job, as with separate nf4_quantize_dq calls in order."""
+    numel = 4096 * 256
+    nb = numel // 64
+    wa = synthetic.normal_f32(numel, 0.02, 131)
+    wb = synthetic.normal_f32(numel, 0.05, 132)
+    outs = (torch.empty(numel // 2, dtype=torch.uint8, device="cuda"), torch.empty(nb, device="cuda"),
+            torch.empty(nb, dtype=torch.int8, device="cuda"), torch.empty(nb // 256, device="cuda"),
+            torch.empty(1, device="cuda"))
+    jobs = [(torch.from_numpy(wa).cuda(), *outs, "int8"), (torch.from_numpy(wb).cuda(), *outs, "int8")]
+    api.nf4_quantize_dq_batch(jobs)
+    torch.cuda.synchronize()
+    codes, absmax, q, b, mu = [t.cpu().numpy() for t in outs]
+    c_ref, a_ref = codec.quantize(wb)
+    q_ref, b_ref, mu_ref = codec.double_quant(a_ref)
+    assert np.array_equal(codes, c_ref) and np.array_equal(absmax.view(np.uint32), a_ref.view(np.uint32))
+    assert np.float32(mu[0]).view(np.uint32) == np.float32(mu_ref).view(np.uint32)
+    assert np.array_equal(b.view(np.uint32), b_ref.view(np.uint32)) and np.array_equal(q, q_ref)
