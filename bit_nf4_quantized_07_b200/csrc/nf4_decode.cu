@@ -230,14 +230,14 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
         }
     };
 
-    // ---- 1. requests: the code boxes first (the longest latency), then the block
-    //         constants, X and the B rows --------------------------------------------------
+    // ---- 1. requests: the code boxes first (the longest latency), then X and the
+    //         B rows (asynchronous copies), then the block constants, whose loads
+    //         this thread waits for -- so all of them are in flight together -------------
     pdl_wait();  // the weight, X, A, B and the workspace may be written by the previous kernel
     pdl_trigger();
     if (blockIdx.x == 0 && tid == 0) *p.status = QLN_OK;
 #pragma unroll 1
     for (int k = 0; k < RS; ++k) issue_next();
-    stage_ah(0);
     // X chunk: line (token t, block bl) at row t * nkbx + bl, second half; 16-B chunks swizzled by t & 1
 #pragma unroll 1
     for (int t = warp; t < 8 * NT; t += kDfWarps)
@@ -251,6 +251,7 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
         }
     stage_b(0);
     cp_async_commit();
+    stage_ah(0);
     cp_async_wait<0>();
     __syncthreads();  // table, X, block constants and the B rows of epoch 0 in place
 
