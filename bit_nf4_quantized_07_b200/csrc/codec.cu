@@ -577,47 +577,78 @@ struct DqPhases {
 };
 
 // Both phases with the whole grid (any block size that is a multiple of 32);
-// every thread of every CTA calls it.  slim: kXLimbs words of shared memory.
+// every thread of every CTA calls it.  CTA b takes a contiguous share of the
+// constants (sum) and of the groups, staged through `stage` (kPhStage floats
+// of shared memory) by cp.async, so a CTA of few threads still has its whole
+// share in flight at once.  slim: kXLimbs words of shared memory.
+constexpr int kPhStage = 4096;  // floats per staging round (16 KB)
 __device__ __noinline__ void dq_run_phases(const DqPhases &ph, unsigned long long *slim, float *mu_s,
-                                           unsigned *gen_s) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    if (ph.status && blockIdx.x == 0 && threadIdx.x == 0) *ph.status = QLN_OK;
+                                           unsigned *gen_s, float *stage) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5, nt = blockDim.x;
+    if (ph.status && blockIdx.x == 0 && tid == 0) *ph.status = QLN_OK;
+    // copy constants [j0, j1) of `a` (j1 - j0 <= kPhStage, j0 a multiple of 4) into stage,
+    // zero-filled past nb; every thread waits for its copies, then the CTA meets
+    auto stage_in = [&](const float *a, int64_t j0, int64_t j1, int64_t nb) {
+        for (int64_t c = tid; 4 * c < j1 - j0; c += nt) {
+            const int64_t j = j0 + 4 * c;
+            const int64_t left = nb - j;
+            cp_async16_zfill(stage + 4 * c, a + (left > 0 ? j : 0), left >= 4 ? 16 : (left > 0 ? (int)left * 4 : 0));
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+    };
     const DqScratch gs = dq_scratch(ph.g_ws, false);
-    if (ph.g_absmax && warp == 0) {  // mu of job i-2: its sum advanced the generation
+    if (ph.g_absmax && warp == 0) {  // mu of the earlier weight: its sum advanced the generation
         const float mu = xsum_mean_warp(gs.bank[(__ldcg(gs.gen) + 1) & 1], (uint32_t)ph.g_nb);
         if (lane == 0) {
             *mu_s = mu;
             if (blockIdx.x == 0) *ph.g_mu = mu;
         }
     }
-    if (ph.s_absmax) {  // the exact sum of job i-1, 8 consecutive constants per thread and pass
+    if (ph.s_absmax) {  // the exact sum of the later weight's constants
         const DqScratch ss = dq_scratch(ph.s_ws, false);
-        if (threadIdx.x < kXLimbs) slim[threadIdx.x] = 0ull;
+        if (tid < kXLimbs) slim[tid] = 0ull;
         const unsigned g0 = dq_read_gen(ss, gen_s);  // includes a __syncthreads
+        const int64_t nb = ph.s_nb;
+        const int64_t per = ((nb + gridDim.x - 1) / gridDim.x + 3) & ~(int64_t)3;
+        const int64_t lo = (int64_t)blockIdx.x * per < nb ? (int64_t)blockIdx.x * per : nb;
+        const int64_t hi = lo + per < nb ? lo + per : nb;
         XRun x;
-        const int64_t step = (int64_t)gridDim.x * blockDim.x * 8;
-        for (int64_t j = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; j < ph.s_nb; j += step) {
-            float v[8];
-            load8_const(v, ph.s_absmax, j, ph.s_nb);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) xsum_add(x, v[u], slim);
+        for (int64_t r0 = lo; r0 < hi; r0 += kPhStage) {
+            const int64_t r1 = r0 + kPhStage < hi ? r0 + kPhStage : hi;
+            stage_in(ph.s_absmax, r0, r1, nb);
+            for (int64_t k = tid; k < r1 - r0; k += nt) xsum_add(x, stage[k], slim);
+            __syncthreads();  // the stage is read before the next round refills it
         }
         xsum_flush_warp(x, slim);
         __syncthreads();
-        if (threadIdx.x < kXLimbs && slim[threadIdx.x] != 0ull)
-            atomicAdd(&ss.bank[g0 & 1][threadIdx.x], slim[threadIdx.x]);
+        if (tid < kXLimbs && slim[tid] != 0ull) atomicAdd(&ss.bank[g0 & 1][tid], slim[tid]);
         __syncthreads();
-        if (threadIdx.x == 0) dq_arrive(ss, g0, (int)gridDim.x);
+        if (tid == 0) dq_arrive(ss, g0, (int)gridDim.x);
     }
     __syncthreads();  // mu is in shared memory
     if (ph.g_absmax) {
         const float mu = *mu_s;
-        const int64_t ng = (ph.g_nb + kDqGroup - 1) / kDqGroup;
-        for (int64_t g = (int64_t)blockIdx.x * nw + warp; g < ng; g += (int64_t)gridDim.x * nw) {
-            float e[8];
-            load8_const(e, ph.g_absmax, g * kDqGroup + 8 * lane, ph.g_nb);
-            dq_quantize_group(e, g * kDqGroup + 8 * lane, ph.g_nb, mu, ph.g_e4m3 != 0, lane, g, ph.g_qabs,
-                              ph.g_scale);
+        const int64_t nb = ph.g_nb;
+        const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
+        const int64_t per = (ng + gridDim.x - 1) / gridDim.x;
+        const int64_t glo = (int64_t)blockIdx.x * per < ng ? (int64_t)blockIdx.x * per : ng;
+        const int64_t ghi = glo + per < ng ? glo + per : ng;
+        constexpr int kGroupsPerRound = kPhStage / kDqGroup;
+        for (int64_t g0 = glo; g0 < ghi; g0 += kGroupsPerRound) {
+            const int64_t g1 = g0 + kGroupsPerRound < ghi ? g0 + kGroupsPerRound : ghi;
+            const int64_t j1 = g1 * kDqGroup < nb ? g1 * kDqGroup : nb;
+            stage_in(ph.g_absmax, g0 * kDqGroup, j1, nb);
+            for (int64_t g = g0 + warp; g < g1; g += nw) {
+                const float *src = stage + (g - g0) * kDqGroup + 8 * lane;
+                const float4 u = *reinterpret_cast<const float4 *>(src);
+                const float4 v = *reinterpret_cast<const float4 *>(src + 4);
+                const float e[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};  // entries past nb are not used
+                dq_quantize_group(e, g * kDqGroup + 8 * lane, nb, mu, ph.g_e4m3 != 0, lane, g, ph.g_qabs,
+                                  ph.g_scale);
+            }
+            __syncthreads();  // the stage is read before the next round refills it
         }
     }
 }
@@ -1063,13 +1094,29 @@ static_assert(kDqScratchBytes == kDqBatchScratchBytes, "one DQ scratch per batch
 constexpr int kPhThreads = 128;
 template <bool kEarlyRelease>
 __global__ void __launch_bounds__(kPhThreads, 16) dq_phase_kernel(DqPhases ph) {
+    extern __shared__ __align__(16) float ph_stage[];  // kPhStage floats
     __shared__ unsigned long long slim[kXLimbs];
     __shared__ float mu_s;
     __shared__ unsigned gen_s;
     if (kEarlyRelease) pdl_trigger();
     pdl_wait();
     if (!kEarlyRelease) pdl_trigger();
-    dq_run_phases(ph, slim, &mu_s, &gen_s);
+    dq_run_phases(ph, slim, &mu_s, &gen_s, ph_stage);
+}
+constexpr size_t kPhSmem = kPhStage * sizeof(float);
+
+// One phase launch (the kernel asks for the largest shared-memory carveout so
+// that it can sit beside two quantize CTAs on an SM).
+template <bool kEarlyRelease>
+static cudaError_t launch_phase(int grid, const DqPhases &ph, cudaStream_t st) {
+    static std::atomic<int> configured{0};
+    if (!configured.load(std::memory_order_relaxed)) {
+        cudaError_t e = cudaFuncSetAttribute(dq_phase_kernel<kEarlyRelease>,
+                                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess) return e;
+        configured.store(1, std::memory_order_relaxed);
+    }
+    return launch_pdl(dq_phase_kernel<kEarlyRelease>, dim3(grid), dim3(kPhThreads), kPhSmem, st, ph);
 }
 
 namespace {
@@ -1160,20 +1207,20 @@ cudaError_t launch_nf4_quantize_dq_batch(const QuantJob *jobs, int njobs, void *
     for (int i = 1; i < njobs; ++i) {
         const QuantJob &q = jobs[i];
         if (overlap) {
-            e = launch_pdl(dq_phase_kernel<true>, dim3(num_sms), dim3(kPhThreads), 0, st, phases(i - 1, i - 2));
+            e = launch_phase<true>(num_sms, phases(i - 1, i - 2), st);
             if (e == cudaSuccess)
                 e = launch_quantize_dtype<true>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
         } else {
-            e = launch_pdl(dq_phase_kernel<false>, dim3(num_sms), dim3(kPhThreads), 0, st, phases(i - 1, i - 2));
+            e = launch_phase<false>(num_sms, phases(i - 1, i - 2), st);
             if (e == cudaSuccess)
                 e = launch_quantize_dtype<false>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
         }
         if (e != cudaSuccess) return e;
     }
     const int tail_grid = 4 * num_sms;
-    e = launch_pdl(dq_phase_kernel<false>, dim3(tail_grid), dim3(kPhThreads), 0, st, phases(njobs - 1, njobs - 2));
+    e = launch_phase<false>(tail_grid, phases(njobs - 1, njobs - 2), st);
     if (e != cudaSuccess) return e;
-    return launch_pdl(dq_phase_kernel<false>, dim3(tail_grid), dim3(kPhThreads), 0, st, phases(-1, njobs - 1));
+    return launch_phase<false>(tail_grid, phases(-1, njobs - 1), st);
 }
 
 // ===========================================================================
