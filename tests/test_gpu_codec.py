@@ -512,3 +512,38 @@ def test_quantize_dq_batch_with_shared_outputs_runs_in_order():
     assert np.array_equal(codes, c_ref) and np.array_equal(absmax.view(np.uint32), a_ref.view(np.uint32))
     assert np.float32(mu[0]).view(np.uint32) == np.float32(mu_ref).view(np.uint32)
     assert np.array_equal(b.view(np.uint32), b_ref.view(np.uint32)) and np.array_equal(q, q_ref)
+
+
+def test_quantize_dq_batch_long_chain_and_shared_input():
+    """A batch of 24 small weights of assorted sizes (a long chain of deferred
+    double quantizations, every phase launch beside a quantize), two of them
+    quantizing the same input tensor (read-only overlap keeps the early-start
+    schedule): every job equals the oracle."""
+    rng = np.random.default_rng(140)
+    jobs, host = [], []
+    shared = None
+    for k in range(24):
+        numel = int(rng.integers(1, 40)) * 4096 + int(rng.integers(0, 64))
+        if k == 7:
+            Wd, w = shared
+        else:
+            w = synthetic.normal_f32(numel, float(rng.uniform(0.005, 0.05)), 150 + k)
+            Wd = torch.from_numpy(w).cuda()
+            if k == 3:
+                shared = (Wd, w)
+        numel = w.size
+        nb = (numel + 63) // 64
+        host.append(w)
+        jobs.append((Wd, torch.empty((numel + 1) // 2, dtype=torch.uint8, device="cuda"),
+                     torch.empty(nb, device="cuda"), torch.empty(nb, dtype=torch.int8, device="cuda"),
+                     torch.empty((nb + 255) // 256, device="cuda"), torch.empty(1, device="cuda"), "int8"))
+    api.nf4_quantize_dq_batch(jobs)
+    torch.cuda.synchronize()
+    for k, (w, j) in enumerate(zip(host, jobs)):
+        codes, absmax, q, b, mu = [t.cpu().numpy() for t in j[1:6]]
+        c_ref, a_ref = codec.quantize(w)
+        q_ref, b_ref, mu_ref = codec.double_quant(a_ref)
+        assert np.array_equal(codes, c_ref), f"job {k}: codes"
+        assert np.float32(mu[0]).view(np.uint32) == np.float32(mu_ref).view(np.uint32), f"job {k}: mu"
+        assert np.array_equal(b.view(np.uint32), b_ref.view(np.uint32)), f"job {k}: dq scale"
+        assert np.array_equal(q, q_ref), f"job {k}: dq codes"
