@@ -830,21 +830,18 @@ constexpr int kDqGroupsPerCta = kDqThreads / 32;  // one group of 256 constants 
 // generation.  Nothing waits: K3 reads the bank only after this grid has
 // completed.
 // ===========================================================================
-__global__ void __launch_bounds__(kDqThreads) dq_sum_kernel(const float *__restrict__ a, int64_t nb,
-                                                            unsigned char *ws, bool with_status) {
-    __shared__ unsigned long long slim[kXLimbs];
-    __shared__ unsigned gen_s;
-    if (threadIdx.x < kXLimbs) slim[threadIdx.x] = 0ull;
-    __syncthreads();
-    pdl_wait();  // the constants come from the previous kernel (the quantize)
-    pdl_trigger();
+// CTA `bid` of the `nblk` that sum one weight's constants (slim zeroed and
+// visible to the CTA on entry).
+__device__ __forceinline__ void dq_sum_part(const float *__restrict__ a, int64_t nb, unsigned char *ws,
+                                            bool with_status, int64_t bid, int64_t nblk, unsigned long long *slim,
+                                            unsigned *gen_s) {
     const DqScratch sc = dq_scratch(ws, with_status);
-    if (blockIdx.x == 0 && threadIdx.x == 0 && sc.status) *sc.status = QLN_OK;
-    const unsigned g0 = dq_read_gen(sc, &gen_s);
+    if (bid == 0 && threadIdx.x == 0 && sc.status) *sc.status = QLN_OK;
+    const unsigned g0 = dq_read_gen(sc, gen_s);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
     XRun x;
-    for (int64_t g = (int64_t)blockIdx.x * kDqGroupsPerCta + warp; g < ng; g += (int64_t)gridDim.x * kDqGroupsPerCta) {
+    for (int64_t g = bid * kDqGroupsPerCta + warp; g < ng; g += nblk * kDqGroupsPerCta) {
         float e[8];
         load8_const(e, a, g * kDqGroup + 8 * lane, nb);
 #pragma unroll
@@ -854,7 +851,18 @@ __global__ void __launch_bounds__(kDqThreads) dq_sum_kernel(const float *__restr
     __syncthreads();
     if (threadIdx.x < kXLimbs && slim[threadIdx.x] != 0ull) atomicAdd(&sc.bank[g0 & 1][threadIdx.x], slim[threadIdx.x]);
     __syncthreads();
-    if (threadIdx.x == 0) dq_arrive(sc, g0, (int)gridDim.x);
+    if (threadIdx.x == 0) dq_arrive(sc, g0, (int)nblk);
+}
+
+__global__ void __launch_bounds__(kDqThreads) dq_sum_kernel(const float *__restrict__ a, int64_t nb,
+                                                            unsigned char *ws, bool with_status) {
+    __shared__ unsigned long long slim[kXLimbs];
+    __shared__ unsigned gen_s;
+    if (threadIdx.x < kXLimbs) slim[threadIdx.x] = 0ull;
+    __syncthreads();
+    pdl_wait();  // the constants come from the previous kernel (the quantize)
+    pdl_trigger();
+    dq_sum_part(a, nb, ws, with_status, blockIdx.x, gridDim.x, slim, &gen_s);
 }
 
 // ===========================================================================
@@ -864,18 +872,16 @@ __global__ void __launch_bounds__(kDqThreads) dq_sum_kernel(const float *__restr
 // bank is zeroed by the next call's K2 (or single launch), not here.  A warp takes groups warp, warp + 8 gridDim, ... with the next group's
 // constants requested before the current one is quantized.
 // ===========================================================================
-__global__ void __launch_bounds__(kDqThreads) dq_quant_kernel(const float *__restrict__ a, int64_t nb,
-                                                              int8_t *__restrict__ qabs, float *__restrict__ scale,
-                                                              const float *__restrict__ mu_in,
-                                                              float *__restrict__ mu_out, unsigned char *scratch,
-                                                              bool e4m3) {
-    __shared__ float mu_s;
+// CTA `bid` of the `nblk` that quantize one weight's groups.
+__device__ __forceinline__ void dq_quant_part(const float *__restrict__ a, int64_t nb, int8_t *__restrict__ qabs,
+                                              float *__restrict__ scale, const float *__restrict__ mu_in,
+                                              float *__restrict__ mu_out, unsigned char *scratch, bool e4m3,
+                                              int64_t bid, int64_t nblk, float *mu_sh) {
+    float &mu_s = *mu_sh;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
-    const int64_t gstep = (int64_t)gridDim.x * kDqGroupsPerCta;
-    int64_t g = (int64_t)blockIdx.x * kDqGroupsPerCta + warp;
-    pdl_wait();
-    pdl_trigger();
+    const int64_t gstep = nblk * kDqGroupsPerCta;
+    int64_t g = bid * kDqGroupsPerCta + warp;
     float e[8];
     load8_const(e, a, g < ng ? g * kDqGroup + 8 * lane : nb, nb);
     const DqScratch sc = dq_scratch(scratch, false);
@@ -884,7 +890,7 @@ __global__ void __launch_bounds__(kDqThreads) dq_quant_kernel(const float *__res
             const float mu = xsum_mean_warp(sc.bank[(__ldcg(sc.gen) + 1) & 1], (uint32_t)nb);
             if (lane == 0) {
                 mu_s = mu;
-                if (blockIdx.x == 0) *mu_out = mu;
+                if (bid == 0) *mu_out = mu;
             }
         } else if (lane == 0) {
             mu_s = __ldcg(mu_in);
@@ -899,6 +905,17 @@ __global__ void __launch_bounds__(kDqThreads) dq_quant_kernel(const float *__res
 #pragma unroll
         for (int u = 0; u < 8; ++u) e[u] = nx[u];
     }
+}
+
+__global__ void __launch_bounds__(kDqThreads) dq_quant_kernel(const float *__restrict__ a, int64_t nb,
+                                                              int8_t *__restrict__ qabs, float *__restrict__ scale,
+                                                              const float *__restrict__ mu_in,
+                                                              float *__restrict__ mu_out, unsigned char *scratch,
+                                                              bool e4m3) {
+    __shared__ float mu_s;
+    pdl_wait();
+    pdl_trigger();
+    dq_quant_part(a, nb, qabs, scale, mu_in, mu_out, scratch, e4m3, blockIdx.x, gridDim.x, &mu_s);
 }
 
 // K3's grid: one group per warp up to the CTAs the device holds at once (a
@@ -1085,38 +1102,34 @@ cudaError_t launch_nf4_quantize_dq(const void *W, int dtype, int64_t numel, uint
 
 static_assert(kDqScratchBytes == kDqBatchScratchBytes, "one DQ scratch per batch job");
 
-// The deferred double quantization of a batch, one small CTA per SM: 128
-// threads of at most 32 registers fit beside the two quantize CTAs of an SM
-// (the registers those leave free), so it runs alongside the quantize
-// kernels.  It always waits for its predecessor before touching memory;
-// kEarlyRelease lets the next weight's quantize start before that wait (only
-// for a batch whose buffers are disjoint, see kLateWait).
+// The deferred double quantization of a batch whose buffers overlap, one
+// small CTA per SM: 128 threads of at most 32 registers fit beside the two
+// quantize CTAs of an SM (the registers those leave free), so it runs
+// alongside the quantize kernels.  It waits for its predecessor before
+// touching memory.
 constexpr int kPhThreads = 128;
-template <bool kEarlyRelease>
 __global__ void __launch_bounds__(kPhThreads, 16) dq_phase_kernel(DqPhases ph) {
     extern __shared__ __align__(16) float ph_stage[];  // kPhStage floats
     __shared__ unsigned long long slim[kXLimbs];
     __shared__ float mu_s;
     __shared__ unsigned gen_s;
-    if (kEarlyRelease) pdl_trigger();
     pdl_wait();
-    if (!kEarlyRelease) pdl_trigger();
+    pdl_trigger();
     dq_run_phases(ph, slim, &mu_s, &gen_s, ph_stage);
 }
 constexpr size_t kPhSmem = kPhStage * sizeof(float);
 
 // One phase launch (the kernel asks for the largest shared-memory carveout so
 // that it can sit beside two quantize CTAs on an SM).
-template <bool kEarlyRelease>
 static cudaError_t launch_phase(int grid, const DqPhases &ph, cudaStream_t st) {
     static std::atomic<int> configured{0};
     if (!configured.load(std::memory_order_relaxed)) {
-        cudaError_t e = cudaFuncSetAttribute(dq_phase_kernel<kEarlyRelease>,
+        cudaError_t e = cudaFuncSetAttribute(dq_phase_kernel,
                                              cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) return e;
         configured.store(1, std::memory_order_relaxed);
     }
-    return launch_pdl(dq_phase_kernel<kEarlyRelease>, dim3(grid), dim3(kPhThreads), kPhSmem, st, ph);
+    return launch_pdl(dq_phase_kernel, dim3(grid), dim3(kPhThreads), kPhSmem, st, ph);
 }
 
 namespace {
@@ -1164,15 +1177,111 @@ bool batch_disjoint(const QuantJob *jobs, int njobs, const void *ws) {
 }
 }  // namespace
 
-// Batch: quantize(0); then for i >= 1 the phase launch (sum of weight i-1,
-// groups of weight i-2) followed by quantize(i); then the two tail phase
-// launches (sum of n-1 and groups of n-2; groups of n-1).  Every phase launch
-// waits for the quantize before it, whose completion implies that of all
-// earlier launches (a late-waiting quantize waits at its end), so each phase
-// reads only completed constants and sums.  With disjoint buffers the
-// quantize kernels start early (see kLateWait); otherwise every launch waits
-// at its start as usual.  Job i's scratch is ws + 256 i; the first phase
-// launch clears the status word at ws + 0.
+// The double quantization of a disjoint batch after its last quantize: one
+// launch sums the constants of up to kTailJobs weights, a second quantizes
+// their groups.  A job's CTAs are a contiguous range of the launch (job j owns
+// CTAs cta0[j] .. cta0[j+1]-1) and run the single-weight code with that range
+// as their grid, so the exact sums and groups are those of separate calls.
+// The job table travels as the kernel's parameter (about 7 KB).
+constexpr int kTailJobs = 128;
+constexpr int kTailPasses = 4;  // groups per warp and CTA, at most
+struct DqTailJob {
+    const float *absmax;
+    int64_t nb;
+    unsigned char *ws;
+    int8_t *qabs;
+    float *scale;
+    float *mu;
+    int e4m3;
+    int cta0;  // first CTA of the job
+};
+struct DqTail {
+    int njobs;
+    int status;  // job 0's CTA 0 writes QLN_OK to its scratch status word
+    DqTailJob job[kTailJobs];
+};
+
+// The job whose CTA range holds CTA b, and the CTA's place in that range.
+__device__ __forceinline__ int dq_tail_job(const DqTail &t, int b, int64_t *bid, int64_t *nblk) {
+    int lo = 0, hi = t.njobs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (t.job[mid].cta0 <= b) lo = mid;
+        else hi = mid - 1;
+    }
+    *bid = b - t.job[lo].cta0;
+    *nblk = (lo + 1 < t.njobs ? t.job[lo + 1].cta0 : (int)gridDim.x) - t.job[lo].cta0;
+    return lo;
+}
+
+__global__ void __launch_bounds__(kDqThreads) dq_sum_tail_kernel(const __grid_constant__ DqTail t) {
+    __shared__ unsigned long long slim[kXLimbs];
+    __shared__ unsigned gen_s;
+    if (threadIdx.x < kXLimbs) slim[threadIdx.x] = 0ull;
+    __syncthreads();
+    pdl_wait();  // the constants come from earlier kernels
+    pdl_trigger();
+    int64_t bid, nblk;
+    const int j = dq_tail_job(t, blockIdx.x, &bid, &nblk);
+    const DqTailJob &J = t.job[j];
+    dq_sum_part(J.absmax, J.nb, J.ws, t.status && j == 0, bid, nblk, slim, &gen_s);
+}
+
+__global__ void __launch_bounds__(kDqThreads) dq_quant_tail_kernel(const __grid_constant__ DqTail t) {
+    __shared__ float mu_s;
+    pdl_wait();  // the sums of the earlier launch
+    pdl_trigger();
+    int64_t bid, nblk;
+    const int j = dq_tail_job(t, blockIdx.x, &bid, &nblk);
+    const DqTailJob &J = t.job[j];
+    dq_quant_part(J.absmax, J.nb, J.qabs, J.scale, nullptr, J.mu, J.ws, J.e4m3 != 0, bid, nblk, &mu_s);
+}
+
+// Sum launches for every kTailJobs jobs, then the group launches.
+static cudaError_t launch_dq_tails(const QuantJob *jobs, int njobs, unsigned char *ws, cudaStream_t st) {
+    static_assert(sizeof(DqTail) <= 8192, "the job table stays a small kernel parameter");
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int j0 = 0; j0 < njobs; j0 += kTailJobs) {
+            DqTail t{};
+            t.njobs = njobs - j0 < kTailJobs ? njobs - j0 : kTailJobs;
+            t.status = (j0 == 0) ? 1 : 0;
+            int64_t ctas = 0;
+            for (int k = 0; k < t.njobs; ++k) {
+                const QuantJob &q = jobs[j0 + k];
+                DqTailJob &J = t.job[k];
+                J.absmax = q.absmax;
+                J.nb = (q.numel + 63) / 64;
+                J.ws = ws + kDqScratchBytes * (size_t)(j0 + k);
+                J.qabs = q.qabs;
+                J.scale = q.scale;
+                J.mu = q.mu;
+                J.e4m3 = q.e4m3 ? 1 : 0;
+                J.cta0 = (int)ctas;
+                const int64_t ng = (J.nb + kDqGroup - 1) / kDqGroup;
+                ctas += (ng + kDqGroupsPerCta * kTailPasses - 1) / (kDqGroupsPerCta * kTailPasses);
+            }
+            const cudaError_t e = pass == 0
+                                      ? launch_pdl(dq_sum_tail_kernel, dim3((unsigned)ctas), dim3(kDqThreads), 0, st, t)
+                                      : launch_pdl(dq_quant_tail_kernel, dim3((unsigned)ctas), dim3(kDqThreads), 0, st, t);
+            if (e != cudaSuccess) return e;
+        }
+    }
+    return cudaSuccess;
+}
+
+// Batch with disjoint buffers: the quantize kernels back to back (from the
+// second on they start early, see kLateWait), then the tail launches of
+// launch_dq_tails.  The first tail launch waits for the last quantize, whose
+// completion implies that of every earlier one.  Phase kernels running beside
+// the quantize kernels instead took the 6.48 B-parameter sweep from 5.35 ms
+// to 6.6 ms: their work, on one small CTA per SM, ran longer than the
+// quantize of the smaller weights it had to finish within.
+// Otherwise: quantize(0); then for i >= 1 the phase launch (sum of weight
+// i-1, groups of weight i-2) followed by quantize(i); then the two tail phase
+// launches (sum of n-1 and groups of n-2; groups of n-1).  Every launch waits
+// at its start for the one before it, so each phase reads only completed
+// constants and sums.  Job i's scratch is ws + 256 i; the first sum launch
+// clears the status word at ws + 0.
 cudaError_t launch_nf4_quantize_dq_batch(const QuantJob *jobs, int njobs, void *ws, cudaStream_t st, int num_sms) {
     unsigned char *w = static_cast<unsigned char *>(ws);
     auto scratch = [&](int i) { return w + kDqScratchBytes * (size_t)i; };
@@ -1200,27 +1309,28 @@ cudaError_t launch_nf4_quantize_dq_batch(const QuantJob *jobs, int njobs, void *
         }
         return ph;
     };
-    const bool overlap = batch_disjoint(jobs, njobs, ws);
+    const bool disjoint = batch_disjoint(jobs, njobs, ws);
     cudaError_t e = launch_quantize_dtype<false>(jobs[0].W, jobs[0].dtype, jobs[0].numel, jobs[0].codes,
                                                  jobs[0].absmax, st, num_sms);
     if (e != cudaSuccess) return e;
+    if (disjoint) {  // the quantize chain alone, then the double quantization of all jobs
+        for (int i = 1; i < njobs; ++i) {
+            const QuantJob &q = jobs[i];
+            e = launch_quantize_dtype<true>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
+            if (e != cudaSuccess) return e;
+        }
+        return launch_dq_tails(jobs, njobs, w, st);
+    }
     for (int i = 1; i < njobs; ++i) {
         const QuantJob &q = jobs[i];
-        if (overlap) {
-            e = launch_phase<true>(num_sms, phases(i - 1, i - 2), st);
-            if (e == cudaSuccess)
-                e = launch_quantize_dtype<true>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
-        } else {
-            e = launch_phase<false>(num_sms, phases(i - 1, i - 2), st);
-            if (e == cudaSuccess)
-                e = launch_quantize_dtype<false>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
-        }
+        e = launch_phase(num_sms, phases(i - 1, i - 2), st);
+        if (e == cudaSuccess) e = launch_quantize_dtype<false>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
         if (e != cudaSuccess) return e;
     }
     const int tail_grid = 4 * num_sms;
-    e = launch_phase<false>(tail_grid, phases(njobs - 1, njobs - 2), st);
+    e = launch_phase(tail_grid, phases(njobs - 1, njobs - 2), st);
     if (e != cudaSuccess) return e;
-    return launch_phase<false>(tail_grid, phases(-1, njobs - 1), st);
+    return launch_phase(tail_grid, phases(-1, njobs - 1), st);
 }
 
 // ===========================================================================

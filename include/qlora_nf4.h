@@ -240,14 +240,15 @@ typedef struct {
  * same bits as calling it for each job in order.  This is how a whole model is
  * quantized for QLoRA ("LoRA 与 QLoRA" section QLoRA: every frozen weight
  * stored as NF4 with double-quantized constants).
- * The double quantization of weight i, whose latency is mostly waiting (an
- * exact sum over all constants, then the groups), is not run after weight i:
- * the sum of weight i's constants runs at the start of weight i+1's quantize
- * launch and the group quantization at the start of weight i+2's, while those
- * launches' first weight chunks are in flight; two small launches finish the
- * last two weights.  Launches still run one after the other in stream order,
- * each reading only what earlier launches completed, so the jobs' buffers may
- * be laid out in any way that separate nf4_quantize_dq calls allow.
+ * When no job's outputs overlap another job's buffers, the quantize launches
+ * run back to back (each one starts while the one before it drains) and the
+ * double quantization of all jobs follows in two launches per 128 jobs (the
+ * exact sums, then the groups), so that its latency is paid once per call
+ * rather than once per weight.  Otherwise the double quantization of weight i
+ * runs in small launches between the later quantize launches (its sum before
+ * weight i+1's, its groups before weight i+2's).  Either way every launch
+ * reads only what earlier launches completed, so the jobs' buffers may be
+ * laid out in any way that separate nf4_quantize_dq calls allow.
  *   ws / ws_bytes: qln_workspace_bytes(QLN_OP_QUANTIZE_DQ_BATCH, njobs, 0, 0,
  *   0) = 256 * njobs bytes, 256-byte aligned, zeroed once before the first
  *   call and then left to the library (job i uses bytes 256 i .. 256 i + 255

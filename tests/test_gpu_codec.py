@@ -456,10 +456,10 @@ BATCH_SHAPES = [(64 * 1000 + 37, torch.float32, "int8"), (4096 * 1024, torch.bfl
 @pytest.mark.parametrize("njobs", [1, 2, 3, 5])
 def test_quantize_dq_batch_matches_oracle_per_job(njobs):
     """nf4_quantize_dq_batch: every job's codes, constants, DQ codes, scales and
-    mu equal the oracle's quantize + double_quant of that job (the sum of job i
-    runs inside job i+1's launch and its groups inside job i+2's, the last two
-    in the tail launches).  A second call on the same workspace gives the same
-    bits, and the scratch of every job is ready for the next call."""
+    mu equal the oracle's quantize + double_quant of that job (the quantize
+    launches back to back, then the sums and groups of all jobs in the tail
+    launches).  A second call on the same workspace gives the same bits, and
+    the scratch of every job is ready for the next call."""
     shapes = [BATCH_SHAPES[k % len(BATCH_SHAPES)] for k in range(njobs)]
     jobs, host = [], []
     for k, (numel, dtype, fmt) in enumerate(shapes):
@@ -515,10 +515,10 @@ def test_quantize_dq_batch_with_shared_outputs_runs_in_order():
 
 
 def test_quantize_dq_batch_long_chain_and_shared_input():
-    """A batch of 24 small weights of assorted sizes (a long chain of deferred
-    double quantizations, every phase launch beside a quantize), two of them
-    quantizing the same input tensor (read-only overlap keeps the early-start
-    schedule): every job equals the oracle."""
+    """A batch of 24 small weights of assorted sizes (a long quantize chain,
+    then one tail launch pair whose CTA ranges cover jobs of very different
+    sizes), two of them quantizing the same input tensor (read-only overlap
+    keeps the early-start schedule): every job equals the oracle."""
     rng = np.random.default_rng(140)
     jobs, host = [], []
     shared = None
@@ -547,3 +547,43 @@ def test_quantize_dq_batch_long_chain_and_shared_input():
         assert np.float32(mu[0]).view(np.uint32) == np.float32(mu_ref).view(np.uint32), f"job {k}: mu"
         assert np.array_equal(b.view(np.uint32), b_ref.view(np.uint32)), f"job {k}: dq scale"
         assert np.array_equal(q, q_ref), f"job {k}: dq codes"
+
+
+@pytest.mark.gpu
+def test_quantize_dq_batch_spanning_several_tail_launches():
+    """131 weights, from one element to a few groups of constants: the double
+    quantization takes two tail launch pairs (128 jobs per launch), and jobs
+    of a single CTA sit next to jobs of several.  Every job equals the oracle,
+    also after a second call on the same workspace."""
+    rng = np.random.default_rng(141)
+    jobs, host = [], []
+    for k in range(131):
+        numel = [1, 63, 64, 65][k] if k < 4 else int(rng.integers(1, 9)) * 16384 + int(rng.integers(0, 130))
+        w = synthetic.normal_f32(numel, float(rng.uniform(0.005, 0.05)), 300 + k)
+        nb = (numel + 63) // 64
+        host.append(w)
+        jobs.append((torch.from_numpy(w).cuda(), torch.empty((numel + 1) // 2, dtype=torch.uint8, device="cuda"),
+                     torch.empty(nb, device="cuda"), torch.empty(nb, dtype=torch.int8, device="cuda"),
+                     torch.empty((nb + 255) // 256, device="cuda"), torch.empty(1, device="cuda"), "int8"))
+    refs = []
+    for w in host:
+        c_ref, a_ref = codec.quantize(w)
+        refs.append((c_ref, a_ref) + tuple(codec.double_quant(a_ref)))
+    ws = api.alloc_workspace(api.workspace_bytes(api.OP_QUANTIZE_DQ_BATCH, len(jobs)))
+    for call in range(2):
+        for j in jobs:
+            for t in j[1:6]:
+                t.fill_(0)
+        api.nf4_quantize_dq_batch(jobs, ws=ws)
+        torch.cuda.synchronize()
+        assert api.device_status(ws) == 0
+        for k, (ref, j) in enumerate(zip(refs, jobs)):
+            codes, absmax, q, b, mu = [t.cpu().numpy() for t in j[1:6]]
+            c_ref, a_ref, q_ref, b_ref, mu_ref = ref
+            assert np.array_equal(codes, c_ref), f"call {call}, job {k}: codes"
+            assert np.array_equal(absmax.view(np.uint32), a_ref.view(np.uint32)), f"call {call}, job {k}: absmax"
+            assert np.float32(mu[0]).view(np.uint32) == np.float32(mu_ref).view(np.uint32), f"call {call}, job {k}: mu"
+            assert np.array_equal(b.view(np.uint32), np.asarray(b_ref, np.float32).view(np.uint32)), \
+                f"call {call}, job {k}: scales"
+            assert np.array_equal(q, np.asarray(q_ref, np.int8)), f"call {call}, job {k}: qabs"
+            assert _scratch_at_rest(ws[256 * k:256 * (k + 1)])
