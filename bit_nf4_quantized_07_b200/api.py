@@ -233,12 +233,25 @@ def nf4_quantize_dq_batch(jobs, ws=None):
     for i, (W, codes, absmax, qabs, dq_scale, dq_mean, fmt) in enumerate(jobs):
         if W.dtype not in _DTYPES:
             raise ValueError(f"unsupported weight dtype {W.dtype}")
-        _need_cuda(W, codes, absmax, qabs, dq_scale, dq_mean)
+        if fmt not in DQ_FORMATS:
+            raise ValueError(f"job {i}: unknown double-quantization format {fmt!r}")
         n = W.numel()
         nb = (n + 63) // 64
-        if (codes.numel() < (n + 1) // 2 or absmax.numel() < nb or qabs.numel() < nb
-                or dq_scale.numel() < (nb + 255) // 256 or dq_mean.numel() < 1):
-            raise ValueError(f"job {i}: an output is too small")
+        # the library writes through raw pointers: check dtypes, sizes and layout here
+        for name, t, dts, need in (("codes", codes, (torch.uint8,), (n + 1) // 2),
+                                   ("absmax", absmax, (torch.float32,), nb),
+                                   ("qabs", qabs, (torch.int8, torch.uint8), nb),
+                                   ("dq_scale", dq_scale, (torch.float32,), (nb + 255) // 256),
+                                   ("dq_mean", dq_mean, (torch.float32,), 1)):
+            if t.dtype not in dts:
+                raise ValueError(f"job {i}: {name} must be {' or '.join(map(str, dts))}, got {t.dtype}")
+            if t.numel() < need:
+                raise ValueError(f"job {i}: {name} holds {t.numel()} elements, needs {need}")
+            if not t.is_contiguous():
+                raise ValueError(f"job {i}: {name} must be contiguous")
+            if t.device != W.device:
+                raise ValueError(f"job {i}: {name} is on {t.device}, W on {W.device}")
+        _need_cuda(W, codes, absmax, qabs, dq_scale, dq_mean)
         arr[i] = CQuantJob(_p(W), n, _DTYPES[W.dtype], DQ_FORMATS[fmt], _p(codes), _p(absmax), _p(qabs),
                            _p(dq_scale), _p(dq_mean))
     if ws is None:

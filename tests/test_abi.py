@@ -143,6 +143,30 @@ def test_quantize_dq_batch_argument_errors(L):
     assert api.workspace_bytes(api.OP_QUANTIZE_DQ_BATCH, 0) == 0
 
 
+def test_quantize_dq_batch_wrapper_checks_outputs():
+    """The Python wrapper rejects outputs of the wrong dtype, size or layout
+    before the C call (CPU tensors: the checks come before the device check)."""
+    import torch
+    n = 4096
+    nb = n // 64
+
+    def job(**bad):
+        t = dict(W=torch.zeros(n), codes=torch.zeros(n // 2, dtype=torch.uint8), absmax=torch.zeros(nb),
+                 qabs=torch.zeros(nb, dtype=torch.int8), dq_scale=torch.zeros(1), dq_mean=torch.zeros(1), fmt="int8")
+        t.update(bad)
+        return (t["W"], t["codes"], t["absmax"], t["qabs"], t["dq_scale"], t["dq_mean"], t["fmt"])
+    for bad, msg in ((dict(absmax=torch.zeros(nb, dtype=torch.float16)), "absmax must be"),
+                     (dict(codes=torch.zeros(n // 2 - 1, dtype=torch.uint8)), "codes holds"),
+                     (dict(qabs=torch.zeros(nb, dtype=torch.int16)), "qabs must be"),
+                     (dict(dq_scale=torch.zeros(2, 2)[:, 0]), "dq_scale must be contiguous"),
+                     (dict(dq_mean=torch.zeros(0)), "dq_mean holds"),
+                     (dict(fmt="int4"), "unknown double-quantization format")):
+        with pytest.raises(ValueError, match=msg):
+            api.nf4_quantize_dq_batch([job(**bad), job()])
+    with pytest.raises(ValueError, match="CUDA"):  # well-formed CPU tensors stop at the device check
+        api.nf4_quantize_dq_batch([job()])
+
+
 def test_dequant_argument_errors(L):
     out = A16
     assert L.nf4_dequant(None, out, None) == 1
