@@ -551,16 +551,15 @@ __device__ __forceinline__ uint64_t dqf_timer_ns() {
 }
 
 // ===========================================================================
-// Deferred double quantization (the batch entry point).  A quantize kernel of
-// job i can also carry, before its own chunks, two pieces of the double
-// quantization of earlier jobs whose block constants are complete because
-// their quantize has finished:
+// Deferred double quantization (the batch entry point, when the jobs' buffers
+// overlap).  A phase launch before the quantize of job i carries two pieces of
+// the double quantization of earlier jobs whose block constants are complete
+// because their quantize has finished:
 //  * the exact sum of job i-1's constants into that job's scratch bank (the
 //    last CTA to arrive advances the generation, as K2 does), and
 //  * the group quantization of job i-2, with mu formed from its bank (as K3).
-// Every kernel still waits for the one before it, so nothing runs concurrently
-// with anything it depends on; the double quantization's latency simply hides
-// behind the next weight's stream.
+// Every kernel waits for the one before it, so nothing runs concurrently with
+// anything it depends on.
 // ===========================================================================
 struct DqPhases {
     const float *s_absmax;  // sum phase: null for none
