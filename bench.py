@@ -464,18 +464,11 @@ def measure_layer(api, dev, cfg, nsets=2, reps=4):
 # ---------------------------------------------------------------------------
 def run_ours(args):
     import torch
-    import torch.distributed as dist
 
     from bit_nf4_quantized_07_b200 import api, dp, synthetic
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    rank, world, local = dp.init_from_env("cuda", timeout_s=120.0)
     cfg = _workload(args.workload)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
@@ -592,21 +585,14 @@ def run_ours(args):
         # codec + forward + backward, the data-parallel all-reduce of dA/dB
         # (N > 1), then the optimizer
         if graphs is not None:
-            graphs[i % NSETS][0].replay()
+            dp.train_step(graphs[i % NSETS][0].replay, graphs[i % NSETS][1].replay, dA, dB, world)
         else:
-            step_body(i)
-        if world > 1:
-            dp.allreduce_adapter_grads(dA, dB)
-        if graphs is not None:
-            graphs[i % NSETS][1].replay()
-        else:
-            optim_body(i)
+            dp.train_step(lambda: step_body(i), lambda: optim_body(i), dA, dB, world)
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    dp.barrier(world)
     torch.cuda.synchronize()
 
     start, stop = ev(), ev()
@@ -618,8 +604,7 @@ def run_ours(args):
         stop.record(stream)
         torch.cuda.synchronize()
     launches = api.launch_count() - launches0 if graphs is None else launches_per_step * args.steps
-    if world > 1:
-        dist.barrier()
+    dp.barrier(world)
     torch.cuda.synchronize()
     elapsed_ms = start.elapsed_time(stop)
     if world > 1:
@@ -672,8 +657,7 @@ def run_ours(args):
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    dp.barrier(world)
     e0, e1 = ev(), ev()
     e0.record(stream)
     for _ in range(e2e_steps):
@@ -739,9 +723,7 @@ def run_ours(args):
         step_s, info = oracle_sample(cfg)
         out["cpu_baseline"] = {"value": flops / step_s / 1e12, "unit": "TFLOP/s", "cores": info["cores"],
                                "kind": "oracle", "sample": info["sample"]}
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    dp.finish(world)
     if rank == 0:
         print(json.dumps(out))
 

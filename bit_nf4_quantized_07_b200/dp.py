@@ -10,7 +10,9 @@ per rank (it belongs to that rank's tokens) and W0 has no gradient.
 torch.distributed carries the collective (NCCL on GPUs, gloo on CPU); the
 helpers work with either backend.
 """
-from typing import Tuple
+import datetime
+import os
+from typing import Callable, Tuple
 
 import torch
 import torch.distributed as dist
@@ -34,3 +36,47 @@ def max_over_ranks(value: float, device=None, group=None) -> float:
     t = torch.tensor([float(value)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
     return float(t.item())
+
+
+def init_from_env(device_type: str = "cuda", timeout_s: float = 120.0) -> Tuple[int, int, int]:
+    """(rank, world, local_rank) from the launcher's environment (RANK,
+    WORLD_SIZE, LOCAL_RANK; MASTER_ADDR and MASTER_PORT for the rendezvous).
+    With more than one rank this joins the default process group: NCCL bound
+    to this rank's GPU for CUDA devices, gloo otherwise.  A short timeout
+    turns a rank that never arrives into an error on the others."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        timeout = datetime.timedelta(seconds=timeout_s)
+        if device_type == "cuda":
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
+    return rank, world, local
+
+
+def train_step(backward: Callable[[], None], update: Callable[[], None], dA: torch.Tensor, dB: torch.Tensor,
+               world: int, group=None) -> None:
+    """One data-parallel training step, the same on every rank: this rank's
+    forward and backward over its own tokens (`backward`, which leaves the
+    adapter gradients in dA and dB), their sum over the ranks, then the
+    optimizer update (`update`), which every rank applies to identical
+    gradients, so the replicas of A and B stay identical."""
+    backward()
+    if world > 1:
+        allreduce_adapter_grads(dA, dB, group=group)
+    update()
+
+
+def barrier(world: int) -> None:
+    """Meet every rank (nothing with one rank)."""
+    if world > 1:
+        dist.barrier()
+
+
+def finish(world: int) -> None:
+    """Meet every rank, then leave the process group (nothing with one rank)."""
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
