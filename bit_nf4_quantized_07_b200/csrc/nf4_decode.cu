@@ -203,7 +203,7 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
     // restored block constants ahat of the epoch's tiles over this CTA's K
     // range (doubleDequant, first step): a thread takes 4 consecutive blocks of
     // one weight row, loads their codes and scales, then restores them
-    const float mu = dq ? __ldg(p.dq_mean) : 0.f;
+    float mu = 0.f;  // the mean of the constants: read after the dependency wait (below)
     const int nq = (nkb + 3) >> 2;
     auto stage_ah = [&](int e) {
         const int Ee = e + 1 < nep ? E : El;
@@ -235,6 +235,7 @@ nf4_decode_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const DfPara
     //         this thread waits for -- so all of them are in flight together -------------
     pdl_wait();  // the weight, X, A, B and the workspace may be written by the previous kernel
     pdl_trigger();
+    if (dq) mu = __ldg(p.dq_mean);
     if (blockIdx.x == 0 && tid == 0) *p.status = QLN_OK;
 #pragma unroll 1
     for (int k = 0; k < RS; ++k) issue_next();

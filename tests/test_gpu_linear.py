@@ -103,6 +103,35 @@ def test_decode_shaped_forward(cfg, dq):
     _compare("Y", got["Y"], Y)
 
 
+def test_decode_forward_right_behind_the_quantize_sees_its_outputs():
+    """The decode forward enqueued directly behind nf4_quantize_dq on the same
+    stream, with no synchronisation between, reads the fresh codes, scales
+    and mean: every read of the weight comes after its dependency wait.  The
+    output buffers hold wrong values (a mean of 123) before each quantize; the
+    result must equal that of a forward run after the stream has drained, and
+    the oracle's."""
+    cfg = synthetic.DECODE[4]
+    w, X, A, B, dY = workload(cfg)
+    Wd = torch.from_numpy(w).cuda()
+    wq = api.quantize_weight(Wd)
+    Xd, Ad, Bd = bf16_to_dev(X), bf16_to_dev(A), bf16_to_dev(B)
+    ws = api.alloc_workspace(api.workspace_bytes(api.OP_LINEAR_FWD, cfg.dout, cfg.din, cfg.n, cfg.r))
+    torch.cuda.synchronize()
+    Yref, Uref = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s, ws=ws)
+    torch.cuda.synchronize()
+    for _ in range(4):
+        wq.dq_mean.fill_(123.0)
+        wq.dq_scale.fill_(7.0)
+        wq.qabs.fill_(-100)
+        api.nf4_quantize_dq(Wd, wq.codes, wq.absmax, wq.qabs, wq.dq_scale, wq.dq_mean)
+        Y, U = api.qlora_linear_fwd(wq, Xd, Ad, Bd, cfg.s, ws=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, Yref) and torch.equal(U, Uref)
+    assert api.device_status(ws) == 0
+    Yo, _ = forward_ref(OracleWeight(w), X, A, B, cfg.s)
+    _compare("Y", f64(dev_bf16_bits(Y)), Yo)
+
+
 def test_decode_forward_repeats_and_replays_bit_identically():
     """The one-launch decode forward folds its split-K partials in an order
     fixed by the shape: back-to-back calls on one workspace, a call after a
