@@ -550,6 +550,39 @@ def test_quantize_dq_batch_long_chain_and_shared_input():
 
 
 @pytest.mark.gpu
+def test_quantize_dq_batch_chained_through_an_earlier_output():
+    """Three jobs where the third quantizes the first one's block constants
+    (its weights are job 0's absmax buffer): the buffers overlap, so the
+    ordered schedule runs, and the result is that of separate calls in order."""
+    n0, n1 = 256 * 1024, 64 * 4096 + 40
+    w0 = synthetic.normal_f32(n0, 0.02, 160)
+    w1 = synthetic.normal_f32(n1, 0.03, 161)
+
+    def outs(numel):
+        nb = (numel + 63) // 64
+        return (torch.empty((numel + 1) // 2, dtype=torch.uint8, device="cuda"), torch.empty(nb, device="cuda"),
+                torch.empty(nb, dtype=torch.int8, device="cuda"), torch.empty((nb + 255) // 256, device="cuda"),
+                torch.empty(1, device="cuda"))
+    o0, o1 = outs(n0), outs(n1)
+    o2 = outs(n0 // 64)
+    jobs = [(torch.from_numpy(w0).cuda(), *o0, "int8"), (torch.from_numpy(w1).cuda(), *o1, "int8"),
+            (o0[1], *o2, "int8")]
+    api.nf4_quantize_dq_batch(jobs)
+    torch.cuda.synchronize()
+    c0, a0 = codec.quantize(w0)
+    c1, a1 = codec.quantize(w1)
+    c2, a2 = codec.quantize(np.asarray(a0, np.float32))
+    for k, (o, (c_ref, a_ref)) in enumerate(zip((o0, o1, o2), ((c0, a0), (c1, a1), (c2, a2)))):
+        codes, absmax, q, b, mu = [t.cpu().numpy() for t in o]
+        q_ref, b_ref, mu_ref = codec.double_quant(a_ref)
+        assert np.array_equal(codes, c_ref), f"job {k}: codes"
+        assert np.array_equal(absmax.view(np.uint32), np.asarray(a_ref, np.float32).view(np.uint32)), f"job {k}: absmax"
+        assert np.float32(mu[0]).view(np.uint32) == np.float32(mu_ref).view(np.uint32), f"job {k}: mu"
+        assert np.array_equal(b.view(np.uint32), np.asarray(b_ref, np.float32).view(np.uint32)), f"job {k}: scales"
+        assert np.array_equal(q, np.asarray(q_ref, np.int8)), f"job {k}: qabs"
+
+
+@pytest.mark.gpu
 def test_quantize_dq_batch_spanning_several_tail_launches():
     """131 weights, from one element to a few groups of constants: the double
     quantization takes two tail launch pairs (128 jobs per launch), and jobs
