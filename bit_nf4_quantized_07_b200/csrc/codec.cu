@@ -550,108 +550,6 @@ __device__ __forceinline__ uint64_t dqf_timer_ns() {
     return t;
 }
 
-// ===========================================================================
-// Deferred double quantization (the batch entry point, when the jobs' buffers
-// overlap).  A phase launch before the quantize of job i carries two pieces of
-// the double quantization of earlier jobs whose block constants are complete
-// because their quantize has finished:
-//  * the exact sum of job i-1's constants into that job's scratch bank (the
-//    last CTA to arrive advances the generation, as K2 does), and
-//  * the group quantization of job i-2, with mu formed from its bank (as K3).
-// Every kernel waits for the one before it, so nothing runs concurrently with
-// anything it depends on.
-// ===========================================================================
-struct DqPhases {
-    const float *s_absmax;  // sum phase: null for none
-    int64_t s_nb;
-    unsigned char *s_ws;
-    const float *g_absmax;  // group phase: null for none
-    int64_t g_nb;
-    unsigned char *g_ws;
-    int8_t *g_qabs;
-    float *g_scale;
-    float *g_mu;
-    int g_e4m3;
-    int *status;  // cleared by CTA 0 when not null
-};
-
-// Both phases with the whole grid (any block size that is a multiple of 32);
-// every thread of every CTA calls it.  CTA b takes a contiguous share of the
-// constants (sum) and of the groups, staged through `stage` (kPhStage floats
-// of shared memory) by cp.async, so a CTA of few threads still has its whole
-// share in flight at once.  slim: kXLimbs words of shared memory.
-constexpr int kPhStage = 4096;  // floats per staging round (16 KB)
-__device__ __noinline__ void dq_run_phases(const DqPhases &ph, unsigned long long *slim, float *mu_s,
-                                           unsigned *gen_s, float *stage) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5, nt = blockDim.x;
-    if (ph.status && blockIdx.x == 0 && tid == 0) *ph.status = QLN_OK;
-    // copy constants [j0, j1) of `a` (j1 - j0 <= kPhStage, j0 a multiple of 4) into stage,
-    // zero-filled past nb; every thread waits for its copies, then the CTA meets
-    auto stage_in = [&](const float *a, int64_t j0, int64_t j1, int64_t nb) {
-        for (int64_t c = tid; 4 * c < j1 - j0; c += nt) {
-            const int64_t j = j0 + 4 * c;
-            const int64_t left = nb - j;
-            cp_async16_zfill(stage + 4 * c, a + (left > 0 ? j : 0), left >= 4 ? 16 : (left > 0 ? (int)left * 4 : 0));
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
-        __syncthreads();
-    };
-    const DqScratch gs = dq_scratch(ph.g_ws, false);
-    if (ph.g_absmax && warp == 0) {  // mu of the earlier weight: its sum advanced the generation
-        const float mu = xsum_mean_warp(gs.bank[(__ldcg(gs.gen) + 1) & 1], (uint32_t)ph.g_nb);
-        if (lane == 0) {
-            *mu_s = mu;
-            if (blockIdx.x == 0) *ph.g_mu = mu;
-        }
-    }
-    if (ph.s_absmax) {  // the exact sum of the later weight's constants
-        const DqScratch ss = dq_scratch(ph.s_ws, false);
-        if (tid < kXLimbs) slim[tid] = 0ull;
-        const unsigned g0 = dq_read_gen(ss, gen_s);  // includes a __syncthreads
-        const int64_t nb = ph.s_nb;
-        const int64_t per = ((nb + gridDim.x - 1) / gridDim.x + 3) & ~(int64_t)3;
-        const int64_t lo = (int64_t)blockIdx.x * per < nb ? (int64_t)blockIdx.x * per : nb;
-        const int64_t hi = lo + per < nb ? lo + per : nb;
-        XRun x;
-        for (int64_t r0 = lo; r0 < hi; r0 += kPhStage) {
-            const int64_t r1 = r0 + kPhStage < hi ? r0 + kPhStage : hi;
-            stage_in(ph.s_absmax, r0, r1, nb);
-            for (int64_t k = tid; k < r1 - r0; k += nt) xsum_add(x, stage[k], slim);
-            __syncthreads();  // the stage is read before the next round refills it
-        }
-        xsum_flush_warp(x, slim);
-        __syncthreads();
-        if (tid < kXLimbs && slim[tid] != 0ull) atomicAdd(&ss.bank[g0 & 1][tid], slim[tid]);
-        __syncthreads();
-        if (tid == 0) dq_arrive(ss, g0, (int)gridDim.x);
-    }
-    __syncthreads();  // mu is in shared memory
-    if (ph.g_absmax) {
-        const float mu = *mu_s;
-        const int64_t nb = ph.g_nb;
-        const int64_t ng = (nb + kDqGroup - 1) / kDqGroup;
-        const int64_t per = (ng + gridDim.x - 1) / gridDim.x;
-        const int64_t glo = (int64_t)blockIdx.x * per < ng ? (int64_t)blockIdx.x * per : ng;
-        const int64_t ghi = glo + per < ng ? glo + per : ng;
-        constexpr int kGroupsPerRound = kPhStage / kDqGroup;
-        for (int64_t g0 = glo; g0 < ghi; g0 += kGroupsPerRound) {
-            const int64_t g1 = g0 + kGroupsPerRound < ghi ? g0 + kGroupsPerRound : ghi;
-            const int64_t j1 = g1 * kDqGroup < nb ? g1 * kDqGroup : nb;
-            stage_in(ph.g_absmax, g0 * kDqGroup, j1, nb);
-            for (int64_t g = g0 + warp; g < g1; g += nw) {
-                const float *src = stage + (g - g0) * kDqGroup + 8 * lane;
-                const float4 u = *reinterpret_cast<const float4 *>(src);
-                const float4 v = *reinterpret_cast<const float4 *>(src + 4);
-                const float e[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};  // entries past nb are not used
-                dq_quantize_group(e, g * kDqGroup + 8 * lane, nb, mu, ph.g_e4m3 != 0, lane, g, ph.g_qabs,
-                                  ph.g_scale);
-            }
-            __syncthreads();  // the stage is read before the next round refills it
-        }
-    }
-}
-
 constexpr int kQzWarps = 24;       // two CTAs of 24 warps per SM
 constexpr int kQzCtasPerSm = 2;
 constexpr int kQzStages = 3;       // chunks per warp ring
@@ -1101,36 +999,6 @@ cudaError_t launch_nf4_quantize_dq(const void *W, int dtype, int64_t numel, uint
 
 static_assert(kDqScratchBytes == kDqBatchScratchBytes, "one DQ scratch per batch job");
 
-// The deferred double quantization of a batch whose buffers overlap, one
-// small CTA per SM: 128 threads of at most 32 registers fit beside the two
-// quantize CTAs of an SM (the registers those leave free), so it runs
-// alongside the quantize kernels.  It waits for its predecessor before
-// touching memory.
-constexpr int kPhThreads = 128;
-__global__ void __launch_bounds__(kPhThreads, 16) dq_phase_kernel(DqPhases ph) {
-    extern __shared__ __align__(16) float ph_stage[];  // kPhStage floats
-    __shared__ unsigned long long slim[kXLimbs];
-    __shared__ float mu_s;
-    __shared__ unsigned gen_s;
-    pdl_wait();
-    pdl_trigger();
-    dq_run_phases(ph, slim, &mu_s, &gen_s, ph_stage);
-}
-constexpr size_t kPhSmem = kPhStage * sizeof(float);
-
-// One phase launch (the kernel asks for the largest shared-memory carveout so
-// that it can sit beside two quantize CTAs on an SM).
-static cudaError_t launch_phase(int grid, const DqPhases &ph, cudaStream_t st) {
-    static std::atomic<int> configured{0};
-    if (!configured.load(std::memory_order_relaxed)) {
-        cudaError_t e = cudaFuncSetAttribute(dq_phase_kernel,
-                                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        if (e != cudaSuccess) return e;
-        configured.store(1, std::memory_order_relaxed);
-    }
-    return launch_pdl(dq_phase_kernel, dim3(grid), dim3(kPhThreads), kPhSmem, st, ph);
-}
-
 namespace {
 struct ByteRange {
     uintptr_t lo, hi;  // [lo, hi)
@@ -1275,61 +1143,28 @@ static cudaError_t launch_dq_tails(const QuantJob *jobs, int njobs, unsigned cha
 // the quantize kernels instead took the 6.48 B-parameter sweep from 5.35 ms
 // to 6.6 ms: their work, on one small CTA per SM, ran longer than the
 // quantize of the smaller weights it had to finish within.
-// Otherwise: quantize(0); then for i >= 1 the phase launch (sum of weight
-// i-1, groups of weight i-2) followed by quantize(i); then the two tail phase
-// launches (sum of n-1 and groups of n-2; groups of n-1).  Every launch waits
-// at its start for the one before it, so each phase reads only completed
-// constants and sums.  Job i's scratch is ws + 256 i; the first sum launch
-// clears the status word at ws + 0.
+// Otherwise (a job reads or writes another job's outputs) each job's
+// quantize is followed by its own sum and group launches, every launch
+// waiting at its start for the one before it: the order of separate calls.
+// Job i's scratch is ws + 256 i; job 0's sum launch writes QLN_OK to the
+// status word at ws + 0.
 cudaError_t launch_nf4_quantize_dq_batch(const QuantJob *jobs, int njobs, void *ws, cudaStream_t st, int num_sms) {
     unsigned char *w = static_cast<unsigned char *>(ws);
-    auto scratch = [&](int i) { return w + kDqScratchBytes * (size_t)i; };
-    auto nb_of = [&](int i) { return (jobs[i].numel + 63) / 64; };
-    bool status_cleared = false;
-    auto phases = [&](int s_job, int g_job) {  // -1: none
-        DqPhases ph{};
-        if (s_job >= 0) {
-            ph.s_absmax = jobs[s_job].absmax;
-            ph.s_nb = nb_of(s_job);
-            ph.s_ws = scratch(s_job);
-        }
-        if (g_job >= 0) {
-            ph.g_absmax = jobs[g_job].absmax;
-            ph.g_nb = nb_of(g_job);
-            ph.g_ws = scratch(g_job);
-            ph.g_qabs = jobs[g_job].qabs;
-            ph.g_scale = jobs[g_job].scale;
-            ph.g_mu = jobs[g_job].mu;
-            ph.g_e4m3 = jobs[g_job].e4m3 ? 1 : 0;
-        }
-        if (!status_cleared) {
-            ph.status = reinterpret_cast<int *>(w);
-            status_cleared = true;
-        }
-        return ph;
-    };
-    const bool disjoint = batch_disjoint(jobs, njobs, ws);
-    cudaError_t e = launch_quantize_dtype<false>(jobs[0].W, jobs[0].dtype, jobs[0].numel, jobs[0].codes,
-                                                 jobs[0].absmax, st, num_sms);
-    if (e != cudaSuccess) return e;
-    if (disjoint) {  // the quantize chain alone, then the double quantization of all jobs
-        for (int i = 1; i < njobs; ++i) {
+    cudaError_t e = cudaSuccess;
+    if (batch_disjoint(jobs, njobs, ws)) {  // the quantize chain alone, then the double quantization of all jobs
+        for (int i = 0; i < njobs && e == cudaSuccess; ++i) {
             const QuantJob &q = jobs[i];
-            e = launch_quantize_dtype<true>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
-            if (e != cudaSuccess) return e;
+            e = i == 0 ? launch_quantize_dtype<false>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms)
+                       : launch_quantize_dtype<true>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
         }
-        return launch_dq_tails(jobs, njobs, w, st);
+        return e == cudaSuccess ? launch_dq_tails(jobs, njobs, w, st) : e;
     }
-    for (int i = 1; i < njobs; ++i) {
+    for (int i = 0; i < njobs && e == cudaSuccess; ++i) {  // job by job, as separate calls in order
         const QuantJob &q = jobs[i];
-        e = launch_phase(num_sms, phases(i - 1, i - 2), st);
-        if (e == cudaSuccess) e = launch_quantize_dtype<false>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
-        if (e != cudaSuccess) return e;
+        e = launch_quantize_dtype<false>(q.W, q.dtype, q.numel, q.codes, q.absmax, st, num_sms);
+        if (e == cudaSuccess) e = launch_dq_tails(&q, 1, w + kDqScratchBytes * (size_t)i, st);
     }
-    const int tail_grid = 4 * num_sms;
-    e = launch_phase(tail_grid, phases(njobs - 1, njobs - 2), st);
-    if (e != cudaSuccess) return e;
-    return launch_phase(tail_grid, phases(-1, njobs - 1), st);
+    return e;
 }
 
 // ===========================================================================

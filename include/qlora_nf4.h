@@ -244,11 +244,11 @@ typedef struct {
  * run back to back (each one starts while the one before it drains) and the
  * double quantization of all jobs follows in two launches per 128 jobs (the
  * exact sums, then the groups), so that its latency is paid once per call
- * rather than once per weight.  Otherwise the double quantization of weight i
- * runs in small launches between the later quantize launches (its sum before
- * weight i+1's, its groups before weight i+2's).  Either way every launch
- * reads only what earlier launches completed, so the jobs' buffers may be
- * laid out in any way that separate nf4_quantize_dq calls allow.
+ * rather than once per weight.  Otherwise each weight's quantize is followed
+ * by its own two double-quantization launches before the next weight's, as
+ * separate calls would run.  Either way every launch reads only what earlier
+ * launches completed, so the jobs' buffers may be laid out in any way that
+ * separate nf4_quantize_dq calls allow.
  *   ws / ws_bytes: qln_workspace_bytes(QLN_OP_QUANTIZE_DQ_BATCH, njobs, 0, 0,
  *   0) = 256 * njobs bytes, 256-byte aligned, zeroed once before the first
  *   call and then left to the library (job i uses bytes 256 i .. 256 i + 255
